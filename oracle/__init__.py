@@ -1,0 +1,34 @@
+"""CPU reference (the oracle) for paged attention over a block-table KV cache.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product package imports, calls or
+links anything here; only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may use it.
+
+It is the plain definition, written for a reader to check by eye against the
+source pages, in float64 with numpy:
+
+* ``block_pool``  - the Block / BlockTable bookkeeping of the page
+  "Nano-vLLM-Ascend: lightweight LLM inference framework for Ascend NPU",
+  section 2.1 (PageAttention memory management): fixed 16-token blocks, a
+  logical-to-physical block map per sequence, a reference count per block;
+  and the free-list allocator role of BlockAllocator from the page "Ascend NPU
+  LLM inference optimisation: the vLLM-Ascend approach", section 2.1.
+* ``kv_write``    - writing new tokens' K/V into their slots, as bytes.
+* ``attention``   - gather through the block table, then softmax(q K^T * scale) V
+  per query head (Nano-vLLM-Ascend page, section 2.2.1, the unfused attention;
+  section 4.2 names the 1/sqrt(d) scale), with the softmax done in fp64 (the
+  vLLM-Ascend page, section 3.1, moves softmax out of fp16 for accuracy); causal
+  chunked prefill over the paged context (vllm-ascend page, section 1.1, PCP).
+* ``brute``       - a scalar pure-Python twin of ``attention`` for tiny cases.
+
+Parity pins (tests/test_oracle_pins.py): the pages' worked block arithmetic
+(tests/golden/), closed forms, torch's float64 scaled_dot_product_attention on
+dense inputs, the scalar twin, and invariants (block permutation, prefix
+sharing, prefill row i == decode of the first prefix+i+1 tokens).  No function
+here is "parity unpinned".
+"""
+
+from . import attention, block_pool, brute, kv_write  # noqa: F401
+from .attention import decode_attention, gather_kv, prefill_attention, split_partials  # noqa: F401
+from .block_pool import OraclePool, replay  # noqa: F401
+from .kv_write import write_kv  # noqa: F401

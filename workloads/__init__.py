@@ -1,0 +1,13 @@
+"""Seeded synthetic inputs shared by the oracle tests, the GPU tests and the bench.
+
+This package draws random numbers and lays out workload *structure* (how many
+sequences, their lengths, which sequences share a prefix, the order in which
+the block pool hands out physical blocks).  It holds none of the method's
+arithmetic: no slot or block-index computation, no attention maths.  Both the
+CPU oracle and the CUDA path start from what it returns and derive everything
+else on their own.
+"""
+
+from .synth import CONFIGS, Workload, make_workload, fill_cache_blocks, ops_for
+
+__all__ = ["CONFIGS", "Workload", "make_workload", "fill_cache_blocks", "ops_for"]
