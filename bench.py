@@ -1,0 +1,393 @@
+#!/usr/bin/env python
+"""Benchmark: paged decode KV GB/s (and decode tokens/s) at batch 128, Qwen3-0.6B-shaped heads.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = the whole decode hot path over one batch: pa_write_kv of each
+sequence's new token into its slot, then pa_decode (split kernel + split-K
+reduce kernel) over every sequence's paged context.  Inputs are resident in
+HBM; the KV working set (~295 MB) is larger than the 126 MB L2, so no flush is
+needed between steps.  Timed with CUDA events on the launching stream,
+bracketed by barrier + synchronize, max over ranks.  N > 1 runs independent
+data-parallel replicas (each rank its own batch of sequences and its own
+pool; no collective on the data path), so the scaling is weak.
+
+`--impl reference` times the CPU oracle (oracle/) on the host cores on
+bounded samples of the same workload; it is the deliberately slow baseline.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode KV GB/s (% of HBM peak) and decode tokens/s at batch 128"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+
+WORKLOAD_TEXT = {
+    "qwen_decode": "Qwen3-0.6B-shaped decode: batch 128, 16 q / 8 kv heads (GQA 2), head_dim 128, bf16, block_size 16, "
+                   "context_lens uniform[100,1024], blocks shuffled over a pool of total context + 10% free",
+    "llama70b_long": "Llama-2-70B-shaped long decode: batch 64, 64 q / 8 kv heads (GQA 8), head_dim 128, bf16, "
+                     "block_size 16, context_lens uniform[4096,8192]",
+    "prefix_sweep": "prefix-shared decode: batch 256 = 8 groups x 32 sharing a 2048-token prefix, suffix uniform[0,512], "
+                    "16 q / 8 kv heads, head_dim 128, bf16",
+    "tiny": "tiny decode: 4 seqs, 4/4 heads, head_dim 64, fp16, block_size 16",
+}
+
+# DRAM bytes (read + write) per launch of the decode split kernel from one ncu capture of this workload,
+# valid only for the kernel source it was taken on (sha256 prefix of decode.cu + common.cuh).
+NCU_TRAFFIC = {}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("decode.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "paged_kv_cache_330_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML (read-only) while a region runs."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------------------ helpers
+def kv_bytes(wl) -> int:
+    """Algorithmic bytes of one decode: every context token's K and V row of every KV head, read once."""
+    c = wl.cfg
+    return int(wl.context_lens.astype(np.int64).sum()) * c["num_kv_heads"] * c["head_dim"] * 2 * 2
+
+
+def unique_kv_bytes(wl) -> int:
+    """For shared prefixes, bytes of distinct cache rows read (each shared block counted once)."""
+    c = wl.cfg
+    if c["kind"] != "prefix":
+        return kv_bytes(wl)
+    toks = c["groups"] * c["prefix_len"] + int((wl.context_lens - c["prefix_len"]).sum())
+    return toks * c["num_kv_heads"] * c["head_dim"] * 2 * 2
+
+
+def io_bytes(wl) -> int:
+    """q read + out written + block tables + context lengths, per decode call."""
+    c = wl.cfg
+    qo = wl.batch * c["num_q_heads"] * c["head_dim"] * 2 * 2
+    bt = int(sum(-(-int(L) // c["block_size"]) for L in wl.context_lens)) * 4
+    return qo + bt + wl.batch * 4
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ------------------------------------------------------------------------------------------------ reference arm
+def oracle_step_cpu(wl, n_seqs=None):
+    """One oracle pass (pool replay, byte write, fp64 decode) over the first n_seqs sequences."""
+    import oracle
+    from oracle import attention as oatt
+    import torch
+    pool, rows, lens, slots, _ = oracle.replay(wl.ops, wl.num_blocks, wl.cfg["block_size"], wl.free_order, wl.batch)
+    kc = wl.k_cache0.view(torch.int16).numpy().view(np.uint16).copy()
+    vc = wl.v_cache0.view(torch.int16).numpy().view(np.uint16).copy()
+    oracle.write_kv(wl.k_new.view(torch.int16).numpy().view(np.uint16), wl.v_new.view(torch.int16).numpy().view(np.uint16),
+                    slots, kc, vc)
+    n = wl.batch if n_seqs is None else n_seqs
+    dt = wl.k_cache0.dtype
+    kt = torch.from_numpy(kc.view(np.int16)).view(dt)
+    vt = torch.from_numpy(vc.view(np.int16)).view(dt)
+    return oatt.decode_attention(wl.q[:n], kt, vt, rows[:n], lens[:n], wl.scale)
+
+
+def time_oracle(wl, budget_s: float, n_seqs: int):
+    """Repeat the oracle step on the first n_seqs sequences until budget_s of CPU time; returns (GB/s, desc, threads)."""
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        threads = 1
+    c = wl.cfg
+    bytes_per = int(wl.context_lens[:n_seqs].astype(np.int64).sum()) * c["num_kv_heads"] * c["head_dim"] * 4
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle_step_cpu(wl, n_seqs)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    gbs = bytes_per * reps / el / 1e9
+    desc = (f"oracle (numpy fp64, pool replay + byte write + decode) on the first {n_seqs} of {wl.batch} sequences "
+            f"of {wl.name}, {reps} repetitions in {el:.1f} s; GB/s counts those sequences' KV bytes")
+    return gbs, desc, threads, el / reps
+
+
+def run_reference(args):
+    ws, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    from workloads import make_workload
+    wl = make_workload(args.workload)
+    n = min(wl.batch, args.ref_seqs)
+    step_times = []
+    gbs_all = []
+    desc = threads = None
+    for i in range(args.warmup + args.steps):
+        gbs, desc, threads, per = time_oracle(wl, args.ref_budget, n)
+        if i >= args.warmup:
+            step_times.append(per)
+            gbs_all.append(gbs)
+    value = float(np.mean(gbs_all))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * float(np.mean(step_times)), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT.get(args.workload, args.workload), "sample_seqs": n},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------------ our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_330_b200 as pa
+    from workloads import make_workload
+
+    ws, rank, local = dist_setup()
+    if ws > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = make_workload(args.workload, seed=None if rank == 0 else 1000 * rank + 1)
+    c = wl.cfg
+    _, bt, lens, sm, _ = pa.replay_ops(wl.ops, wl.num_blocks, c["block_size"], wl.free_order, wl.batch)
+    maxL = int(lens.max())
+    B, Hq, Hkv, D = wl.batch, c["num_q_heads"], c["num_kv_heads"], c["head_dim"]
+    sl, msplit, wsb = pa.decode_plan(B, Hq, Hkv, D, maxL, args.num_splits)
+
+    # device-resident inputs
+    kc = wl.k_cache0.to(dev)
+    vc = wl.v_cache0.to(dev)
+    q = wl.q.to(dev)
+    kn, vn = wl.k_new.to(dev), wl.v_new.to(dev)
+    smd = torch.from_numpy(sm).to(dev)
+    btd = torch.from_numpy(bt).to(dev)
+    lensd = torch.from_numpy(lens).to(dev)
+    out = torch.empty_like(q)
+    work = torch.empty(max(wsb, 256), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev_pair=None):
+        pa.write_kv(kn, vn, smd, kc, vc, stream=stream)
+        if ev_pair is not None:
+            ev_pair[0].record(stream)
+        pa.decode(q, kc, vc, btd, lensd, maxL, wl.scale, out=out, workspace=work, num_splits=args.num_splits,
+                  stream=stream)
+        if ev_pair is not None:
+            ev_pair[1].record(stream)
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert pa.device_error() == 0
+
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize(dev)
+        t_start.record(stream)
+        for i in range(K):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+    ms_total = t_start.elapsed_time(t_end)
+    dec_ms = [a.elapsed_time(b) for a, b in evs]
+    ms_step = ms_total / K
+
+    # ---- end to end through the public API: pinned host inputs -> device, step, result -> host
+    pin = lambda t: t.pin_memory()
+    h_q, h_kn, h_vn = pin(wl.q), pin(wl.k_new), pin(wl.v_new)
+    h_sm, h_bt, h_lens = pin(torch.from_numpy(sm)), pin(torch.from_numpy(bt)), pin(torch.from_numpy(lens))
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_kn, h_vn, h_sm, h_bt, h_lens))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        q.copy_(h_q, non_blocking=True)
+        kn.copy_(h_kn, non_blocking=True)
+        vn.copy_(h_vn, non_blocking=True)
+        smd.copy_(h_sm, non_blocking=True)
+        btd.copy_(h_bt, non_blocking=True)
+        lensd.copy_(h_lens, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / K
+    assert pa.device_error() == 0
+
+    # ---- max over ranks, totals
+    kvb = kv_bytes(wl)
+    vals = torch.tensor([ms_step, e2e_ms, float(np.mean(dec_ms))], dtype=torch.float64, device=dev)
+    tot = torch.tensor([float(kvb), float(B)], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
+    ms_step, e2e_ms, dec_avg = vals.tolist()
+    kv_all, seqs_all = tot.tolist()
+    value = kv_all / (ms_step * 1e-3) / 1e9
+    e2e_value = kv_all / (e2e_ms * 1e-3) / 1e9
+
+    peak, peak_kind = measured_hbm_peak()
+    alg = kvb + io_bytes(wl)
+    achieved = alg / (dec_avg * 1e-3) / 1e9
+    tr = NCU_TRAFFIC.get(args.workload)
+    traffic = tr["bytes"] if tr and tr.get("src") == kernel_source_hash() else None
+    launches_per_step = 1 + 1 + (1 if msplit > 1 else 0)
+    if rank == 0:
+        cpu = None
+        if ws == 1 and not args.no_cpu_baseline:
+            gbs, desc, threads, _ = time_oracle(wl, args.ref_budget, min(wl.batch, args.ref_seqs))
+            cpu = {"value": gbs, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
+                   "host_cpus": os.cpu_count()}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": str(c["dtype"]), "data": "synthetic",
+            "config": {"workload": WORKLOAD_TEXT.get(args.workload, args.workload), "global_batch": int(seqs_all),
+                       "parallelism": f"dp{ws} (independent replicas)", "l2": "inputs larger than L2 (no flush)",
+                       "split_len": sl, "max_splits": msplit},
+            "tokens_per_s": seqs_all / (ms_step * 1e-3),
+            "pct_hbm_peak": {"of_measured": value / ws / peak if peak_kind == "measured" else None,
+                             "of_nominal_8000": value / ws / 8000.0},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "roofline": {"bound": "hbm", "kernel": "pa_decode (split + split-K reduce kernels)",
+                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic, "algorithmic_bytes": alg,
+                         "avg_launch_ms": dec_avg},
+            "gpu_launches": launches_per_step * K,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen_decode", choices=sorted(WORKLOAD_TEXT))
+    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--ref-budget", type=float, default=12.0, help="seconds of oracle time per reference sample")
+    ap.add_argument("--ref-seqs", type=int, default=128)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        if args.steps * args.ref_budget > 120:
+            args.ref_budget = max(1.0, 120.0 / max(1, args.steps + args.warmup))
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

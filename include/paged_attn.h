@@ -1,0 +1,226 @@
+/*
+ * paged_attn.h - C ABI of the B200 (sm_100a) paged KV-cache attention library.
+ *
+ * The library implements PagedAttention over a block-table KV cache as the
+ * source pages describe it:
+ *
+ *   [P1] "Nano-vLLM-Ascend: lightweight LLM inference framework for Ascend NPU"
+ *        section 2.1 (PageAttention memory management: 16-token blocks, the
+ *        Block and BlockTable structures, per-block reference counts),
+ *        section 2.2.1 (attention = softmax(q k^T / sqrt(d)) v),
+ *        section 4.2 (the 1/sqrt(d) scale; reference counts checked for leaks).
+ *   [P2] "Ascend NPU LLM inference optimisation: the vLLM-Ascend approach"
+ *        section 2.1 (BlockAllocator over one pool), section 2.2 (PagedAttention
+ *        operator: fill requests into fixed blocks, tile QK^T, softmax and V
+ *        weighting), section 3.1 (256-byte aligned accesses; softmax in fp32),
+ *        section 4 (block sharing for long contexts).
+ *   [P3] "In-depth analysis of vllm-ascend: LLM inference architecture on
+ *        Ascend hardware" section 1.1 / 3.1 (chunked prefill inside one device).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Device pointers are owned by the caller (e.g. PyTorch tensors).  The
+ *   compute calls allocate no device memory and never synchronise the host;
+ *   work is enqueued on `stream` (a cudaStream_t passed as void*, NULL = the
+ *   legacy default stream).
+ * - Every call returns a pa_status.  Arguments are validated on the host
+ *   before anything is launched; a rejected call launches nothing and leaves
+ *   all buffers untouched.  No call aborts or traps.
+ * - Tensors are dense, row-major, in the layouts given per argument.
+ * - Element type: PA_F16 (IEEE half) or PA_BF16 (bfloat16) for q, k, v, caches
+ *   and out.  All softmax statistics and accumulators are fp32.
+ * - KV cache layout (P1 s2.1, blocks stacked into one pool, P2 s2.1):
+ *       cache[num_blocks][block_size][num_kv_heads][head_dim]
+ *   separately for K and V.  Slot s = physical_block * block_size + row.
+ * - block_tables: int32 [batch][max_blocks_per_seq]; entry j of row b is the
+ *   physical block that holds tokens j*block_size .. j*block_size+block_size-1
+ *   of sequence b; entries past ceil(context_lens[b]/block_size) are never read.
+ * - context_lens: int32 [batch], tokens of each sequence INCLUDING any token
+ *   written in this step.
+ * - Supported: head_dim in {64, 128}; block_size in {16, 32, 64, 128, 256};
+ *   num_q_heads a multiple of num_kv_heads with group size G = Hq/Hkv in
+ *   {1, 2, 4, 8, 16}; query head h reads KV head h / G.
+ * - Alignment (P2 s3.1): every tensor pointer must be 16-byte aligned.
+ * - Device-resident indices (block table entries, slots, lengths) are trusted:
+ *   the caller guarantees 0 <= entry < num_blocks, slot < num_blocks*block_size
+ *   and context_lens[b] <= min(max_context_len, max_blocks_per_seq*block_size).
+ *   Kernels that detect a broken device-side invariant record it in a device
+ *   error word (pa_device_error) instead of trapping.
+ */
+#ifndef PAGED_ATTN_H
+#define PAGED_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID = -1,      /* null pointer, negative size, inconsistent shapes */
+  PA_ERR_UNSUPPORTED = -2,  /* head_dim, block_size, group size or dtype outside the supported set */
+  PA_ERR_ALIGN = -3,        /* a tensor pointer is not 16-byte aligned */
+  PA_ERR_WORKSPACE = -4,    /* workspace missing or smaller than required */
+  PA_ERR_CUDA = -5,         /* a CUDA runtime/driver call failed (launch error etc.) */
+  PA_ERR_OOM = -6,          /* block pool has too few free blocks (state unchanged) */
+  PA_ERR_NOT_FOUND = -7,    /* unknown sequence id / sequence already exists */
+  PA_ERR_DEVICE = -8        /* a kernel recorded a broken device-side invariant */
+} pa_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* pa_strerror(int status);
+
+/* Library version as "major.minor.patch" (static string). */
+const char* pa_version(void);
+
+/* ------------------------------------------------------------------------ */
+/* KV write (P1 s2.1 Block layout; P2 s2.2 "fill requests into fixed-size     */
+/* blocks").                                                                  */
+/*                                                                            */
+/* For every t in [0, num_tokens) with slot_mapping[t] >= 0:                  */
+/*   k_cache[slot / bs][slot % bs][h][:] = k[t][h][:]  (all h), same for v.   */
+/* A bitwise copy (16-byte vectors); slot -1 means "skip this row".           */
+/* k, v: [num_tokens][num_kv_heads][head_dim] device, read only.             */
+/* slot_mapping: int64 [num_tokens] device.  Duplicate slots are undefined.  */
+/* k_cache, v_cache: [num_blocks][block_size][num_kv_heads][head_dim] device.*/
+/* k and v must not overlap the caches.  num_tokens == 0 is a no-op.         */
+/* ------------------------------------------------------------------------ */
+int pa_write_kv(const void* k, const void* v, const int64_t* slot_mapping, int num_tokens,
+                void* k_cache, void* v_cache, int num_blocks, int block_size, int num_kv_heads,
+                int head_dim, int dtype, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Block copy for copy-on-write (P1 s2.1 reference counts; P2 s4 block       */
+/* sharing).  For each pair i: block pairs[2i+1] of both caches becomes a     */
+/* bitwise copy of block pairs[2i].  pairs: int32 [num_pairs][2] device.     */
+/* Source and destination blocks of all pairs must be distinct.             */
+/* ------------------------------------------------------------------------ */
+int pa_copy_blocks(const int32_t* pairs, int num_pairs, void* k_cache, void* v_cache, int num_blocks,
+                   int block_size, int num_kv_heads, int head_dim, int dtype, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Paged decode (P1 s2.2.1, s4.2; P2 s2.2, s3.1): one query token per        */
+/* sequence attends to all context_lens[b] tokens of its sequence:           */
+/*   out[b][h] = sum_t softmax_t(scale * <q[b][h], K_b[t][h/G]>) V_b[t][h/G] */
+/* The context of each sequence is cut into splits of `split_len` tokens     */
+/* (split-K); each split yields fp32 (max, sum, weighted V), merged by a     */
+/* log-sum-exp reduce kernel.  A sequence that fits one split is written     */
+/* directly.  context_lens[b] == 0 gives out[b] = 0.                         */
+/*                                                                           */
+/* pa_decode_plan: the split length and workspace the call will use for     */
+/* these sizes.  num_splits_or_0 > 0 forces about that many splits for the  */
+/* longest sequence; 0 picks the split length from the batch shape.         */
+/* Any output pointer may be NULL.                                           */
+/* ------------------------------------------------------------------------ */
+int pa_decode_plan(int batch, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len,
+                   int num_splits_or_0, int* split_len_out, int* max_splits_out, size_t* workspace_bytes_out);
+
+/* Bytes of device workspace pa_decode needs for these sizes (0 on bad args). */
+size_t pa_decode_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                                int max_context_len, int num_splits_or_0);
+
+/* q: [batch][num_q_heads][head_dim]; out: same shape; caches as above.      */
+/* max_context_len: host-side upper bound of context_lens (sizes the grid).  */
+/* workspace: device scratch of >= pa_decode_workspace_size() bytes, 256-byte */
+/* aligned, owned by the caller, contents need no initialisation; it may be  */
+/* NULL when every sequence fits one split (max_context_len <= split_len).   */
+/* Two calls that run at the same time must use different workspaces.        */
+int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+              int max_blocks_per_seq, const int32_t* context_lens, int batch, int num_q_heads,
+              int num_kv_heads, int head_dim, int block_size, int num_blocks, int max_context_len,
+              float scale, int dtype, void* workspace, size_t workspace_bytes, int num_splits_or_0,
+              void* out, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Chunked prefill (P3 s1.1 / s3.1 PCP: prefill cut into chunks on one       */
+/* device).  Sequence b appends C_b = query_start_loc[b+1]-query_start_loc[b]*/
+/* query tokens whose K/V were already written (pa_write_kv) so that the    */
+/* sequence now holds L_b = context_lens[b] tokens.  Query i of the chunk    */
+/* sits at position p = L_b - C_b + i and attends causally to keys 0..p:     */
+/*   out[r][h] = sum_{t<=p} softmax_t(scale*<q[r][h], K_b[t][h/G]>) V_b[t][h/G] */
+/* with r = query_start_loc[b] + i.                                          */
+/* q, out: [total_q_tokens][num_q_heads][head_dim]; query_start_loc: int32   */
+/* [batch+1] device, query_start_loc[0] = 0, non-decreasing, last =          */
+/* total_q_tokens; C_b <= max_chunk_len and C_b <= L_b.  Requires bf16 or   */
+/* f16 with head_dim 128 on the tensor-core path (tcgen05/TMEM).            */
+/* ------------------------------------------------------------------------ */
+int pa_prefill_chunk(const void* q, const int32_t* query_start_loc, int total_q_tokens, int max_chunk_len,
+                     const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                     int max_blocks_per_seq, const int32_t* context_lens, int batch, int num_q_heads,
+                     int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale, int dtype,
+                     void* out, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Device error word.  Kernels never trap; a kernel that finds a broken     */
+/* device-side invariant (a wait that timed out, an index out of range in   */
+/* checked paths) ORs a bit into a per-device error word.  This call        */
+/* synchronises the current device, copies the word to *out and clears it. */
+/* Bits: 1 = pipeline wait timed out, 2 = index out of range.               */
+/* ------------------------------------------------------------------------ */
+int pa_device_error(int* out);
+
+/* ------------------------------------------------------------------------ */
+/* Host block pool (P1 s2.1 Block/BlockTable with ref_count; P2 s2.1        */
+/* BlockAllocator).  Pure host bookkeeping, no device memory.  Policy: the  */
+/* free list starts in `free_order` (NULL = 0..num_blocks-1); allocation    */
+/* pops from its head; blocks whose count drops to zero go to its tail.     */
+/* A sequence of n tokens holds ceil(n / block_size) blocks.  All calls are */
+/* atomic: on error the pool is unchanged.  Not thread-safe.                */
+/* ------------------------------------------------------------------------ */
+typedef struct pa_pool pa_pool;
+
+typedef struct {
+  int64_t num_blocks;
+  int64_t free_blocks;
+  int64_t used_blocks;    /* blocks with ref_count >= 1 */
+  int64_t shared_blocks;  /* blocks with ref_count >= 2 */
+  int64_t num_seqs;
+  int64_t tokens;         /* sum of sequence lengths */
+  int64_t table_refs;     /* sum over sequences of blocks held (== sum of ref counts) */
+  int64_t ref_sum;        /* sum of ref counts over all blocks */
+  double utilisation;     /* tokens / (table_refs * block_size); 1.0 when empty */
+} pa_pool_stats_t;
+
+/* Returns NULL on bad arguments (num_blocks < 0, block_size <= 0, free_order not a permutation). */
+pa_pool* pa_pool_create(int num_blocks, int block_size, const int32_t* free_order);
+void pa_pool_destroy(pa_pool* pool);
+
+/* New sequence holding num_tokens token slots (ceil(n/bs) blocks, ref_count 1 each). */
+int pa_seq_alloc(pa_pool* pool, int64_t seq_id, int num_tokens);
+
+/* New sequence `child` mapping the first ceil(n_prefix/bs) blocks of `parent` (ref_count += 1 each);
+   its length is n_prefix (0 <= n_prefix <= parent length). */
+int pa_seq_fork(pa_pool* pool, int64_t parent_id, int64_t child_id, int n_prefix);
+
+/* Extend a sequence by n tokens.  slot_mapping_out (host int64 [n], may be NULL) receives the slot of
+   each new token.  If the last block is shared and partly filled it is first replaced by a fresh copy
+   (copy-on-write): the (src, dst) pair goes to cow_pairs_out (host int32 [2], may be NULL) and
+   *num_cow_out (may be NULL) is set to 0 or 1; the caller copies the block (pa_copy_blocks). */
+int pa_seq_append(pa_pool* pool, int64_t seq_id, int n, int64_t* slot_mapping_out, int32_t* cow_pairs_out,
+                  int* num_cow_out);
+
+/* Drop a sequence: ref_count -= 1 on each of its blocks; blocks reaching 0 return to the free list. */
+int pa_seq_free(pa_pool* pool, int64_t seq_id);
+
+/* Length of a sequence (tokens) in *len_out and blocks held in *blocks_out (either may be NULL). */
+int pa_seq_info(const pa_pool* pool, int64_t seq_id, int* len_out, int* blocks_out);
+
+/* Export block table rows for seq_ids[0..n): out is host int32 [n][max_blocks], padded with -1;
+   ctx_lens_out (host int32 [n], may be NULL) receives the lengths.  PA_ERR_INVALID if a row is too short. */
+int pa_pool_block_table(const pa_pool* pool, const int64_t* seq_ids, int n, int32_t* out, int max_blocks,
+                        int32_t* ctx_lens_out);
+
+/* Reference count of one physical block (or -1 for an id out of range). */
+int pa_pool_ref_count(const pa_pool* pool, int block_id);
+
+int pa_pool_stats(const pa_pool* pool, pa_pool_stats_t* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGED_ATTN_H */

@@ -1,0 +1,290 @@
+"""Python binding of libpaged_attn.so: paged KV-cache attention for B200 (sm_100a).
+
+Argument marshalling only.  Every step of the compute path runs in the CUDA
+kernels behind the C ABI declared in ``include/paged_attn.h``; PyTorch is used
+for device memory and streams.  There is no CPU or PyTorch fallback: if the
+shared library is missing, importing this package raises ImportError.
+
+Calls (see the header for exact semantics):
+
+* ``write_kv``       - scatter new tokens' K/V into their cache slots
+* ``copy_blocks``    - copy whole blocks (copy-on-write of shared blocks)
+* ``decode``         - one-token paged attention, split-K with a reduce kernel
+* ``prefill_chunk``  - causal chunked-prefill attention over the paged cache
+* ``BlockPool``      - host block pool: blocks, block tables, reference counts
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+__all__ = ["PagedAttnError", "PoolOutOfBlocks", "BlockPool", "write_kv", "copy_blocks", "decode", "decode_plan",
+           "prefill_chunk", "device_error", "lib", "LIB_PATH", "replay_ops", "version"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpaged_attn.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built; run `python -m paged_kv_cache_330_b200.build` "
+                      "(there is no fallback path)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_vp, _i, _i64, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+_ip = ctypes.POINTER(ctypes.c_int)
+
+
+class _PoolStats(ctypes.Structure):
+    _fields_ = [("num_blocks", ctypes.c_int64), ("free_blocks", ctypes.c_int64), ("used_blocks", ctypes.c_int64),
+                ("shared_blocks", ctypes.c_int64), ("num_seqs", ctypes.c_int64), ("tokens", ctypes.c_int64),
+                ("table_refs", ctypes.c_int64), ("ref_sum", ctypes.c_int64), ("utilisation", ctypes.c_double)]
+
+
+_SIGS = {
+    "pa_strerror": (ctypes.c_char_p, [_i]),
+    "pa_version": (ctypes.c_char_p, []),
+    "pa_write_kv": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
+    "pa_copy_blocks": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
+    "pa_decode_plan": (_i, [_i, _i, _i, _i, _i, _i, _ip, _ip, ctypes.POINTER(_sz)]),
+    "pa_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "pa_decode": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _sz, _i, _vp, _vp]),
+    "pa_prefill_chunk": (_i, [_vp, _vp, _i, _i, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _vp]),
+    "pa_device_error": (_i, [_ip]),
+    "pa_pool_create": (_vp, [_i, _i, _i32p]),
+    "pa_pool_destroy": (None, [_vp]),
+    "pa_seq_alloc": (_i, [_vp, _i64, _i]),
+    "pa_seq_fork": (_i, [_vp, _i64, _i64, _i]),
+    "pa_seq_append": (_i, [_vp, _i64, _i, _i64p, _i32p, _ip]),
+    "pa_seq_free": (_i, [_vp, _i64]),
+    "pa_seq_info": (_i, [_vp, _i64, _ip, _ip]),
+    "pa_pool_block_table": (_i, [_vp, _i64p, _i, _i32p, _i, _i32p]),
+    "pa_pool_ref_count": (_i, [_vp, _i]),
+    "pa_pool_stats": (_i, [_vp, ctypes.POINTER(_PoolStats)]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+PA_OK, PA_ERR_OOM, PA_ERR_NOT_FOUND = 0, -6, -7
+
+
+class PagedAttnError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        msg = lib.pa_strerror(status).decode()
+        super().__init__(f"{what}: {msg}" if what else msg)
+
+
+class PoolOutOfBlocks(PagedAttnError):
+    pass
+
+
+def _check(status: int, what: str = "") -> None:
+    if status != PA_OK:
+        raise PagedAttnError(status, what)
+
+
+def version() -> str:
+    return lib.pa_version().decode()
+
+
+# ---------------------------------------------------------------------------------------------- device calls
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float16:
+        return 0
+    if t.dtype == torch.bfloat16:
+        return 1
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def _stream_handle(stream):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def write_kv(k, v, slot_mapping, k_cache, v_cache, stream=None) -> None:
+    """k, v [T, Hkv, D]; slot_mapping int64 [T] (-1 = skip); caches [NB, bs, Hkv, D]."""
+    _contig(k, v, slot_mapping, k_cache, v_cache)
+    NB, bs, Hkv, D = k_cache.shape
+    _check(lib.pa_write_kv(_ptr(k), _ptr(v), _ptr(slot_mapping), int(k.shape[0]), _ptr(k_cache), _ptr(v_cache),
+                           NB, bs, Hkv, D, _dtype_code(k_cache), _stream_handle(stream)), "pa_write_kv")
+
+
+def copy_blocks(pairs, k_cache, v_cache, stream=None) -> None:
+    """pairs int32 [n, 2] (src, dst) on the device."""
+    _contig(pairs, k_cache, v_cache)
+    NB, bs, Hkv, D = k_cache.shape
+    _check(lib.pa_copy_blocks(_ptr(pairs), int(pairs.shape[0]), _ptr(k_cache), _ptr(v_cache), NB, bs, Hkv, D,
+                              _dtype_code(k_cache), _stream_handle(stream)), "pa_copy_blocks")
+
+
+def decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_splits=0):
+    """(split_len, max_splits, workspace_bytes) the decode call will use."""
+    sl, ms, ws = ctypes.c_int(), ctypes.c_int(), ctypes.c_size_t()
+    _check(lib.pa_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_splits,
+                              ctypes.byref(sl), ctypes.byref(ms), ctypes.byref(ws)), "pa_decode_plan")
+    return sl.value, ms.value, ws.value
+
+
+def decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float, out=None,
+           workspace=None, num_splits: int = 0, stream=None):
+    """q [B, Hq, D]; block_tables int32 [B, max_blocks]; context_lens int32 [B]. Returns out [B, Hq, D]."""
+    torch = _torch()
+    _contig(q, k_cache, v_cache, block_tables, context_lens, out, workspace)
+    B, Hq, D = q.shape
+    NB, bs, Hkv, _ = k_cache.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _, _, need = decode_plan(B, Hq, Hkv, D, max_context_len, num_splits)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.pa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), int(block_tables.shape[1]),
+                         _ptr(context_lens), B, Hq, Hkv, D, bs, NB, int(max_context_len), float(scale),
+                         _dtype_code(q), _ptr(workspace), ws_bytes, int(num_splits), _ptr(out),
+                         _stream_handle(stream)), "pa_decode")
+    return out
+
+
+def prefill_chunk(q, query_start_loc, k_cache, v_cache, block_tables, context_lens, max_chunk_len: int,
+                  scale: float, out=None, stream=None):
+    """q [sum C, Hq, D]; query_start_loc int32 [B+1]; returns out [sum C, Hq, D]."""
+    torch = _torch()
+    _contig(q, query_start_loc, k_cache, v_cache, block_tables, context_lens, out)
+    T, Hq, D = q.shape
+    NB, bs, Hkv, _ = k_cache.shape
+    B = int(context_lens.shape[0])
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib.pa_prefill_chunk(_ptr(q), _ptr(query_start_loc), T, int(max_chunk_len), _ptr(k_cache), _ptr(v_cache),
+                                _ptr(block_tables), int(block_tables.shape[1]), _ptr(context_lens), B, Hq, Hkv, D,
+                                bs, NB, float(scale), _dtype_code(q), _ptr(out), _stream_handle(stream)),
+           "pa_prefill_chunk")
+    return out
+
+
+def device_error() -> int:
+    """Synchronise the device, return and clear the kernels' error bits (0 = none)."""
+    v = ctypes.c_int()
+    _check(lib.pa_device_error(ctypes.byref(v)), "pa_device_error")
+    return v.value
+
+
+# ---------------------------------------------------------------------------------------------- host pool
+class BlockPool:
+    """Host block pool (C++): blocks, per-sequence block tables, reference counts, copy-on-write."""
+
+    def __init__(self, num_blocks: int, block_size: int, free_order=None):
+        self.block_size = block_size
+        self.num_blocks = num_blocks
+        arr = None
+        if free_order is not None:
+            arr = np.ascontiguousarray(np.asarray(free_order, dtype=np.int32))
+            if arr.shape != (num_blocks,):
+                raise ValueError("free_order must have num_blocks entries")
+        ptr = arr.ctypes.data_as(_i32p) if arr is not None else None
+        self._h = lib.pa_pool_create(num_blocks, block_size, ptr)
+        if not self._h:
+            raise ValueError("pa_pool_create rejected its arguments")
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib.pa_pool_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
+
+    @staticmethod
+    def _pool_check(status, what):
+        if status == PA_ERR_OOM:
+            raise PoolOutOfBlocks(status, what)
+        _check(status, what)
+
+    def alloc(self, seq_id: int, num_tokens: int) -> None:
+        self._pool_check(lib.pa_seq_alloc(self._h, seq_id, num_tokens), "alloc")
+
+    def fork(self, parent: int, child: int, n_prefix: int) -> None:
+        self._pool_check(lib.pa_seq_fork(self._h, parent, child, n_prefix), "fork")
+
+    def append(self, seq_id: int, n: int):
+        """Returns (slots int64[n], copy-on-write pairs [(src, dst)])."""
+        slots = np.empty(max(n, 1), dtype=np.int64)
+        pair = np.empty(2, dtype=np.int32)
+        ncow = ctypes.c_int(0)
+        self._pool_check(lib.pa_seq_append(self._h, seq_id, n, slots.ctypes.data_as(_i64p), pair.ctypes.data_as(_i32p),
+                                           ctypes.byref(ncow)), "append")
+        return slots[:n], ([(int(pair[0]), int(pair[1]))] if ncow.value else [])
+
+    def free(self, seq_id: int) -> None:
+        self._pool_check(lib.pa_seq_free(self._h, seq_id), "free")
+
+    def info(self, seq_id: int):
+        n, nb = ctypes.c_int(), ctypes.c_int()
+        self._pool_check(lib.pa_seq_info(self._h, seq_id, ctypes.byref(n), ctypes.byref(nb)), "info")
+        return n.value, nb.value
+
+    def block_table(self, seq_ids, max_blocks: int):
+        ids = np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int64))
+        out = np.empty((len(ids), max(max_blocks, 0)), dtype=np.int32)
+        lens = np.empty(len(ids), dtype=np.int32)
+        self._pool_check(lib.pa_pool_block_table(self._h, ids.ctypes.data_as(_i64p), len(ids),
+                                                 out.ctypes.data_as(_i32p), max_blocks, lens.ctypes.data_as(_i32p)),
+                         "block_table")
+        return out, lens
+
+    def ref_count(self, block_id: int) -> int:
+        return lib.pa_pool_ref_count(self._h, block_id)
+
+    def stats(self) -> dict:
+        st = _PoolStats()
+        _check(lib.pa_pool_stats(self._h, ctypes.byref(st)), "stats")
+        return {f: getattr(st, f) for f, _ in _PoolStats._fields_}
+
+
+def replay_ops(ops, num_blocks: int, block_size: int, free_order, batch: int):
+    """Run a list of pool operations ('alloc', id, n) / ('fork', parent, child, n) / ('append', id, n) /
+    ('append_new', id, n) on a new BlockPool.
+
+    Returns (pool, block_tables int32 [batch, max_blocks], context_lens int32 [batch], slot_mapping int64
+    of the 'append_new' tokens in order, copy-on-write pairs)."""
+    pool = BlockPool(num_blocks, block_size, free_order)
+    slots, pairs = [], []
+    for op in ops:
+        if op[0] == "alloc":
+            pool.alloc(op[1], op[2])
+        elif op[0] == "fork":
+            pool.fork(op[1], op[2], op[3])
+        elif op[0] in ("append", "append_new"):
+            s, p = pool.append(op[1], op[2])
+            pairs += p
+            if op[0] == "append_new":
+                slots.append(s)
+        else:
+            raise ValueError(op[0])
+    max_blocks = max([pool.info(b)[1] for b in range(batch)] + [1])
+    bt, lens = pool.block_table(list(range(batch)), max_blocks)
+    sm = np.concatenate(slots) if slots else np.zeros(0, dtype=np.int64)
+    return pool, bt, lens, sm, pairs

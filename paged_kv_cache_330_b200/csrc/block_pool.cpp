@@ -1,0 +1,188 @@
+// Host block pool: the Block / BlockTable bookkeeping of the page
+// "Nano-vLLM-Ascend: lightweight LLM inference framework for Ascend NPU",
+// section 2.1 (16-token blocks, logical -> physical block map per sequence,
+// a reference count per block), with the single-pool allocator role of
+// BlockAllocator from "Ascend NPU LLM inference optimisation: the vLLM-Ascend
+// approach", section 2.1, and block sharing across sequences (same page,
+// section 4).
+//
+// The pool is pure host bookkeeping over block ids; the K/V bytes live in the
+// caller's device tensors.  Every operation checks first and mutates second,
+// so a failed call leaves the pool unchanged.
+
+#include <algorithm>
+#include <cstdint>
+#include <deque>
+#include <unordered_map>
+#include <vector>
+
+#include "paged_attn.h"
+
+struct pa_pool {
+  int num_blocks = 0;
+  int block_size = 0;
+  std::deque<int32_t> free_list;        // head = next block handed out
+  std::vector<int32_t> ref;             // reference count per physical block
+  struct Seq {
+    std::vector<int32_t> blocks;        // logical block j -> physical block
+    int64_t len = 0;                    // tokens
+  };
+  std::unordered_map<int64_t, Seq> seqs;
+
+  int32_t take() {
+    int32_t b = free_list.front();
+    free_list.pop_front();
+    ref[b] = 1;
+    return b;
+  }
+};
+
+static inline int64_t blocks_for(int64_t n, int bs) { return (n + bs - 1) / bs; }
+
+extern "C" pa_pool* pa_pool_create(int num_blocks, int block_size, const int32_t* free_order) {
+  if (num_blocks < 0 || block_size <= 0) return nullptr;
+  pa_pool* p = new pa_pool;
+  p->num_blocks = num_blocks;
+  p->block_size = block_size;
+  p->ref.assign(num_blocks, 0);
+  if (free_order) {
+    std::vector<char> seen(num_blocks, 0);
+    for (int i = 0; i < num_blocks; ++i) {
+      int32_t b = free_order[i];
+      if (b < 0 || b >= num_blocks || seen[b]) {
+        delete p;
+        return nullptr;
+      }
+      seen[b] = 1;
+      p->free_list.push_back(b);
+    }
+  } else {
+    for (int i = 0; i < num_blocks; ++i) p->free_list.push_back(i);
+  }
+  return p;
+}
+
+extern "C" void pa_pool_destroy(pa_pool* pool) { delete pool; }
+
+extern "C" int pa_seq_alloc(pa_pool* pool, int64_t seq_id, int num_tokens) {
+  if (!pool || num_tokens < 0) return PA_ERR_INVALID;
+  if (pool->seqs.count(seq_id)) return PA_ERR_NOT_FOUND;
+  int64_t need = blocks_for(num_tokens, pool->block_size);
+  if (need > (int64_t)pool->free_list.size()) return PA_ERR_OOM;
+  pa_pool::Seq s;
+  s.blocks.reserve(need);
+  for (int64_t i = 0; i < need; ++i) s.blocks.push_back(pool->take());
+  s.len = num_tokens;
+  pool->seqs.emplace(seq_id, std::move(s));
+  return PA_OK;
+}
+
+extern "C" int pa_seq_fork(pa_pool* pool, int64_t parent_id, int64_t child_id, int n_prefix) {
+  if (!pool || n_prefix < 0) return PA_ERR_INVALID;
+  auto it = pool->seqs.find(parent_id);
+  if (it == pool->seqs.end() || pool->seqs.count(child_id)) return PA_ERR_NOT_FOUND;
+  if (n_prefix > it->second.len) return PA_ERR_INVALID;
+  pa_pool::Seq c;
+  int64_t nb = blocks_for(n_prefix, pool->block_size);
+  c.blocks.assign(it->second.blocks.begin(), it->second.blocks.begin() + nb);
+  for (int32_t b : c.blocks) pool->ref[b] += 1;
+  c.len = n_prefix;
+  pool->seqs.emplace(child_id, std::move(c));
+  return PA_OK;
+}
+
+extern "C" int pa_seq_append(pa_pool* pool, int64_t seq_id, int n, int64_t* slot_mapping_out,
+                             int32_t* cow_pairs_out, int* num_cow_out) {
+  if (!pool || n < 0) return PA_ERR_INVALID;
+  auto it = pool->seqs.find(seq_id);
+  if (it == pool->seqs.end()) return PA_ERR_NOT_FOUND;
+  pa_pool::Seq& s = it->second;
+  const int bs = pool->block_size;
+  const int64_t n0 = s.len;
+  const bool cow = n > 0 && (n0 % bs) != 0 && pool->ref[s.blocks.back()] > 1;
+  int64_t need = blocks_for(n0 + n, bs) - (int64_t)s.blocks.size() + (cow ? 1 : 0);
+  if (need > (int64_t)pool->free_list.size()) return PA_ERR_OOM;
+  if (num_cow_out) *num_cow_out = 0;
+  if (cow) {
+    int32_t old_b = s.blocks.back();
+    int32_t new_b = pool->take();
+    pool->ref[old_b] -= 1;
+    s.blocks.back() = new_b;
+    if (cow_pairs_out) {
+      cow_pairs_out[0] = old_b;
+      cow_pairs_out[1] = new_b;
+    }
+    if (num_cow_out) *num_cow_out = 1;
+  }
+  for (int64_t p = n0; p < n0 + n; ++p) {
+    if (p % bs == 0) s.blocks.push_back(pool->take());
+    if (slot_mapping_out) slot_mapping_out[p - n0] = (int64_t)s.blocks[p / bs] * bs + p % bs;
+  }
+  s.len = n0 + n;
+  return PA_OK;
+}
+
+extern "C" int pa_seq_free(pa_pool* pool, int64_t seq_id) {
+  if (!pool) return PA_ERR_INVALID;
+  auto it = pool->seqs.find(seq_id);
+  if (it == pool->seqs.end()) return PA_ERR_NOT_FOUND;
+  for (int32_t b : it->second.blocks) {
+    pool->ref[b] -= 1;
+    if (pool->ref[b] == 0) pool->free_list.push_back(b);
+  }
+  pool->seqs.erase(it);
+  return PA_OK;
+}
+
+extern "C" int pa_seq_info(const pa_pool* pool, int64_t seq_id, int* len_out, int* blocks_out) {
+  if (!pool) return PA_ERR_INVALID;
+  auto it = pool->seqs.find(seq_id);
+  if (it == pool->seqs.end()) return PA_ERR_NOT_FOUND;
+  if (len_out) *len_out = (int)it->second.len;
+  if (blocks_out) *blocks_out = (int)it->second.blocks.size();
+  return PA_OK;
+}
+
+extern "C" int pa_pool_block_table(const pa_pool* pool, const int64_t* seq_ids, int n, int32_t* out,
+                                   int max_blocks, int32_t* ctx_lens_out) {
+  if (!pool || n < 0 || max_blocks < 0 || (n > 0 && (!seq_ids || !out))) return PA_ERR_INVALID;
+  for (int i = 0; i < n; ++i) {  // check every row before writing any
+    auto it = pool->seqs.find(seq_ids[i]);
+    if (it == pool->seqs.end()) return PA_ERR_NOT_FOUND;
+    if ((int64_t)it->second.blocks.size() > max_blocks) return PA_ERR_INVALID;
+  }
+  for (int i = 0; i < n; ++i) {
+    const pa_pool::Seq& s = pool->seqs.find(seq_ids[i])->second;
+    int32_t* row = out + (int64_t)i * max_blocks;
+    size_t j = 0;
+    for (; j < s.blocks.size(); ++j) row[j] = s.blocks[j];
+    for (; j < (size_t)max_blocks; ++j) row[j] = -1;
+    if (ctx_lens_out) ctx_lens_out[i] = (int32_t)s.len;
+  }
+  return PA_OK;
+}
+
+extern "C" int pa_pool_ref_count(const pa_pool* pool, int block_id) {
+  if (!pool || block_id < 0 || block_id >= pool->num_blocks) return -1;
+  return pool->ref[block_id];
+}
+
+extern "C" int pa_pool_stats(const pa_pool* pool, pa_pool_stats_t* out) {
+  if (!pool || !out) return PA_ERR_INVALID;
+  pa_pool_stats_t st{};
+  st.num_blocks = pool->num_blocks;
+  st.free_blocks = (int64_t)pool->free_list.size();
+  for (int32_t r : pool->ref) {
+    if (r > 0) st.used_blocks++;
+    if (r > 1) st.shared_blocks++;
+    st.ref_sum += r;
+  }
+  st.num_seqs = (int64_t)pool->seqs.size();
+  for (const auto& kv : pool->seqs) {
+    st.tokens += kv.second.len;
+    st.table_refs += (int64_t)kv.second.blocks.size();
+  }
+  st.utilisation = st.table_refs ? (double)st.tokens / ((double)st.table_refs * pool->block_size) : 1.0;
+  *out = st;
+  return PA_OK;
+}

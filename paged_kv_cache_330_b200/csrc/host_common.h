@@ -1,0 +1,28 @@
+// Host-side helpers shared by the launch wrappers (internal, not exported).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "paged_attn.h"
+
+namespace pa {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool valid_dtype(int dt) { return dt == PA_F16 || dt == PA_BF16; }
+inline bool valid_block_size(int bs) { return bs == 16 || bs == 32 || bs == 64 || bs == 128 || bs == 256; }
+inline bool valid_head_dim(int d) { return d == 64 || d == 128; }
+inline bool valid_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
+
+// Encode a 2-D tiled tensor map over a row-major [rows][cols] matrix of 16-bit
+// elements with a 128-byte swizzle: box = box_cols x box_rows elements
+// (box_cols * 2 must be <= 128).  Returns PA_OK or PA_ERR_CUDA.
+int encode_2d_sw128(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t row_stride_bytes,
+                    uint32_t box_cols, uint32_t box_rows);
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+}  // namespace pa

@@ -1,0 +1,211 @@
+"""Host-side tests of the C ABI (no GPU): exported symbols, argument validation, decode planning,
+and the C++ block pool against the oracle's pool (bit-exact block tables, slots, counts)."""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import random
+import re
+
+import numpy as np
+import pytest
+
+import paged_kv_cache_330_b200 as pa
+from oracle.block_pool import OraclePool, OutOfBlocks, replay
+from workloads import CONFIGS, make_workload
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "paged_attn.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 18
+    for n in names:
+        assert hasattr(pa.lib, n), f"{n} declared in include/paged_attn.h but not exported"
+
+
+def test_status_strings():
+    for code in range(-8, 1):
+        assert pa.lib.pa_strerror(code).decode().startswith("PA_")
+    assert pa.version().count(".") == 2
+
+
+# --------------------------------------------------------------------------- validation before any launch
+FAKE = ctypes.c_void_p(0x10000)      # aligned, never dereferenced: every call below fails validation first
+MISALIGNED = ctypes.c_void_p(0x10008)
+NULL = ctypes.c_void_p(0)
+
+
+def test_write_kv_validation():
+    L = pa.lib
+    # unsupported dtype / block size / negative sizes
+    assert L.pa_write_kv(FAKE, FAKE, FAKE, 4, FAKE, FAKE, 8, 16, 2, 64, 7, NULL) == -2
+    assert L.pa_write_kv(FAKE, FAKE, FAKE, 4, FAKE, FAKE, 8, 24, 2, 64, 1, NULL) == -2
+    assert L.pa_write_kv(FAKE, FAKE, FAKE, -1, FAKE, FAKE, 8, 16, 2, 64, 1, NULL) == -1
+    assert L.pa_write_kv(FAKE, FAKE, NULL, 4, FAKE, FAKE, 8, 16, 2, 64, 1, NULL) == -1
+    assert L.pa_write_kv(FAKE, FAKE, FAKE, 4, NULL, FAKE, 8, 16, 2, 64, 1, NULL) == -1
+    assert L.pa_write_kv(MISALIGNED, FAKE, FAKE, 4, FAKE, FAKE, 8, 16, 2, 64, 1, NULL) == -3
+    assert L.pa_write_kv(FAKE, FAKE, FAKE, 4, MISALIGNED, FAKE, 8, 16, 2, 64, 1, NULL) == -3
+    assert L.pa_write_kv(FAKE, FAKE, FAKE, 0, FAKE, FAKE, 8, 16, 2, 64, 1, NULL) == 0   # no-op, nothing launched
+
+
+def _dec(**kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, mb=8, cl=FAKE, B=2, Hq=8, Hkv=2, D=128, bs=16, NB=16, maxL=100,
+             scale=0.1, dt=1, ws=FAKE, wsb=1 << 30, ns=0, out=FAKE)
+    a.update(kw)
+    return pa.lib.pa_decode(a["q"], a["kc"], a["vc"], a["bt"], a["mb"], a["cl"], a["B"], a["Hq"], a["Hkv"], a["D"],
+                            a["bs"], a["NB"], a["maxL"], a["scale"], a["dt"], a["ws"], a["wsb"], a["ns"], a["out"],
+                            NULL)
+
+
+def test_decode_validation():
+    assert _dec(D=96) == -2
+    assert _dec(bs=8) == -2
+    assert _dec(dt=3) == -2
+    assert _dec(Hq=6, Hkv=4) == -1          # not a multiple
+    assert _dec(Hq=64, Hkv=2) == -2         # group 32 unsupported
+    assert _dec(q=NULL) == -1
+    assert _dec(out=MISALIGNED) == -3
+    assert _dec(mb=4) == -1                 # block-table rows too short for max_context_len
+    assert _dec(maxL=5000, mb=400, ws=NULL) == -4
+    assert _dec(maxL=5000, mb=400, wsb=16) == -4
+    assert _dec(B=0) == 0
+
+
+def test_prefill_validation():
+    L = pa.lib
+    args = [FAKE, FAKE, 64, 64, FAKE, FAKE, FAKE, 8, FAKE, 1, 8, 2, 128, 16, 16, 0.1, 1, FAKE, NULL]
+    bad = list(args); bad[0] = NULL
+    assert L.pa_prefill_chunk(*bad) == -1
+    bad = list(args); bad[12] = 80
+    assert L.pa_prefill_chunk(*bad) == -2
+    bad = list(args); bad[17] = MISALIGNED
+    assert L.pa_prefill_chunk(*bad) == -3
+
+
+def test_decode_plan():
+    for name in ("tiny", "qwen_decode", "llama70b_long", "prefix_sweep"):
+        c = CONFIGS[name]
+        maxL = {"tiny": 64, "qwen_decode": 1024, "llama70b_long": 8192, "prefix_sweep": 2561}[name]
+        sl, ms, ws = pa.decode_plan(c["batch"], c["num_q_heads"], c["num_kv_heads"], c["head_dim"], maxL)
+        assert sl % 64 == 0 and sl >= 64 and ms == -(-maxL // sl)
+        if ms > 1:
+            rows = c["batch"] * c["num_q_heads"] * ms
+            assert ws >= rows * (c["head_dim"] + 2) * 4
+        else:
+            assert ws == 0
+        assert pa.lib.pa_decode_workspace_size(c["batch"], c["num_q_heads"], c["num_kv_heads"], c["head_dim"], maxL, 0) == ws
+    sl, ms, _ = pa.decode_plan(4, 8, 2, 128, 1000, num_splits=4)
+    assert ms == 4 and sl == 256
+    sl, ms, ws = pa.decode_plan(4, 8, 2, 128, 1000, num_splits=1)
+    assert ms == 1 and ws == 0
+
+
+# --------------------------------------------------------------------------- C++ pool vs oracle pool
+def _compare_pools(cpp: pa.BlockPool, orc: OraclePool, live):
+    st, so = cpp.stats(), orc.stats()
+    for k in ("num_blocks", "free_blocks", "used_blocks", "shared_blocks", "num_seqs", "tokens", "table_refs", "ref_sum"):
+        assert st[k] == so[k], k
+    assert abs(st["utilisation"] - so["utilisation"]) < 1e-12
+    if live:
+        mb = max(len(orc.seqs[s]["blocks"]) for s in live) + 1
+        bt, lens = cpp.block_table(live, mb)
+        rows, olens = orc.block_table(live, mb)
+        np.testing.assert_array_equal(bt, np.array(rows, dtype=np.int32))
+        np.testing.assert_array_equal(lens, np.array(olens, dtype=np.int32))
+    for b in range(orc.num_blocks):
+        assert cpp.ref_count(b) == orc.ref[b]
+
+
+def test_pool_parity_random_ops():
+    rnd = random.Random(5)
+    for bs in (16, 32, 64, 256):
+        NB = 150
+        order = list(np.random.default_rng(bs).permutation(NB))
+        cpp, orc = pa.BlockPool(NB, bs, order), OraclePool(NB, bs, order)
+        live, nid = [], 0
+        for step in range(800):
+            r = rnd.random()
+            if r < 0.3 or not live:
+                op = ("alloc", nid, rnd.randint(0, 400)); nid += 1
+            elif r < 0.45:
+                p = rnd.choice(live)
+                op = ("fork", p, nid, rnd.randint(0, orc.seqs[p]["len"])); nid += 1
+            elif r < 0.8:
+                op = ("append", rnd.choice(live), rnd.randint(0, 50))
+            else:
+                op = ("free", rnd.choice(live))
+            o_err = c_err = None
+            try:
+                if op[0] == "alloc": orc.alloc(op[1], op[2])
+                elif op[0] == "fork": orc.fork(op[1], op[2], op[3])
+                elif op[0] == "append": o_res = orc.append(op[1], op[2])
+                else: orc.free_seq(op[1])
+            except OutOfBlocks:
+                o_err = "oom"
+            try:
+                if op[0] == "alloc": cpp.alloc(op[1], op[2])
+                elif op[0] == "fork": cpp.fork(op[1], op[2], op[3])
+                elif op[0] == "append": c_res = cpp.append(op[1], op[2])
+                else: cpp.free(op[1])
+            except pa.PoolOutOfBlocks:
+                c_err = "oom"
+            assert o_err == c_err, (step, op)
+            if o_err is None:
+                if op[0] in ("alloc", "fork"):
+                    live.append(op[-2] if op[0] == "fork" else op[1])
+                elif op[0] == "free":
+                    live.remove(op[1])
+                elif op[0] == "append":
+                    np.testing.assert_array_equal(c_res[0], np.array(o_res[0], dtype=np.int64))
+                    assert c_res[1] == o_res[1]
+            if step % 50 == 0:
+                _compare_pools(cpp, orc, live)
+        _compare_pools(cpp, orc, live)
+        for s in list(live):
+            cpp.free(s); orc.free_seq(s)
+        _compare_pools(cpp, orc, [])
+        assert cpp.stats()["free_blocks"] == NB
+
+
+def test_pool_errors_leave_state_unchanged():
+    p = pa.BlockPool(4, 16)
+    p.alloc(0, 60)
+    with pytest.raises(pa.PoolOutOfBlocks):
+        p.append(0, 10)
+    assert p.info(0) == (60, 4)
+    with pytest.raises(pa.PagedAttnError):
+        p.alloc(0, 1)                        # duplicate id
+    with pytest.raises(pa.PagedAttnError):
+        p.fork(0, 1, 61)                     # longer than parent
+    with pytest.raises(pa.PagedAttnError):
+        p.free(9)
+    with pytest.raises(ValueError):
+        pa.BlockPool(4, 16, [0, 1, 1, 2])    # not a permutation
+    assert p.stats()["used_blocks"] == 4
+
+
+@pytest.mark.parametrize("name,bs", [("tiny", None), ("qwen_decode", None), ("llama70b_long", None),
+                                     ("prefix_sweep", 16), ("prefix_sweep", 256), ("prefill", None)])
+def test_workload_replay_parity(name, bs):
+    """The C++ pool and the oracle pool hand out identical block tables and slots for every workload."""
+    wl = make_workload(name, block_size=bs) if bs else make_workload(name)
+    bsz = wl.cfg["block_size"]
+    _, bt, lens, sm, cow = pa.replay_ops(wl.ops, wl.num_blocks, bsz, wl.free_order, wl.batch)
+    pool, rows, olens, osm, ocow = replay(wl.ops, wl.num_blocks, bsz, wl.free_order, wl.batch)
+    np.testing.assert_array_equal(bt, np.array(rows, dtype=np.int32))
+    np.testing.assert_array_equal(lens, wl.context_lens)
+    np.testing.assert_array_equal(sm, np.array(osm, dtype=np.int64))
+    assert cow == ocow == []
+    if name == "prefix_sweep":
+        st = pool.stats()
+        per_prefix = -(-wl.cfg["prefix_len"] // bsz)
+        assert st["shared_blocks"] == wl.cfg["groups"] * per_prefix
+        assert max(pool.ref) == wl.batch // wl.cfg["groups"]        # ref_count 32 on prefix blocks

@@ -1,0 +1,170 @@
+"""GPU parity: pa_write_kv (bit-exact) and pa_decode (tolerance) against the oracle, through the C ABI."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import attention as oatt
+from tests.gpu_common import assert_close, bits, gpu_step, oracle_step
+from workloads import make_custom, make_workload
+
+pytestmark = pytest.mark.gpu
+
+pa = pytest.importorskip("paged_kv_cache_330_b200")
+
+
+@pytest.fixture(autouse=True)
+def _need_cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    yield
+    assert pa.device_error() == 0, "a kernel recorded a device-side error"
+
+
+# ------------------------------------------------------------------------------------------ KV write
+@pytest.mark.parametrize("name", ["tiny", "qwen_decode", "prefill"])
+def test_write_kv_bit_exact_workloads(name):
+    wl = make_workload(name)
+    _, kc, vc, *_ = gpu_step(wl) if wl.cfg["kind"] == "prefill" else gpu_step(wl)
+    okc, ovc, *_ = oracle_step(wl)
+    np.testing.assert_array_equal(bits(kc.cpu()), bits(okc))
+    np.testing.assert_array_equal(bits(vc.cpu()), bits(ovc))
+
+
+@pytest.mark.parametrize("Hkv,D,dt", [(1, 64, torch.float16), (8, 128, torch.bfloat16), (3, 64, torch.bfloat16),
+                                      (2, 8, torch.float16)])
+def test_write_kv_sentinel_and_skip(Hkv, D, dt):
+    g = torch.Generator().manual_seed(Hkv * 1000 + D)
+    NB, bs, T = 37, 16, 300
+    kc = torch.full((NB, bs, Hkv, D), 0, dtype=torch.int16).view(dt)
+    kc.view(torch.int16).fill_(0x5A5A)
+    vc = kc.clone()
+    k = torch.randn(T, Hkv, D, generator=g).to(dt)
+    v = torch.randn(T, Hkv, D, generator=g).to(dt)
+    slots = torch.randperm(NB * bs, generator=g)[:T].to(torch.int64)
+    slots[::7] = -1
+    okc, ovc = bits(kc).copy(), bits(vc).copy()
+    oracle.write_kv(bits(k), bits(v), slots.tolist(), okc, ovc)
+    kd, vd = kc.cuda(), vc.cuda()
+    pa.write_kv(k.cuda(), v.cuda(), slots.cuda(), kd, vd)
+    np.testing.assert_array_equal(bits(kd.cpu()), okc)
+    np.testing.assert_array_equal(bits(vd.cpu()), ovc)
+
+
+def test_copy_blocks_bit_exact():
+    g = torch.Generator().manual_seed(3)
+    kc = torch.randn(20, 32, 4, 64, generator=g).to(torch.bfloat16)
+    vc = torch.randn(20, 32, 4, 64, generator=g).to(torch.bfloat16)
+    pairs = torch.tensor([[3, 7], [0, 19], [12, 1]], dtype=torch.int32)
+    kd, vd = kc.cuda(), vc.cuda()
+    pa.copy_blocks(pairs.cuda(), kd, vd)
+    for s, d in pairs.tolist():
+        kc[d] = kc[s]
+        vc[d] = vc[s]
+    np.testing.assert_array_equal(bits(kd.cpu()), bits(kc))
+    np.testing.assert_array_equal(bits(vd.cpu()), bits(vc))
+
+
+# ------------------------------------------------------------------------------------------ decode
+def _oracle_decode(wl, rows=None):
+    okc, ovc, bt, lens, _ = oracle_step(wl)
+    if rows is None:
+        return oatt.decode_attention(wl.q, okc, ovc, bt, lens, wl.scale)
+    return oatt.decode_rows(wl.q, okc, ovc, bt, lens, wl.scale, rows)
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen_decode"])
+def test_decode_full_workload(name):
+    wl = make_workload(name)
+    out, *_ = gpu_step(wl)
+    ref = _oracle_decode(wl)
+    assert_close(out.float().cpu().numpy(), ref, name)
+
+
+def _sample_rows(wl, n, seed):
+    rng = np.random.default_rng(seed)
+    B, Hq = wl.batch, wl.cfg["num_q_heads"]
+    rows = {(0, 0), (B - 1, Hq - 1), (int(np.argmax(wl.context_lens)), Hq // 2),
+            (int(np.argmin(wl.context_lens)), 1)}
+    while len(rows) < n:
+        rows.add((int(rng.integers(B)), int(rng.integers(Hq))))
+    return sorted(rows)
+
+
+def test_decode_llama70b_long_sampled():
+    wl = make_workload("llama70b_long")
+    out, *_ = gpu_step(wl)
+    rows = _sample_rows(wl, 40, 0)
+    ref = _oracle_decode(wl, rows)
+    got = np.stack([out[b, h].float().cpu().numpy() for b, h in rows])
+    assert_close(got, ref, "llama70b_long")
+
+
+@pytest.mark.parametrize("bs", [16, 32, 64, 128, 256])
+def test_decode_prefix_shared_sampled(bs):
+    wl = make_workload("prefix_sweep", block_size=bs)
+    out, *_ = gpu_step(wl)
+    rows = _sample_rows(wl, 40, bs)
+    ref = _oracle_decode(wl, rows)
+    got = np.stack([out[b, h].float().cpu().numpy() for b, h in rows])
+    assert_close(got, ref, f"prefix bs={bs}")
+
+
+RAGGED = [0, 1, 2, 15, 16, 17, 31, 32, 33, 63, 64, 65, 127, 128, 129, 255, 256, 257, 511, 777, 1000, 1500]
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 4), (8, 2), (16, 2), (16, 1)])
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_decode_ragged_shapes(D, Hq, Hkv, dtype):
+    for bs, seed in ((16, 1), (64, 2), (256, 3)):
+        wl = make_custom(seed=seed * 97 + Hq * 7 + D, lens=RAGGED, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D,
+                         block_size=bs, dtype=dtype)
+        ref = _oracle_decode(wl)
+        for ns in (0, 1, 6):
+            out, *_ = gpu_step(wl, num_splits=ns)
+            got = out.float().cpu().numpy()
+            assert_close(got, ref, f"D{D} G{Hq // Hkv} bs{bs} {dtype} splits{ns}")
+            assert (got[0] == 0).all()          # empty sequence -> zeros
+
+
+def test_decode_split_count_invariance():
+    wl = make_workload("qwen_decode")
+    ref = _oracle_decode(wl)
+    outs = []
+    for ns in (0, 1, 2, 5, 16):
+        out, *_ = gpu_step(wl, num_splits=ns)
+        assert_close(out.float().cpu().numpy(), ref, f"splits={ns}")
+        outs.append(out.float().cpu())
+    for o in outs[1:]:
+        assert (o - outs[0]).abs().max().item() < 2e-2
+
+
+def test_decode_block_permutation_bitwise_invariant():
+    """The same logical cache placed with a different physical permutation gives bit-identical output."""
+    wl = make_workload("qwen_decode")
+    out1, kc, vc, bt, lens, bt_h, lens_h = gpu_step(wl)
+    NB = kc.shape[0]
+    perm = torch.randperm(NB, generator=torch.Generator().manual_seed(9))
+    inv = torch.empty_like(perm)
+    inv[perm] = torch.arange(NB)
+    kc2 = torch.empty_like(kc)
+    vc2 = torch.empty_like(vc)
+    kc2[perm.cuda()] = kc
+    vc2[perm.cuda()] = vc
+    bt2 = torch.from_numpy(np.where(bt_h >= 0, perm.numpy()[np.maximum(bt_h, 0)], -1).astype(np.int32)).cuda()
+    out2 = pa.decode(wl.q.cuda(), kc2, vc2, bt2, lens, int(lens_h.max()), wl.scale)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+
+
+def test_decode_large_logits():
+    """q scaled x10: logits far outside fp16 softmax's comfortable range; fp32 softmax keeps parity."""
+    wl = make_workload("qwen_decode", q_scale=10.0)
+    out, *_ = gpu_step(wl)
+    ref = _oracle_decode(wl)
+    got = out.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    assert_close(got, ref, "q x10")

@@ -8,6 +8,6 @@ CPU oracle and the CUDA path start from what it returns and derive everything
 else on their own.
 """
 
-from .synth import CONFIGS, Workload, make_workload, fill_cache_blocks, ops_for
+from .synth import CONFIGS, Workload, fill_cache_blocks, make_custom, make_workload, ops_for
 
-__all__ = ["CONFIGS", "Workload", "make_workload", "fill_cache_blocks", "ops_for"]
+__all__ = ["CONFIGS", "Workload", "make_workload", "make_custom", "fill_cache_blocks", "ops_for"]

@@ -174,3 +174,45 @@ def fill_cache_blocks(shape, dtype: str, seed: int) -> torch.Tensor:
     """A standalone N(0,1) cache tensor (used by tests that need a fresh pool)."""
     g = torch.Generator().manual_seed(int(seed))
     return _randn(g, shape, TORCH_DTYPES[dtype])
+
+
+def make_custom(*, seed: int, lens, num_q_heads: int, num_kv_heads: int, head_dim: int, block_size: int,
+                dtype: str = "bf16", kind: str = "decode", chunk_lens=None, free_frac: float = 0.25,
+                q_scale: float = 1.0) -> Workload:
+    """A small workload with explicit per-sequence lengths (ragged edge cases).
+
+    kind="decode": ``lens`` are context lengths after the write (0 allowed: that sequence writes nothing).
+    kind="prefill": ``lens`` are the final lengths and ``chunk_lens`` the chunk appended to each.
+    """
+    g = torch.Generator().manual_seed(int(seed))
+    L = np.asarray(lens, dtype=np.int32)
+    B = len(L)
+    if kind == "decode":
+        new = (L > 0).astype(np.int32)
+    else:
+        new = np.asarray(chunk_lens, dtype=np.int32)
+    before = (L - new).astype(np.int32)
+    NB = int(math.ceil((int(L.sum()) / block_size + B + 1) * (1.0 + free_frac)))
+    free_order = torch.randperm(NB, generator=g).numpy().astype(np.int32)
+    T = int(new.sum())
+    dt = TORCH_DTYPES[dtype]
+    nq = B if kind == "decode" else T
+    q = _randn(g, (nq, num_q_heads, head_dim), dt)
+    if q_scale != 1.0:
+        q = (q.float() * q_scale).to(dt)
+    k_new = _randn(g, (T, num_kv_heads, head_dim), dt)
+    v_new = _randn(g, (T, num_kv_heads, head_dim), dt)
+    k_cache0 = _randn(g, (NB, block_size, num_kv_heads, head_dim), dt)
+    v_cache0 = _randn(g, (NB, block_size, num_kv_heads, head_dim), dt)
+    ops = [("alloc", b, int(before[b])) for b in range(B)]
+    ops += [("append_new", b, int(new[b])) for b in range(B) if new[b] > 0]
+    qsl = None
+    if kind == "prefill":
+        qsl = np.zeros(B + 1, dtype=np.int32)
+        qsl[1:] = np.cumsum(new)
+    cfg = dict(kind=kind, batch=B, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads, head_dim=head_dim,
+               block_size=block_size, dtype=dtype, seed=seed)
+    scale = float(np.float32(1.0) / np.sqrt(np.float32(head_dim)))
+    return Workload(name="custom", cfg=cfg, ops=ops, free_order=free_order, num_blocks=NB, context_lens=L, q=q,
+                    k_new=k_new, v_new=v_new, k_cache0=k_cache0, v_cache0=v_cache0, query_start_loc=qsl,
+                    scale=scale)
