@@ -240,7 +240,7 @@ def run_ours(args):
     _, bt, lens, sm, _ = pa.replay_ops(wl.ops, wl.num_blocks, c["block_size"], wl.free_order, wl.batch)
     maxL = int(lens.max())
     B, Hq, Hkv, D = wl.batch, c["num_q_heads"], c["num_kv_heads"], c["head_dim"]
-    sl, msplit, wsb = pa.decode_plan(B, Hq, Hkv, D, maxL, args.num_splits)
+    grid, maxp, wsb = pa.decode_plan(B, Hq, Hkv, D, maxL, args.num_partitions)
 
     # device-resident inputs
     kc = wl.k_cache0.to(dev)
@@ -258,7 +258,7 @@ def run_ours(args):
         pa.write_kv(kn, vn, smd, kc, vc, stream=stream)
         if ev_pair is not None:
             ev_pair[0].record(stream)
-        pa.decode(q, kc, vc, btd, lensd, maxL, wl.scale, out=out, workspace=work, num_splits=args.num_splits,
+        pa.decode(q, kc, vc, btd, lensd, maxL, wl.scale, out=out, workspace=work, num_partitions=args.num_partitions,
                   stream=stream)
         if ev_pair is not None:
             ev_pair[1].record(stream)
@@ -337,7 +337,7 @@ def run_ours(args):
     achieved = alg / (dec_avg * 1e-3) / 1e9
     tr = NCU_TRAFFIC.get(args.workload)
     traffic = tr["bytes"] if tr and tr.get("src") == kernel_source_hash() else None
-    launches_per_step = 1 + 1 + (1 if msplit > 1 else 0)
+    launches_per_step = 3  # write_kv, decode, split-K reduce
     if rank == 0:
         cpu = None
         if ws == 1 and not args.no_cpu_baseline:
@@ -350,7 +350,7 @@ def run_ours(args):
             "dtype": str(c["dtype"]), "data": "synthetic",
             "config": {"workload": WORKLOAD_TEXT.get(args.workload, args.workload), "global_batch": int(seqs_all),
                        "parallelism": f"dp{ws} (independent replicas)", "l2": "inputs larger than L2 (no flush)",
-                       "split_len": sl, "max_splits": msplit},
+                       "decode_grid": grid},
             "tokens_per_s": seqs_all / (ms_step * 1e-3),
             "pct_hbm_peak": {"of_measured": value / ws / peak if peak_kind == "measured" else None,
                              "of_nominal_8000": value / ws / 8000.0},
@@ -377,7 +377,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen_decode", choices=sorted(WORKLOAD_TEXT))
-    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--num-partitions", type=int, default=0, help="decode CTAs (0 = fill the GPU)")
     ap.add_argument("--ref-budget", type=float, default=12.0, help="seconds of oracle time per reference sample")
     ap.add_argument("--ref-seqs", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")

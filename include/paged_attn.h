@@ -106,33 +106,37 @@ int pa_copy_blocks(const int32_t* pairs, int num_pairs, void* k_cache, void* v_c
 /* Paged decode (P1 s2.2.1, s4.2; P2 s2.2, s3.1): one query token per        */
 /* sequence attends to all context_lens[b] tokens of its sequence:           */
 /*   out[b][h] = sum_t softmax_t(scale * <q[b][h], K_b[t][h/G]>) V_b[t][h/G] */
-/* The context of each sequence is cut into splits of `split_len` tokens     */
-/* (split-K); each split yields fp32 (max, sum, weighted V), merged by a     */
-/* log-sum-exp reduce kernel.  A sequence that fits one split is written     */
-/* directly.  context_lens[b] == 0 gives out[b] = 0.                         */
+/* context_lens[b] == 0 gives out[b] = 0.                                    */
 /*                                                                           */
-/* pa_decode_plan: the split length and workspace the call will use for     */
-/* these sizes.  num_splits_or_0 > 0 forces about that many splits for the  */
-/* longest sequence; 0 picks the split length from the batch shape.         */
-/* Any output pointer may be NULL.                                           */
+/* Work split (split-K, P3 s3.1 read on one device): every (sequence, KV     */
+/* head) is cut into 16-token chunks; all chunks, end to end, are shared out */
+/* evenly over `grid` persistent CTAs.  The part of a sequence's context     */
+/* that one CTA handles yields fp32 (max, sum, weighted V) in the workspace  */
+/* unless it is the whole context; a reduce kernel merges the parts by the   */
+/* log-sum-exp rule.  Two kernels are launched per call.                     */
+/*                                                                           */
+/* pa_decode_plan: the grid and workspace the call will use on the current   */
+/* device.  num_partitions_or_0 > 0 fixes the number of CTAs (the number of  */
+/* parts the chunk line is cut into); 0 fills the GPU (SMs x CTAs per SM).   */
+/* max_context_len is only checked here (>= 0).  Output pointers may be NULL.*/
 /* ------------------------------------------------------------------------ */
 int pa_decode_plan(int batch, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len,
-                   int num_splits_or_0, int* split_len_out, int* max_splits_out, size_t* workspace_bytes_out);
+                   int num_partitions_or_0, int* grid_out, int* max_pieces_out, size_t* workspace_bytes_out);
 
 /* Bytes of device workspace pa_decode needs for these sizes (0 on bad args). */
 size_t pa_decode_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
-                                int max_context_len, int num_splits_or_0);
+                                int max_context_len, int num_partitions_or_0);
 
 /* q: [batch][num_q_heads][head_dim]; out: same shape; caches as above.      */
-/* max_context_len: host-side upper bound of context_lens (sizes the grid).  */
+/* max_context_len: host-side upper bound of context_lens; block_tables rows */
+/* must cover it (max_blocks_per_seq * block_size >= max_context_len).       */
 /* workspace: device scratch of >= pa_decode_workspace_size() bytes, 256-byte */
-/* aligned, owned by the caller, contents need no initialisation; it may be  */
-/* NULL when every sequence fits one split (max_context_len <= split_len).   */
+/* aligned, owned by the caller; its contents need no initialisation.        */
 /* Two calls that run at the same time must use different workspaces.        */
 int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
               int max_blocks_per_seq, const int32_t* context_lens, int batch, int num_q_heads,
               int num_kv_heads, int head_dim, int block_size, int num_blocks, int max_context_len,
-              float scale, int dtype, void* workspace, size_t workspace_bytes, int num_splits_or_0,
+              float scale, int dtype, void* workspace, size_t workspace_bytes, int num_partitions_or_0,
               void* out, void* stream);
 
 /* ------------------------------------------------------------------------ */

@@ -140,16 +140,16 @@ def copy_blocks(pairs, k_cache, v_cache, stream=None) -> None:
                               _dtype_code(k_cache), _stream_handle(stream)), "pa_copy_blocks")
 
 
-def decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_splits=0):
-    """(split_len, max_splits, workspace_bytes) the decode call will use."""
-    sl, ms, ws = ctypes.c_int(), ctypes.c_int(), ctypes.c_size_t()
-    _check(lib.pa_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_splits,
-                              ctypes.byref(sl), ctypes.byref(ms), ctypes.byref(ws)), "pa_decode_plan")
-    return sl.value, ms.value, ws.value
+def decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_partitions=0):
+    """(grid, max_pieces, workspace_bytes) the decode call will use on the current device."""
+    gr, mp, ws = ctypes.c_int(), ctypes.c_int(), ctypes.c_size_t()
+    _check(lib.pa_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_partitions,
+                              ctypes.byref(gr), ctypes.byref(mp), ctypes.byref(ws)), "pa_decode_plan")
+    return gr.value, mp.value, ws.value
 
 
 def decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float, out=None,
-           workspace=None, num_splits: int = 0, stream=None):
+           workspace=None, num_partitions: int = 0, stream=None):
     """q [B, Hq, D]; block_tables int32 [B, max_blocks]; context_lens int32 [B]. Returns out [B, Hq, D]."""
     torch = _torch()
     _contig(q, k_cache, v_cache, block_tables, context_lens, out, workspace)
@@ -157,13 +157,13 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len: int
     NB, bs, Hkv, _ = k_cache.shape
     if out is None:
         out = torch.empty_like(q)
-    _, _, need = decode_plan(B, Hq, Hkv, D, max_context_len, num_splits)
-    if workspace is None and need > 0:
+    _, _, need = decode_plan(B, Hq, Hkv, D, max_context_len, num_partitions)
+    if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.pa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), int(block_tables.shape[1]),
                          _ptr(context_lens), B, Hq, Hkv, D, bs, NB, int(max_context_len), float(scale),
-                         _dtype_code(q), _ptr(workspace), ws_bytes, int(num_splits), _ptr(out),
+                         _dtype_code(q), _ptr(workspace), ws_bytes, int(num_partitions), _ptr(out),
                          _stream_handle(stream)), "pa_decode")
     return out
 

@@ -1,4 +1,4 @@
-// Paged decode attention, split-K, for sm_100a.
+// Paged decode attention for sm_100a: persistent, evenly partitioned split-K.
 //
 // What it computes (page "Nano-vLLM-Ascend: lightweight LLM inference
 // framework for Ascend NPU", section 2.2.1 attention = softmax(q k^T/sqrt(d)) v
@@ -9,29 +9,33 @@
 // where token t of sequence b lives in physical block block_tables[b][t/bs],
 // row t%bs of the cache.
 //
-// Work split.  One CTA per (sequence b, KV head g, split s); a split is
-// `split_len` consecutive tokens (a multiple of 64), so long contexts spread
-// over many SMs (the single-device reading of the context-parallel split on
-// "In-depth analysis of vllm-ascend", section 3.1).  All G query heads of the
-// group share every K/V tile the CTA loads.
+// Work split.  A segment is one (sequence b, KV head g); it holds
+// ceil(L_b/16) chunks of 16 tokens.  All segments, laid end to end in (b, g)
+// order, form one line of C chunks.  CTA c of the persistent grid takes chunks
+// [C*c/grid, C*(c+1)/grid): every CTA reads the same number of KV bytes,
+// whatever the length mix.  The part of a segment that falls in one CTA is a
+// piece; a piece that is a whole segment writes `out` directly, otherwise it
+// writes fp32 (max, sum, acc) to the workspace and the reduce kernel merges a
+// segment's pieces by the log-sum-exp rule.  This is the single-device reading
+// of the context split on "In-depth analysis of vllm-ascend", section 3.1.
 //
-// Data movement.  One producer warp gathers 16-row K and V boxes through the
-// block table with TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast)
-// into an NSTAGES-deep shared-memory ring guarded by mbarriers (the pages'
-// prefetch-depth / pipeline-stage lesson, vLLM-Ascend page section 2.2).
-// NW consumer warps each take 32 tokens of every stage.
+// Data movement.  One producer warp walks the CTA's chunk range, looks up each
+// chunk's physical block (one lookup ahead) and gathers 16-row K and V boxes
+// with TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast) into an
+// NSTAGES-deep shared-memory ring guarded by mbarriers, straight across piece
+// and segment boundaries (the pages' prefetch-depth / pipeline-stage lesson,
+// vLLM-Ascend page section 2.2).  Each stage also carries a small descriptor
+// and, at a piece's first stage, the G query rows of the group (bulk copy).
+// NW consumer warps take 32 tokens of every stage each.
 //
-// Math.  fp32 scores in the log2 domain (scale*log2(e) folded into q),
-// online softmax with fp32 running max and sum, fp32 accumulators.
-//   * G <= 4: CUDA cores.  QK^T: lane = token, full dot product per lane;
-//     row max/sum by warp shuffles; PV: lane = slice of head_dim.
-//   * G >= 8: the FP32 pipe cannot keep up with HBM at 8 flop per KV byte,
-//     so QK^T and PV use warp-level mma.m16n8k16 (bf16/f16 in, fp32 out) with
-//     the G query heads as rows; softmax rows are reduced with quad shuffles.
-// Each consumer warp keeps its own (max, sum, acc); the warps merge through
-// shared memory at the end.  A sequence that fits one split writes `out`
-// directly; otherwise the split writes fp32 (max, sum, acc) to the workspace
-// and a reduce kernel merges splits by the log-sum-exp rule.
+// Math.  fp32 scores in the log2 domain (scale*log2(e)), online softmax with
+// fp32 running max and sum, fp32 accumulators.
+//   * G <= 4: CUDA cores.  QK^T: lane = token, one full dot product per lane;
+//     max/sum by warp shuffles; PV: lane = slice of head_dim.
+//   * G >= 8: the FP32 pipe cannot keep up with HBM at 8 flop per KV byte, so
+//     QK^T and PV use warp-level mma.m16n8k16 (bf16/f16 in, fp32 out) with the
+//     G query heads as rows.  P enters PV as two 16-bit terms (hi + lo), which
+//     keeps it exact to about 2^-17 instead of the 2^-9 of one bf16 rounding.
 
 #include <algorithm>
 #include <type_traits>
@@ -46,46 +50,54 @@ namespace {
 using namespace pa;
 
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kChunk = 16;  // tokens per chunk = rows per TMA box
 
 struct DecodeParams {
   const void* q;
   void* out;
   const int32_t* block_tables;
   const int32_t* context_lens;
-  float* ws_m;  // [B][Hq][max_splits]  running max (log2 domain)
-  float* ws_l;  // [B][Hq][max_splits]  sum of exp2(x - m)
-  float* ws_o;  // [B][Hq][max_splits][D] sum of exp2(x - m) * v
+  long long* ws_pre;  // [B+1] chunks before sequence b (written by CTA 0)
+  float* ws_m;        // [nslots][G] running max of a piece (log2 domain)
+  float* ws_l;        // [nslots][G] sum of exp2(x - m)
+  float* ws_o;        // [nslots][G][D] sum of exp2(x - m) * v
   int max_blocks_per_seq;
   int batch;
   int num_q_heads;
   int num_kv_heads;
   int block_size;
   int num_blocks;
-  int split_len;
-  int max_splits;
+  int grid;
   float scale_log2;
 };
 
-template <int D, int G, int NW, int NSTAGES>
+enum : int { F_FIRST = 1, F_LAST = 2, F_DIRECT = 4, F_END = 8 };
+
+struct StageMeta {
+  int b, g, tok0, ntok, flags, slot, nchunk, pad;
+};
+
+template <int D, int G, int NW, int NSTAGES, bool MMA>
 struct Layout {
-  static constexpr int TOK = NW * 32;                 // tokens per stage
-  static constexpr int HALVES = D / 64;               // 128-byte column boxes per row
-  static constexpr int STAGE_BYTES = TOK * D * 2;     // K (or V) bytes per stage
-  static constexpr int BOXES = TOK / 16;              // 16-row boxes per stage
+  static constexpr int TOK = NW * 32;             // tokens per stage
+  static constexpr int CPS = TOK / kChunk;        // chunks (16-row boxes) per stage
+  static constexpr int HALVES = D / 64;           // 128-byte column boxes per row
+  static constexpr int STAGE_BYTES = TOK * D * 2; // K (or V) bytes per stage
+  static constexpr int QSLOT = G * D * 2;         // the group's q rows
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + NSTAGES * STAGE_BYTES;
-  static constexpr int Q_OFF = V_OFF + NSTAGES * STAGE_BYTES;           // fp32 [G][D]
-  static constexpr int P_OFF = Q_OFF + G * D * 4;                       // fp32 [NW][32][G]
-  static constexpr int BT_OFF = P_OFF + NW * 32 * G * 4;                // int32 [BT_MAX]
-  // merge area, fp32 [NW][G][D] then [NW][G][2]; aliases the stage buffers,
-  // which are free once every consumer has passed the pipeline
-  static constexpr int M_OFF = K_OFF;
-  static constexpr int ML_OFF = M_OFF + NW * G * D * 4;
-  static_assert(ML_OFF + NW * G * 2 * 4 <= Q_OFF, "merge area must fit in the stage buffers");
-  static constexpr int BT_MAX = 512;                                    // block-table entries per split
-  static constexpr int BAR_OFF = BT_OFF + BT_MAX * 4;                   // uint64 full[NSTAGES], empty[NSTAGES]
+  static constexpr int QS_OFF = V_OFF + NSTAGES * STAGE_BYTES;
+  static constexpr int META_OFF = QS_OFF + NSTAGES * QSLOT;
+  static constexpr int QF_OFF = META_OFF + NSTAGES * (int)sizeof(StageMeta);  // fp32 q per warp (CUDA-core path)
+  static constexpr int QF_BYTES = MMA ? 0 : NW * G * D * 4;
+  static constexpr int P_OFF = QF_OFF + QF_BYTES;                             // fp32 p per warp (CUDA-core path)
+  static constexpr int P_BYTES = MMA ? 0 : NW * 32 * G * 4;
+  static constexpr int M_OFF = P_OFF + P_BYTES;                               // merge: fp32 [NW][G][D]
+  static constexpr int ML_OFF = M_OFF + NW * G * D * 4;                       // merge: fp32 [NW][G][2]
+  static constexpr int BAR_OFF = ML_OFF + NW * G * 2 * 4;                     // full[NSTAGES], empty[NSTAGES]
   static constexpr int BYTES = BAR_OFF + 2 * NSTAGES * 8;
-  static constexpr int ALLOC = BYTES + 1024;                            // slack for 1024-byte alignment
+  static constexpr int ALLOC = BYTES + 1024;                                  // slack for 1024-byte alignment
+  static_assert(QS_OFF % 16 == 0 && QSLOT % 16 == 0 && BAR_OFF % 8 == 0, "alignment");
 };
 
 // Address of element (row r, column d) inside a stage buffer laid out as
@@ -153,11 +165,32 @@ __device__ __forceinline__ float warp_sum(float v) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
+__device__ __forceinline__ long long warp_sum_ll(long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ long long warp_incl_scan_ll(long long v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long t = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += t;
+  }
+  return v;
+}
+
+// 1-D bulk copy global -> shared, completion in bytes on an mbarrier (no multicast).
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(smem_dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
 
 // ------------------------------------------------------------------ CUDA-core consumer (G <= 4)
 template <int DT, int D, int G, int NW, int NSTAGES>
 struct CoreConsumer {
-  using LY = Layout<D, G, NW, NSTAGES>;
+  using LY = Layout<D, G, NW, NSTAGES, false>;
   static constexpr int DPL = D / 32;  // head_dim elements per lane in PV
   float m[G], l[G], o[G][DPL];
 
@@ -169,6 +202,17 @@ struct CoreConsumer {
 #pragma unroll
       for (int j = 0; j < DPL; ++j) o[h][j] = 0.f;
     }
+  }
+
+  // The group's q rows (16-bit, [G][D]) -> this warp's fp32 copy scaled by scale*log2(e).
+  __device__ __forceinline__ void load_q(const uint8_t* qslot, float* qf, float scale_log2, int lane) {
+    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qslot);
+    for (int i = lane; i < G * D / 2; i += 32) {
+      const float2 f = Elt<DT>::to_f2(q32[i]);
+      qf[2 * i] = f.x * scale_log2;
+      qf[2 * i + 1] = f.y * scale_log2;
+    }
+    __syncwarp();
   }
 
   // One 32-token tile: rows r0 .. r0+31 of the stage, nv of them valid.
@@ -274,23 +318,23 @@ struct CoreConsumer {
 // ------------------------------------------------------------------ tensor-core consumer (G >= 8)
 template <int DT, int D, int G, int NW, int NSTAGES>
 struct MmaConsumer {
-  using LY = Layout<D, G, NW, NSTAGES>;
+  using LY = Layout<D, G, NW, NSTAGES, true>;
   static constexpr int KS = D / 16;   // k-steps of QK^T
   static constexpr int ND = D / 8;    // n-tiles of PV
   uint32_t qa[KS][4];                 // A fragments of q (rows = heads, padded to 16)
   float o[ND][4];                     // rows lane/4 and lane/4+8, columns of an n-tile
   float m[2], l[2];                   // per row owned by this thread (lane/4, lane/4+8); l is a partial sum
 
-  __device__ __forceinline__ void load_q(const typename Elt<DT>::T* qg, int lane) {
+  __device__ __forceinline__ void load_q(const uint8_t* qslot, float*, float, int lane) {
     const int r0 = lane >> 2, r1 = r0 + 8;
-    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qg);
+    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qslot);
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
       const int c = ks * 16 + (lane & 3) * 2;
-      qa[ks][0] = r0 < G ? __ldg(q32 + (r0 * D + c) / 2) : 0u;
-      qa[ks][1] = r1 < G ? __ldg(q32 + (r1 * D + c) / 2) : 0u;
-      qa[ks][2] = r0 < G ? __ldg(q32 + (r0 * D + c + 8) / 2) : 0u;
-      qa[ks][3] = r1 < G ? __ldg(q32 + (r1 * D + c + 8) / 2) : 0u;
+      qa[ks][0] = r0 < G ? q32[(r0 * D + c) / 2] : 0u;
+      qa[ks][1] = r1 < G ? q32[(r1 * D + c) / 2] : 0u;
+      qa[ks][2] = r0 < G ? q32[(r0 * D + c + 8) / 2] : 0u;
+      qa[ks][3] = r1 < G ? q32[(r1 * D + c + 8) / 2] : 0u;
     }
   }
 
@@ -299,6 +343,13 @@ struct MmaConsumer {
     l[0] = l[1] = 0.f;
 #pragma unroll
     for (int n = 0; n < ND; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  }
+
+  template <int DT2 = DT>
+  static __device__ __forceinline__ void split_hi_lo(float a, float b, uint32_t& hi, uint32_t& lo) {
+    hi = Elt<DT2>::from_f2(a, b);
+    const float2 h = Elt<DT2>::to_f2(hi);
+    lo = Elt<DT2>::from_f2(a - h.x, b - h.y);
   }
 
   __device__ __forceinline__ void tile(uint32_t kbase, uint32_t vbase, float scale_log2, int r0, int nv, int lane) {
@@ -341,15 +392,15 @@ struct MmaConsumer {
     m[0] = mn0;
     m[1] = mn1;
     float ls0 = 0.f, ls1 = 0.f;
-    uint32_t pa[2][4];  // A fragments of P for the two 16-token k-steps
+    uint32_t ph[2][4], pl[2][4];  // A fragments of P = hi + lo for the two 16-token k-steps
 #pragma unroll
     for (int n = 0; n < 4; ++n) {
       const float p0 = fast_exp2(s[n][0] - mn0), p1 = fast_exp2(s[n][1] - mn0);
       const float p2 = fast_exp2(s[n][2] - mn1), p3 = fast_exp2(s[n][3] - mn1);
       ls0 += p0 + p1;
       ls1 += p2 + p3;
-      pa[n >> 1][(n & 1) * 2 + 0] = Elt<DT>::from_f2(p0, p1);
-      pa[n >> 1][(n & 1) * 2 + 1] = Elt<DT>::from_f2(p2, p3);
+      split_hi_lo(p0, p1, ph[n >> 1][(n & 1) * 2 + 0], pl[n >> 1][(n & 1) * 2 + 0]);
+      split_hi_lo(p2, p3, ph[n >> 1][(n & 1) * 2 + 1], pl[n >> 1][(n & 1) * 2 + 1]);
     }
     l[0] = l[0] * al0 + ls0;
     l[1] = l[1] * al1 + ls1;
@@ -375,8 +426,10 @@ struct MmaConsumer {
           b0 &= lo0; b2 &= lo0;
           b1 &= lo1; b3 &= lo1;
         }
-        mma16816<DT>(o[dp * 2], pa[j][0], pa[j][1], pa[j][2], pa[j][3], b0, b1);
-        mma16816<DT>(o[dp * 2 + 1], pa[j][0], pa[j][1], pa[j][2], pa[j][3], b2, b3);
+        mma16816<DT>(o[dp * 2], ph[j][0], ph[j][1], ph[j][2], ph[j][3], b0, b1);
+        mma16816<DT>(o[dp * 2 + 1], ph[j][0], ph[j][1], ph[j][2], ph[j][3], b2, b3);
+        mma16816<DT>(o[dp * 2], pl[j][0], pl[j][1], pl[j][2], pl[j][3], b0, b1);
+        mma16816<DT>(o[dp * 2 + 1], pl[j][0], pl[j][1], pl[j][2], pl[j][3], b2, b3);
       }
     }
   }
@@ -402,48 +455,87 @@ struct MmaConsumer {
   }
 };
 
-// ------------------------------------------------------------------ split kernel
+// ------------------------------------------------------------------ producer: walk of a CTA's chunk range
+// Lane-uniform state (every lane of the producer warp holds the same values).
+struct Walker {
+  long long pos, end;         // current chunk, end of this CTA's range (global chunk line)
+  long long seg_start;        // first chunk of the current segment
+  long long piece_start;      // first chunk of the current piece
+  int b, g, L, nch;           // current segment: sequence, KV head, clamped length, chunks
+  int win_base, win_len;      // lens window: lane i holds the clamped length of sequence win_base + i
+  int batch, hkv, cap;
+  const int32_t* lens;
+};
+
+__device__ __forceinline__ int clamp_len(int L, int cap) { return L < 0 ? 0 : (L > cap ? cap : L); }
+
+__device__ __forceinline__ void load_window(Walker& w, int base, int lane) {
+  w.win_base = base;
+  const int i = base + lane;
+  w.win_len = i < w.batch ? clamp_len(__ldg(w.lens + i), w.cap) : 0;
+}
+
+// Move to the next sequence with at least one chunk (b must stay < batch while chunks remain).
+__device__ __forceinline__ void next_sequence(Walker& w, int lane) {
+  for (;;) {
+    w.b += 1;
+    if (w.b >= w.batch) return;
+    if (w.b - w.win_base >= 32) load_window(w, w.b, lane);
+    w.L = __shfl_sync(0xffffffffu, w.win_len, w.b - w.win_base);
+    w.nch = (w.L + kChunk - 1) / kChunk;
+    if (w.nch > 0) return;
+  }
+}
+
+template <int CPS>
+__device__ __forceinline__ StageMeta walker_next(Walker& w, int cta, int lane) {
+  StageMeta d;
+  if (w.pos >= w.end) {
+    d.flags = F_END;
+    d.b = d.g = d.tok0 = d.ntok = d.slot = d.nchunk = d.pad = 0;
+    return d;
+  }
+  const long long seg_end = w.seg_start + w.nch;
+  const long long piece_end = seg_end < w.end ? seg_end : w.end;
+  long long stop = w.pos + CPS;
+  if (stop > piece_end) stop = piece_end;
+  d.b = w.b;
+  d.g = w.g;
+  d.tok0 = (int)(w.pos - w.seg_start) * kChunk;
+  const int tok1 = min((int)(stop - w.seg_start) * kChunk, w.L);
+  d.ntok = tok1 - d.tok0;
+  d.nchunk = (int)(stop - w.pos);
+  d.flags = (w.pos == w.piece_start ? F_FIRST : 0) | (stop == piece_end ? F_LAST : 0) |
+            (w.piece_start == w.seg_start && piece_end == seg_end ? F_DIRECT : 0);
+  d.slot = w.b * w.hkv + w.g + cta;
+  d.pad = 0;
+  w.pos = stop;
+  if (stop == piece_end && stop < w.end) {  // next piece starts a new segment
+    w.piece_start = stop;
+    w.seg_start = seg_end;
+    if (++w.g == w.hkv) {
+      w.g = 0;
+      next_sequence(w, lane);
+    }
+  }
+  return d;
+}
+
+// ------------------------------------------------------------------ decode kernel
 template <int DT, int D, int G, int NW, int NSTAGES, bool MMA>
-__global__ void __launch_bounds__((NW + 1) * 32) decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
-                                                                     const __grid_constant__ CUtensorMap vmap,
-                                                                     const DecodeParams p) {
-  using LY = Layout<D, G, NW, NSTAGES>;
+__global__ void __launch_bounds__((NW + 1) * 32) decode_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                               const __grid_constant__ CUtensorMap vmap,
+                                                               const DecodeParams p) {
+  using LY = Layout<D, G, NW, NSTAGES, MMA>;
   using T = typename Elt<DT>::T;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + LY::BAR_OFF);
   uint64_t* empty = full + NSTAGES;
-  int32_t* bt_s = reinterpret_cast<int32_t*>(smem + LY::BT_OFF);
-
-  const int Hkv = p.num_kv_heads;
-  const int u = blockIdx.x;
-  const int g = u % Hkv;
-  const int s = (u / Hkv) % p.max_splits;
-  const int b = u / (Hkv * p.max_splits);
+  StageMeta* meta = reinterpret_cast<StageMeta*>(smem + LY::META_OFF);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  int L = __ldg(p.context_lens + b);
-  {  // a length beyond what the grid or the block-table row covers is a caller error: clamp and record
-    const int cap = min(p.max_splits * p.split_len, p.max_blocks_per_seq * p.block_size);
-    if (L < 0 || L > cap) {
-      if (threadIdx.x == 0 && s == 0 && g == 0) PA_RECORD_ERROR(PA_ERRBIT_INDEX);
-      L = L < 0 ? 0 : cap;
-    }
-  }
-  const int t0 = s * p.split_len;
-  if (t0 >= L) {
-    if (s == 0) {  // empty sequence: out = 0 (documented)
-      T* ob = reinterpret_cast<T*>(p.out) + ((size_t)b * p.num_q_heads + (size_t)g * G) * D;
-      for (int i = threadIdx.x; i < G * D; i += blockDim.x) ob[i] = Elt<DT>::from_f(0.f);
-    }
-    return;
-  }
-  const int t1 = min(L, t0 + p.split_len);
-  const int nsplit = (L + p.split_len - 1) / p.split_len;
-  const int nstages = (t1 - t0 + LY::TOK - 1) / LY::TOK;
-  const int first_blk = t0 / p.block_size;
-  const int nblk = (t1 - 1) / p.block_size - first_blk + 1;
+  const int cta = blockIdx.x;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NSTAGES; ++i) {
@@ -452,67 +544,165 @@ __global__ void __launch_bounds__((NW + 1) * 32) decode_split_kernel(const __gri
     }
     fence_mbar_init();
   }
-  const T* qg = reinterpret_cast<const T*>(p.q) + ((size_t)b * p.num_q_heads + (size_t)g * G) * D;
-  if (warp == NW) {
-    tma_prefetch_desc(&kmap);
-    tma_prefetch_desc(&vmap);
-    const int32_t* bt = p.block_tables + (size_t)b * p.max_blocks_per_seq + first_blk;
-    for (int i = lane; i < nblk; i += 32) bt_s[i] = __ldg(bt + i);
-  } else if constexpr (!MMA) {
-    float* q_s = reinterpret_cast<float*>(smem + LY::Q_OFF);
-    for (int i = threadIdx.x; i < G * D; i += NW * 32) q_s[i] = (float)qg[i] * p.scale_log2;
-  }
   __syncthreads();
 
   if (warp == NW) {
-    // ------------------------------------------------ producer: TMA gather through the block table
-    bool ok = true;
-    for (int k = 0; k < nstages && ok; ++k) {
-      const int st = k % NSTAGES;
-      if (k >= NSTAGES) ok = mbar_wait(&empty[st], ((k / NSTAGES) - 1) & 1);
-      if (!ok) break;
-      const int tok_base = t0 + k * LY::TOK;
-      const int nbox = min(LY::BOXES, (t1 - tok_base + 15) >> 4);
-      if (lane == 0) mbar_arrive_expect_tx(&full[st], (uint32_t)(nbox * 16 * D * 2 * 2));
-      __syncwarp();
-      if (lane < nbox) {
-        const int tok = tok_base + lane * 16;
-        const int phys = bt_s[tok / p.block_size - first_blk];
-        if (phys < 0 || phys >= p.num_blocks) PA_RECORD_ERROR(PA_ERRBIT_INDEX);  // TMA zero-fills out of range
-        const int y = phys * p.block_size + (tok % p.block_size);
-        uint8_t* kd = smem + LY::K_OFF + st * LY::STAGE_BYTES + lane * 16 * 128;
-        uint8_t* vd = smem + LY::V_OFF + st * LY::STAGE_BYTES + lane * 16 * 128;
+    // ================================================= producer warp
+    const int B = p.batch, Hkv = p.num_kv_heads;
+    const int cap = p.max_blocks_per_seq * p.block_size;
+    // pass 1: total chunks over all sequences
+    long long tot = 0;
+    bool clamped = false;
+    for (int base = 0; base < B; base += 256) {
+      long long s = 0;
 #pragma unroll
-        for (int h = 0; h < LY::HALVES; ++h) {
-          tma_load_2d(kd + h * LY::TOK * 128, &kmap, g * D + h * 64, y, &full[st]);
-          tma_load_2d(vd + h * LY::TOK * 128, &vmap, g * D + h * 64, y, &full[st]);
+      for (int j = 0; j < 8; ++j) {
+        const int i = base + lane * 8 + j;
+        if (i < B) {
+          const int L = __ldg(p.context_lens + i);
+          clamped |= (L < 0 || L > cap);
+          s += (clamp_len(L, cap) + kChunk - 1) / kChunk;
         }
       }
+      tot += warp_sum_ll(s);
+    }
+    if (clamped && cta == 0 && lane == 0) PA_RECORD_ERROR(PA_ERRBIT_INDEX);
+    const long long C = tot * Hkv;
+    const long long x0 = C * cta / p.grid, x1 = C * (cta + 1) / p.grid;
+    // pass 2: the sequence holding chunk x0 (CTA 0 also publishes the prefix sums for the reduce)
+    Walker w;
+    w.pos = x0;
+    w.end = x1;
+    w.batch = B;
+    w.hkv = Hkv;
+    w.cap = cap;
+    w.lens = p.context_lens;
+    int fb = -1;
+    long long fpre = 0;
+    {
+      long long run = 0;
+      for (int base = 0; base < B; base += 256) {
+        int v[8];
+        long long s = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int i = base + lane * 8 + j;
+          v[j] = i < B ? (clamp_len(__ldg(p.context_lens + i), cap) + kChunk - 1) / kChunk : 0;
+          s += v[j];
+        }
+        const long long incl = warp_incl_scan_ll(s, lane);
+        long long pre = run + incl - s;
+        int found = -1;
+        long long found_pre = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int i = base + lane * 8 + j;
+          if (i < B) {
+            if (cta == 0) p.ws_pre[i] = pre;
+            if (v[j] > 0 && pre * Hkv <= x0 && x0 < (pre + v[j]) * Hkv) {
+              found = i;
+              found_pre = pre;
+            }
+          }
+          pre += v[j];
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, found >= 0);
+        if (hit && fb < 0) {
+          const int src = __ffs(hit) - 1;
+          fb = __shfl_sync(0xffffffffu, found, src);
+          fpre = __shfl_sync(0xffffffffu, found_pre, src);
+        }
+        run += __shfl_sync(0xffffffffu, incl, 31);
+        if (fb >= 0 && cta != 0) break;
+      }
+      if (cta == 0 && lane == 0) p.ws_pre[B] = tot;
+    }
+    if (x0 < x1) {
+      load_window(w, fb, lane);
+      w.b = fb;
+      w.L = __shfl_sync(0xffffffffu, w.win_len, 0);
+      w.nch = (w.L + kChunk - 1) / kChunk;
+      w.g = (int)((x0 - fpre * Hkv) / w.nch);
+      w.seg_start = fpre * Hkv + (long long)w.g * w.nch;
+      w.piece_start = x0;
+    }
+    const int32_t* bt_all = p.block_tables;
+    const int mb = p.max_blocks_per_seq, bs = p.block_size;
+    auto lookup = [&](const StageMeta& d) -> int {
+      if (d.flags & F_END || lane >= d.nchunk) return 0;
+      return __ldg(bt_all + (size_t)d.b * mb + (d.tok0 + lane * kChunk) / bs);
+    };
+    StageMeta d = walker_next<LY::CPS>(w, cta, lane);
+    int phys = lookup(d);
+    bool ok = true;
+    int k = 0;
+    for (;; ++k) {
+      const int st = k % NSTAGES;
+      if (k >= NSTAGES && !mbar_wait(&empty[st], ((k / NSTAGES) - 1) & 1)) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) meta[st] = d;
+      if (d.flags & F_END) {
+        if (lane == 0) mbar_arrive(&full[st]);
+        break;
+      }
+      const bool first = d.flags & F_FIRST;
+      if (lane == 0)
+        mbar_arrive_expect_tx(&full[st], (uint32_t)(d.nchunk * kChunk * D * 2 * 2 + (first ? LY::QSLOT : 0)));
+      __syncwarp();
+      if (lane < d.nchunk) {
+        if (phys < 0 || phys >= p.num_blocks) PA_RECORD_ERROR(PA_ERRBIT_INDEX);  // TMA zero-fills out of range
+        const int tok = d.tok0 + lane * kChunk;
+        const int y = phys * bs + (tok % bs);
+        uint8_t* kd = smem + LY::K_OFF + st * LY::STAGE_BYTES + lane * kChunk * 128;
+        uint8_t* vd = smem + LY::V_OFF + st * LY::STAGE_BYTES + lane * kChunk * 128;
+#pragma unroll
+        for (int h = 0; h < LY::HALVES; ++h) {
+          tma_load_2d(kd + h * LY::TOK * 128, &kmap, d.g * D + h * 64, y, &full[st]);
+          tma_load_2d(vd + h * LY::TOK * 128, &vmap, d.g * D + h * 64, y, &full[st]);
+        }
+      }
+      if (first && lane == 31) {
+        const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q) +
+                              ((size_t)d.b * p.num_q_heads + (size_t)d.g * G) * D * 2;
+        bulk_load(smem + LY::QS_OFF + st * LY::QSLOT, qsrc, LY::QSLOT, &full[st]);
+      }
+      d = walker_next<LY::CPS>(w, cta, lane);
+      phys = lookup(d);
     }
     if (!ok && lane == 0) PA_RECORD_ERROR(PA_ERRBIT_TIMEOUT);
-    // drain: make sure every TMA this CTA issued has landed before the CTA can exit
+    // drain: every copy this CTA issued has landed before the warp leaves
     if (lane == 0) {
-      for (int k = max(0, nstages - NSTAGES); k < nstages; ++k)
-        if (!mbar_wait(&full[k % NSTAGES], (k / NSTAGES) & 1)) PA_RECORD_ERROR(PA_ERRBIT_TIMEOUT);
+      for (int j = max(0, k - NSTAGES + 1); j < k; ++j)
+        if (!mbar_wait(&full[j % NSTAGES], (j / NSTAGES) & 1)) PA_RECORD_ERROR(PA_ERRBIT_TIMEOUT);
     }
     return;
   }
 
-  // -------------------------------------------------- consumers
+  // =================================================== consumer warps
   using C = typename std::conditional<MMA, MmaConsumer<DT, D, G, NW, NSTAGES>, CoreConsumer<DT, D, G, NW, NSTAGES>>::type;
   C c;
   c.init();
-  if constexpr (MMA) c.load_q(qg, lane);
-  const uint32_t qbase = sbase + LY::Q_OFF;
+  float* qf = reinterpret_cast<float*>(smem + LY::QF_OFF) + warp * G * D;
+  const uint32_t qbase = smem_u32(qf);
   const uint32_t pbase = sbase + LY::P_OFF + warp * 32 * G * 4;
+  float* merge_o = reinterpret_cast<float*>(smem + LY::M_OFF);
+  float* merge_ml = reinterpret_cast<float*>(smem + LY::ML_OFF);
   bool ok = true;
-  for (int k = 0; k < nstages; ++k) {
+  for (int k = 0;; ++k) {
     const int st = k % NSTAGES;
     if (!mbar_wait(&full[st], (k / NSTAGES) & 1)) {
       ok = false;
       break;
     }
-    const int nv = min(32, max(0, t1 - (t0 + k * LY::TOK + warp * 32)));
+    const StageMeta d = meta[st];
+    if (d.flags & F_END) break;
+    if (d.flags & F_FIRST) {
+      c.init();
+      c.load_q(smem + LY::QS_OFF + st * LY::QSLOT, qf, p.scale_log2, lane);
+    }
+    const int nv = min(32, max(0, d.ntok - warp * 32));
     if (nv > 0) {
       const uint32_t kb = sbase + LY::K_OFF + st * LY::STAGE_BYTES;
       const uint32_t vb = sbase + LY::V_OFF + st * LY::STAGE_BYTES;
@@ -523,139 +713,165 @@ __global__ void __launch_bounds__((NW + 1) * 32) decode_split_kernel(const __gri
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
+    if (d.flags & F_LAST) {
+      // merge the NW warps' states of this piece; write out (whole segment) or a partial
+      c.stash(merge_o + warp * G * D, merge_ml + warp * G * 2, lane);
+      named_barrier_sync(1, NW * 32);
+      const int hq0 = d.g * G;
+      for (int i = threadIdx.x; i < G * D; i += NW * 32) {
+        const int h = i / D, dd = i - h * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w2 = 0; w2 < NW; ++w2) M = fmaxf(M, merge_ml[(w2 * G + h) * 2]);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < NW; ++w2) {
+          const float sc = fast_exp2(merge_ml[(w2 * G + h) * 2] - M);
+          num = fmaf(sc, merge_o[(w2 * G + h) * D + dd], num);
+          den = fmaf(sc, merge_ml[(w2 * G + h) * 2 + 1], den);
+        }
+        if (d.flags & F_DIRECT) {
+          const size_t row = (size_t)d.b * p.num_q_heads + hq0 + h;
+          reinterpret_cast<T*>(p.out)[row * D + dd] = Elt<DT>::from_f(num / den);
+        } else {
+          const size_t srow = (size_t)d.slot * G + h;
+          p.ws_o[srow * D + dd] = num;
+          if (dd == 0) {
+            p.ws_m[srow] = M;
+            p.ws_l[srow] = den;
+          }
+        }
+      }
+      named_barrier_sync(1, NW * 32);
+    }
   }
   if (!ok && lane == 0) PA_RECORD_ERROR(PA_ERRBIT_TIMEOUT);
-
-  // -------------------------------------------------- merge the NW warps, write out or a split partial
-  float* merge_o = reinterpret_cast<float*>(smem + LY::M_OFF);
-  float* merge_ml = reinterpret_cast<float*>(smem + LY::ML_OFF);
-  named_barrier_sync(1, NW * 32);  // every consumer is done reading the stage buffers
-  c.stash(merge_o + warp * G * D, merge_ml + warp * G * 2, lane);
-  named_barrier_sync(1, NW * 32);
-  const int hq0 = g * G;
-  for (int i = threadIdx.x; i < G * D; i += NW * 32) {
-    const int h = i / D, d = i - h * D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, merge_ml[(w * G + h) * 2]);
-    float num = 0.f, den = 0.f;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const float sc = fast_exp2(merge_ml[(w * G + h) * 2] - M);
-      num = fmaf(sc, merge_o[(w * G + h) * D + d], num);
-      den = fmaf(sc, merge_ml[(w * G + h) * 2 + 1], den);
-    }
-    const size_t row = (size_t)b * p.num_q_heads + hq0 + h;
-    if (nsplit == 1) {
-      reinterpret_cast<T*>(p.out)[row * D + d] = Elt<DT>::from_f(num / den);
-    } else {
-      const size_t srow = row * p.max_splits + s;
-      p.ws_o[srow * D + d] = num;
-      if (d == 0) {
-        p.ws_m[srow] = M;
-        p.ws_l[srow] = den;
-      }
-    }
-  }
 }
 
-// ------------------------------------------------------------------ split-K reduce
-// One warp per (b, h): out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s, M = max_s m_s.
-template <int DT, int D>
+// ------------------------------------------------------------------ reduce
+// One warp per (b, h): merges the pieces of segment (b, h/G) written by CTAs
+// c0..c1 (out = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c), writes zeros
+// for empty sequences, and leaves whole-segment pieces (already written) alone.
+template <int DT, int D, int G>
 __global__ void __launch_bounds__(128) decode_reduce_kernel(const DecodeParams p) {
   using T = typename Elt<DT>::T;
+  constexpr int DPL = D / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 4 + warp;  // b * Hq + h
   if (row >= p.batch * p.num_q_heads) return;
-  const int b = row / p.num_q_heads;
-  const int L = __ldg(p.context_lens + b);
-  const int ns = min((max(L, 0) + p.split_len - 1) / p.split_len, p.max_splits);
-  if (ns <= 1) return;  // written directly by the split kernel
-  const float* m = p.ws_m + (size_t)row * p.max_splits;
-  const float* l = p.ws_l + (size_t)row * p.max_splits;
+  const int b = row / p.num_q_heads, h = row - b * p.num_q_heads;
+  const int g = h / G, j = h - g * G;
+  const long long pre = p.ws_pre[b];
+  const long long nch = p.ws_pre[b + 1] - pre;
+  T* out = reinterpret_cast<T*>(p.out) + (size_t)row * D + lane * DPL;
+  if (nch <= 0) {
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) out[e] = Elt<DT>::from_f(0.f);
+    return;
+  }
+  const long long Hkv = p.num_kv_heads, grid = p.grid;
+  const long long C = Hkv * p.ws_pre[p.batch];
+  const long long cs = Hkv * pre + g * nch, ce = cs + nch;
+  const long long c0 = ((cs + 1) * grid - 1) / C, c1 = (ce * grid - 1) / C;  // owners of the first and last chunk
+  if (c0 == c1) return;
   float M = -INFINITY;
-  for (int i = lane; i < ns; i += 32) M = fmaxf(M, m[i]);
-  M = warp_max(M);
-  constexpr int DPL = D / 32;
+  for (long long c = c0; c <= c1; ++c) {
+    if (C * c / grid == C * (c + 1) / grid) continue;  // a CTA with an empty range wrote nothing
+    const long long slot = (long long)b * p.num_kv_heads + g + c;
+    M = fmaxf(M, p.ws_m[slot * G + j]);
+  }
   float acc[DPL];
 #pragma unroll
-  for (int j = 0; j < DPL; ++j) acc[j] = 0.f;
+  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
   float den = 0.f;
-  const float* o = p.ws_o + (size_t)row * p.max_splits * D + lane * DPL;
-  for (int i = 0; i < ns; ++i) {
-    const float w = fast_exp2(m[i] - M);
-    den = fmaf(w, l[i], den);
+  for (long long c = c0; c <= c1; ++c) {
+    if (C * c / grid == C * (c + 1) / grid) continue;
+    const long long srow = ((long long)b * p.num_kv_heads + g + c) * G + j;
+    const float w = fast_exp2(p.ws_m[srow] - M);
+    den = fmaf(w, p.ws_l[srow], den);
+    const float* o = p.ws_o + srow * D + lane * DPL;
     if constexpr (DPL == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(o + (size_t)i * D);
+      const float4 v = *reinterpret_cast<const float4*>(o);
       acc[0] = fmaf(w, v.x, acc[0]); acc[1] = fmaf(w, v.y, acc[1]);
       acc[2] = fmaf(w, v.z, acc[2]); acc[3] = fmaf(w, v.w, acc[3]);
     } else {
-      const float2 v = *reinterpret_cast<const float2*>(o + (size_t)i * D);
+      const float2 v = *reinterpret_cast<const float2*>(o);
       acc[0] = fmaf(w, v.x, acc[0]); acc[1] = fmaf(w, v.y, acc[1]);
     }
   }
   const float inv = 1.f / den;
-  T* out = reinterpret_cast<T*>(p.out) + (size_t)row * D + lane * DPL;
   if constexpr (DPL == 4) {
-    uint2 w;
-    w.x = Elt<DT>::from_f2(acc[0] * inv, acc[1] * inv);
-    w.y = Elt<DT>::from_f2(acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<uint2*>(out) = w;
+    uint2 wv;
+    wv.x = Elt<DT>::from_f2(acc[0] * inv, acc[1] * inv);
+    wv.y = Elt<DT>::from_f2(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(out) = wv;
   } else {
     *reinterpret_cast<uint32_t*>(out) = Elt<DT>::from_f2(acc[0] * inv, acc[1] * inv);
   }
 }
 
 // ------------------------------------------------------------------ host side
-constexpr int kNW = 2;        // consumer warps per CTA (64-token stages)
-constexpr int kStages = 2;    // ring depth
+constexpr int kNW = 2;       // consumer warps per CTA (64-token stages)
+constexpr int kStages = 3;   // ring depth
+
+template <int D, int G>
+constexpr int alloc_bytes() {
+  return Layout<D, G, kNW, kStages, (G >= 8)>::ALLOC;
+}
+
+int smem_per_cta(int D, int G) {
+  switch (D * 100 + G) {
+    case 6401: return alloc_bytes<64, 1>();
+    case 6402: return alloc_bytes<64, 2>();
+    case 6404: return alloc_bytes<64, 4>();
+    case 6408: return alloc_bytes<64, 8>();
+    case 6416: return alloc_bytes<64, 16>();
+    case 12801: return alloc_bytes<128, 1>();
+    case 12802: return alloc_bytes<128, 2>();
+    case 12804: return alloc_bytes<128, 4>();
+    case 12808: return alloc_bytes<128, 8>();
+    case 12816: return alloc_bytes<128, 16>();
+  }
+  return 0;
+}
 
 struct Plan {
-  int split_len;
-  int max_splits;
+  int grid;
   size_t ws_bytes;
-  size_t off_l, off_o;
+  size_t off_m, off_l, off_o;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-bool make_plan(int batch, int Hq, int Hkv, int D, int max_ctx, int num_splits, Plan* pl) {
-  if (batch < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || max_ctx < 0 || num_splits < 0) return false;
-  const int gran = 64;
-  const int max_split_len = 8192;  // keeps a split's block-table slice within BT_MAX entries
-  int sl;
-  if (num_splits > 0) {
-    sl = (max_ctx + num_splits - 1) / num_splits;
-    sl = std::max(gran, (sl + gran - 1) / gran * gran);
-  } else {
-    // Enough CTAs to fill the GPU several times over, but splits long enough
-    // to amortise their partial write and pipeline fill.
-    const long units = (long)batch * Hkv;
-    const long target = 148L * 16;
-    sl = 256;
-    while (sl * 2 <= 4096 && units * ((max_ctx + 2 * sl - 1) / (2 * sl)) >= target) sl *= 2;
+bool make_plan(int batch, int Hq, int Hkv, int D, int num_partitions, Plan* pl) {
+  if (batch < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || num_partitions < 0 || Hq % Hkv) return false;
+  const int G = Hq / Hkv;
+  const int smem = smem_per_cta(D, G);
+  if (smem == 0) return false;
+  int grid = num_partitions;
+  if (grid == 0) {
+    int dev = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess)
+      per_sm = 228 * 1024;
+    int occ = per_sm / (smem + 1024);
+    occ = std::max(1, std::min(occ, 4));
+    grid = pa::sm_count() * occ;
   }
-  if (max_ctx > 0 && sl > ((max_ctx + gran - 1) / gran) * gran) sl = ((max_ctx + gran - 1) / gran) * gran;
-  if (sl > max_split_len) sl = max_split_len;
-  pl->split_len = sl;
-  pl->max_splits = max_ctx > 0 ? (max_ctx + sl - 1) / sl : 1;
-  const size_t rows = (size_t)batch * Hq * pl->max_splits;
-  if (pl->max_splits <= 1) {
-    pl->ws_bytes = 0;
-    pl->off_l = pl->off_o = 0;
-    return true;
-  }
-  pl->off_l = align256(rows * 4);
-  pl->off_o = pl->off_l + align256(rows * 4);
-  pl->ws_bytes = pl->off_o + align256(rows * D * 4);
+  pl->grid = grid;
+  const size_t slots = (size_t)batch * Hkv + grid;
+  pl->off_m = align256((size_t)(batch + 1) * 8);
+  pl->off_l = pl->off_m + align256(slots * G * 4);
+  pl->off_o = pl->off_l + align256(slots * G * 4);
+  pl->ws_bytes = pl->off_o + align256(slots * G * D * 4);
   return true;
 }
 
 template <int DT, int D, int G>
 int launch(const CUtensorMap& km, const CUtensorMap& vm, const DecodeParams& p, cudaStream_t st) {
   constexpr bool MMA = G >= 8;
-  using LY = Layout<D, G, kNW, kStages>;
-  auto kern = decode_split_kernel<DT, D, G, kNW, kStages, MMA>;
+  using LY = Layout<D, G, kNW, kStages, MMA>;
+  auto kern = decode_kernel<DT, D, G, kNW, kStages, MMA>;
   static bool attr_set[64] = {};  // per instantiation and device
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
@@ -664,16 +880,11 @@ int launch(const CUtensorMap& km, const CUtensorMap& vm, const DecodeParams& p, 
       return PA_ERR_CUDA;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  const long grid = (long)p.batch * p.max_splits * p.num_kv_heads;
-  if (grid > 0) {
-    kern<<<(unsigned)grid, (kNW + 1) * 32, LY::ALLOC, st>>>(km, vm, p);
-    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  }
-  if (p.max_splits > 1) {
-    const int rows = p.batch * p.num_q_heads;
-    decode_reduce_kernel<DT, D><<<(rows + 3) / 4, 128, 0, st>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  }
+  kern<<<p.grid, (kNW + 1) * 32, LY::ALLOC, st>>>(km, vm, p);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  const int rows = p.batch * p.num_q_heads;
+  decode_reduce_kernel<DT, D, G><<<(rows + 3) / 4, 128, 0, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   return PA_OK;
 }
 
@@ -692,31 +903,33 @@ int dispatch_g(int G, const CUtensorMap& km, const CUtensorMap& vm, const Decode
 }  // namespace
 
 extern "C" int pa_decode_plan(int batch, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len,
-                              int num_splits_or_0, int* split_len_out, int* max_splits_out,
+                              int num_partitions_or_0, int* grid_out, int* max_pieces_out,
                               size_t* workspace_bytes_out) {
+  if (max_context_len < 0 || !pa::valid_head_dim(head_dim)) return PA_ERR_INVALID;
   Plan pl;
-  if (!make_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_splits_or_0, &pl))
-    return PA_ERR_INVALID;
-  if (split_len_out) *split_len_out = pl.split_len;
-  if (max_splits_out) *max_splits_out = pl.max_splits;
+  if (!make_plan(batch, num_q_heads, num_kv_heads, head_dim, num_partitions_or_0, &pl)) return PA_ERR_INVALID;
+  if (grid_out) *grid_out = pl.grid;
+  if (max_pieces_out) *max_pieces_out = batch * num_kv_heads + pl.grid;
   if (workspace_bytes_out) *workspace_bytes_out = pl.ws_bytes;
   return PA_OK;
 }
 
 extern "C" size_t pa_decode_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
-                                           int max_context_len, int num_splits_or_0) {
-  Plan pl;
-  if (!make_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_splits_or_0, &pl)) return 0;
-  return pl.ws_bytes;
+                                           int max_context_len, int num_partitions_or_0) {
+  size_t ws = 0;
+  if (pa_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_partitions_or_0, nullptr,
+                     nullptr, &ws) != PA_OK)
+    return 0;
+  return ws;
 }
 
 extern "C" int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
                          int max_blocks_per_seq, const int32_t* context_lens, int batch, int num_q_heads,
                          int num_kv_heads, int head_dim, int block_size, int num_blocks, int max_context_len,
-                         float scale, int dtype, void* workspace, size_t workspace_bytes, int num_splits_or_0,
+                         float scale, int dtype, void* workspace, size_t workspace_bytes, int num_partitions_or_0,
                          void* out, void* stream) {
   if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks < 0 ||
-      max_context_len < 0 || max_blocks_per_seq < 0 || num_splits_or_0 < 0)
+      max_context_len < 0 || max_blocks_per_seq < 0 || num_partitions_or_0 < 0)
     return PA_ERR_INVALID;
   if (!pa::valid_dtype(dtype) || !pa::valid_head_dim(head_dim) || !pa::valid_block_size(block_size))
     return PA_ERR_UNSUPPORTED;
@@ -730,14 +943,11 @@ extern "C" int pa_decode(const void* q, const void* k_cache, const void* v_cache
     return PA_ERR_ALIGN;
   if ((long)max_blocks_per_seq * block_size < max_context_len) return PA_ERR_INVALID;
   if (num_blocks == 0 && max_context_len > 0) return PA_ERR_INVALID;
+  if ((long)num_blocks * block_size >= (1L << 31)) return PA_ERR_UNSUPPORTED;
   Plan pl;
-  if (!make_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_splits_or_0, &pl))
-    return PA_ERR_INVALID;
-  if (pl.max_splits > 1) {
-    if (!workspace || workspace_bytes < pl.ws_bytes) return PA_ERR_WORKSPACE;
-    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PA_ERR_ALIGN;
-  }
-  if ((long)batch * pl.max_splits * num_kv_heads > 0x7fffffffL) return PA_ERR_UNSUPPORTED;
+  if (!make_plan(batch, num_q_heads, num_kv_heads, head_dim, num_partitions_or_0, &pl)) return PA_ERR_INVALID;
+  if (!workspace || workspace_bytes < pl.ws_bytes) return PA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PA_ERR_ALIGN;
 
   DecodeParams p;
   p.q = q;
@@ -745,17 +955,17 @@ extern "C" int pa_decode(const void* q, const void* k_cache, const void* v_cache
   p.block_tables = block_tables;
   p.context_lens = context_lens;
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
-  p.ws_m = reinterpret_cast<float*>(ws);
-  p.ws_l = reinterpret_cast<float*>(ws ? ws + pl.off_l : nullptr);
-  p.ws_o = reinterpret_cast<float*>(ws ? ws + pl.off_o : nullptr);
+  p.ws_pre = reinterpret_cast<long long*>(ws);
+  p.ws_m = reinterpret_cast<float*>(ws + pl.off_m);
+  p.ws_l = reinterpret_cast<float*>(ws + pl.off_l);
+  p.ws_o = reinterpret_cast<float*>(ws + pl.off_o);
   p.max_blocks_per_seq = max_blocks_per_seq;
   p.batch = batch;
   p.num_q_heads = num_q_heads;
   p.num_kv_heads = num_kv_heads;
   p.block_size = block_size;
   p.num_blocks = num_blocks;
-  p.split_len = pl.split_len;
-  p.max_splits = pl.max_splits;
+  p.grid = pl.grid;
   p.scale_log2 = scale * kLog2e;
 
   // One tensor map per cache over the [num_blocks*block_size][Hkv*D] row view; 16-row x 64-column boxes.

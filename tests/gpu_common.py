@@ -44,7 +44,7 @@ def oracle_step(wl):
     return from_bits(kc, dt), from_bits(vc, dt), rows, lens, slots
 
 
-def gpu_step(wl, num_splits: int = 0, device="cuda"):
+def gpu_step(wl, num_partitions: int = 0, device="cuda"):
     """Product side: C++ pool replay, then pa_write_kv and pa_decode (or nothing else for prefill)."""
     import paged_kv_cache_330_b200 as pa
     _, bt, lens, sm, _ = pa.replay_ops(wl.ops, wl.num_blocks, wl.cfg["block_size"], wl.free_order, wl.batch)
@@ -55,5 +55,5 @@ def gpu_step(wl, num_splits: int = 0, device="cuda"):
     pa.write_kv(wl.k_new.to(device), wl.v_new.to(device), torch.from_numpy(sm).to(device), kc, vc)
     out = None
     if wl.cfg["kind"] != "prefill":
-        out = pa.decode(wl.q.to(device), kc, vc, bt_d, lens_d, int(lens.max()), wl.scale, num_splits=num_splits)
+        out = pa.decode(wl.q.to(device), kc, vc, bt_d, lens_d, int(lens.max()), wl.scale, num_partitions=num_partitions)
     return out, kc, vc, bt_d, lens_d, bt, lens

@@ -93,19 +93,16 @@ def test_prefill_validation():
 def test_decode_plan():
     for name in ("tiny", "qwen_decode", "llama70b_long", "prefix_sweep"):
         c = CONFIGS[name]
-        maxL = {"tiny": 64, "qwen_decode": 1024, "llama70b_long": 8192, "prefix_sweep": 2561}[name]
-        sl, ms, ws = pa.decode_plan(c["batch"], c["num_q_heads"], c["num_kv_heads"], c["head_dim"], maxL)
-        assert sl % 64 == 0 and sl >= 64 and ms == -(-maxL // sl)
-        if ms > 1:
-            rows = c["batch"] * c["num_q_heads"] * ms
-            assert ws >= rows * (c["head_dim"] + 2) * 4
-        else:
-            assert ws == 0
-        assert pa.lib.pa_decode_workspace_size(c["batch"], c["num_q_heads"], c["num_kv_heads"], c["head_dim"], maxL, 0) == ws
-    sl, ms, _ = pa.decode_plan(4, 8, 2, 128, 1000, num_splits=4)
-    assert ms == 4 and sl == 256
-    sl, ms, ws = pa.decode_plan(4, 8, 2, 128, 1000, num_splits=1)
-    assert ms == 1 and ws == 0
+        B, Hq, Hkv, D = c["batch"], c["num_q_heads"], c["num_kv_heads"], c["head_dim"]
+        grid, maxp, ws = pa.decode_plan(B, Hq, Hkv, D, 1000)
+        assert grid >= 1 and maxp == B * Hkv + grid
+        G = Hq // Hkv
+        assert ws >= (B + 1) * 8 + maxp * G * (D + 2) * 4
+        assert pa.lib.pa_decode_workspace_size(B, Hq, Hkv, D, 1000, 0) == ws
+    grid, maxp, ws = pa.decode_plan(4, 8, 2, 128, 1000, num_partitions=7)
+    assert grid == 7 and maxp == 4 * 2 + 7
+    assert pa.lib.pa_decode_workspace_size(4, 8, 2, 96, 1000, 0) == 0      # unsupported head_dim
+    assert pa.lib.pa_decode_workspace_size(4, 6, 4, 128, 1000, 0) == 0     # heads not a multiple
 
 
 # --------------------------------------------------------------------------- C++ pool vs oracle pool
