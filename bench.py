@@ -4,8 +4,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
 One step = the whole decode hot path over one batch: pa_write_kv of each
-sequence's new token into its slot, then pa_decode (split kernel + split-K
-reduce kernel) over every sequence's paged context.  Inputs are resident in
+sequence's new token into its slot, then pa_decode (one kernel: block-table
+gather, attention, split-K merge) over every sequence's paged context.  Each
+call is captured once in a CUDA graph and replayed, so the timed loop measures
+the GPU rather than Python launch overhead.  Inputs are resident in
 HBM; the KV working set (~295 MB) is larger than the 126 MB L2, so no flush is
 needed between steps.  Timed with CUDA events on the launching stream,
 bracketed by barrier + synchronize, max over ranks.  N > 1 runs independent
@@ -81,6 +83,7 @@ class ClockSampler:
 
     def __init__(self, device_index: int, period_s: float = 0.02):
         self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.mem_samples, self.power_w = [], []
         self.period = period_s
         self._stop = threading.Event()
         self._t = None
@@ -98,6 +101,8 @@ class ClockSampler:
         while not self._stop.is_set():
             try:
                 self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.mem_samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_MEM))
+                self.power_w.append(nv.nvmlDeviceGetPowerUsage(self._h) / 1000.0)
                 r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
                 for bit, name in self.REASONS.items():
                     if r & bit and name != "gpu_idle":
@@ -118,8 +123,10 @@ class ClockSampler:
             self._t.join()
 
     def summary(self):
-        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        med = lambda v: statistics.median(v) if v else None
+        return {"sm_mhz": med(self.samples), "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples), "mem_mhz": med(self.mem_samples),
+                "power_w_median": med(self.power_w), "power_w_max": max(self.power_w) if self.power_w else None}
 
 
 # ------------------------------------------------------------------------------------------------ helpers
@@ -251,42 +258,74 @@ def run_ours(args):
     btd = torch.from_numpy(bt).to(dev)
     lensd = torch.from_numpy(lens).to(dev)
     out = torch.empty_like(q)
-    work = torch.empty(max(wsb, 256), dtype=torch.uint8, device=dev)
+    work = torch.zeros(max(wsb, 256), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(ev_pair=None):
+    def write_step():
         pa.write_kv(kn, vn, smd, kc, vc, stream=stream)
-        if ev_pair is not None:
-            ev_pair[0].record(stream)
+
+    def decode_step():
         pa.decode(q, kc, vc, btd, lensd, maxL, wl.scale, out=out, workspace=work, num_partitions=args.num_partitions,
                   stream=stream)
-        if ev_pair is not None:
-            ev_pair[1].record(stream)
 
     def barrier():
         if ws > 1:
             dist.barrier()
 
+    # eager warm-up (first calls set kernel attributes), then CUDA graphs of several whole steps so
+    # the timed loop measures the GPU, not Python launch overhead
     for _ in range(args.warmup):
-        step()
+        write_step()
+        decode_step()
     torch.cuda.synchronize(dev)
     assert pa.device_error() == 0
 
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap_stream):
+            fn()
+        return g
+
+    cap_stream = torch.cuda.Stream(dev)
+    S = args.steps_per_graph
     K = args.steps
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    if K % S:
+        S = 1
+    # one graph = S whole steps (write_kv + decode each); a second graph = S decodes alone, for the
+    # decode kernel's own average duration (the roofline denominator's time)
+    g_steps = capture(lambda: [(pa.write_kv(kn, vn, smd, kc, vc, stream=cap_stream),
+                                pa.decode(q, kc, vc, btd, lensd, maxL, wl.scale, out=out, workspace=work,
+                                          num_partitions=args.num_partitions, stream=cap_stream)) for _ in range(S)])
+    g_decs = capture(lambda: [pa.decode(q, kc, vc, btd, lensd, maxL, wl.scale, out=out, workspace=work,
+                                        num_partitions=args.num_partitions, stream=cap_stream) for _ in range(S)])
+    g_write = capture(lambda: pa.write_kv(kn, vn, smd, kc, vc, stream=cap_stream))
+    g_dec = capture(lambda: pa.decode(q, kc, vc, btd, lensd, maxL, wl.scale, out=out, workspace=work,
+                                      num_partitions=args.num_partitions, stream=cap_stream))
+    for _ in range(max(1, args.warmup // S)):
+        g_steps.replay()
+    torch.cuda.synchronize(dev)
+
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d_start, d_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier()
         torch.cuda.synchronize(dev)
         t_start.record(stream)
-        for i in range(K):
-            step(evs[i])
+        for _ in range(K // S):
+            g_steps.replay()
         t_end.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
+        # decode kernel alone, same launch count, straight after the timed region
+        d_start.record(stream)
+        for _ in range(K // S):
+            g_decs.replay()
+        d_end.record(stream)
+        torch.cuda.synchronize(dev)
     ms_total = t_start.elapsed_time(t_end)
-    dec_ms = [a.elapsed_time(b) for a, b in evs]
+    dec_ms = [d_start.elapsed_time(d_end) / K]
     ms_step = ms_total / K
+    assert pa.device_error() == 0
 
     # ---- end to end through the public API: pinned host inputs -> device, step, result -> host
     pin = lambda t: t.pin_memory()
@@ -296,29 +335,35 @@ def run_ours(args):
     h2d = sum(t.numel() * t.element_size() for t in (h_q, h_kn, h_vn, h_sm, h_bt, h_lens))
     d2h = h_out.numel() * h_out.element_size()
 
-    def e2e_step():
+    def e2e_step(st):
         q.copy_(h_q, non_blocking=True)
         kn.copy_(h_kn, non_blocking=True)
         vn.copy_(h_vn, non_blocking=True)
         smd.copy_(h_sm, non_blocking=True)
         btd.copy_(h_bt, non_blocking=True)
         lensd.copy_(h_lens, non_blocking=True)
-        step()
+        pa.write_kv(kn, vn, smd, kc, vc, stream=st)
+        pa.decode(q, kc, vc, btd, lensd, maxL, wl.scale, out=out, workspace=work, num_partitions=args.num_partitions,
+                  stream=st)
         h_out.copy_(out, non_blocking=True)
 
     for _ in range(args.warmup):
-        e2e_step()
+        e2e_step(stream)
+    torch.cuda.synchronize(dev)
+    g_e2e = capture(lambda: [e2e_step(cap_stream) for _ in range(S)])
+    g_e2e.replay()
     torch.cuda.synchronize(dev)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(K):
-        e2e_step()
+    for _ in range(K // S):
+        g_e2e.replay()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
     e2e_ms = e0.elapsed_time(e1) / K
     assert pa.device_error() == 0
+    del g_write, g_dec, g_steps, g_decs, g_e2e
 
     # ---- max over ranks, totals
     kvb = kv_bytes(wl)
@@ -337,7 +382,7 @@ def run_ours(args):
     achieved = alg / (dec_avg * 1e-3) / 1e9
     tr = NCU_TRAFFIC.get(args.workload)
     traffic = tr["bytes"] if tr and tr.get("src") == kernel_source_hash() else None
-    launches_per_step = 3  # write_kv, decode, split-K reduce
+    launches_per_step = 2  # write_kv, decode (split-K merge inside)
     if rank == 0:
         cpu = None
         if ws == 1 and not args.no_cpu_baseline:
@@ -356,10 +401,11 @@ def run_ours(args):
                              "of_nominal_8000": value / ws / 8000.0},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms},
-            "roofline": {"bound": "hbm", "kernel": "pa_decode (split + split-K reduce kernels)",
+            "roofline": {"bound": "hbm", "kernel": "pa_decode (one kernel: gather, attention, split-K merge)",
                          "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "algorithmic_bytes": alg,
-                         "avg_launch_ms": dec_avg},
+                         "avg_launch_ms": dec_avg,
+                         "timing": "decode-only graph replays, same launch count, right after the timed region"},
             "gpu_launches": launches_per_step * K,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
@@ -378,6 +424,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen_decode", choices=sorted(WORKLOAD_TEXT))
     ap.add_argument("--num-partitions", type=int, default=0, help="decode CTAs (0 = fill the GPU)")
+    ap.add_argument("--steps-per-graph", type=int, default=10, help="whole steps captured per CUDA graph")
     ap.add_argument("--ref-budget", type=float, default=12.0, help="seconds of oracle time per reference sample")
     ap.add_argument("--ref-seqs", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")

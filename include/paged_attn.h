@@ -112,8 +112,9 @@ int pa_copy_blocks(const int32_t* pairs, int num_pairs, void* k_cache, void* v_c
 /* head) is cut into 16-token chunks; all chunks, end to end, are shared out */
 /* evenly over `grid` persistent CTAs.  The part of a sequence's context     */
 /* that one CTA handles yields fp32 (max, sum, weighted V) in the workspace  */
-/* unless it is the whole context; a reduce kernel merges the parts by the   */
-/* log-sum-exp rule.  Two kernels are launched per call.                     */
+/* unless it is the whole context; the CTA that finishes a context's last    */
+/* part merges the parts by the log-sum-exp rule (atomic count, no waiting). */
+/* One kernel is launched per call.                                          */
 /*                                                                           */
 /* pa_decode_plan: the grid and workspace the call will use on the current   */
 /* device.  num_partitions_or_0 > 0 fixes the number of CTAs (the number of  */
@@ -131,7 +132,10 @@ size_t pa_decode_workspace_size(int batch, int num_q_heads, int num_kv_heads, in
 /* max_context_len: host-side upper bound of context_lens; block_tables rows */
 /* must cover it (max_blocks_per_seq * block_size >= max_context_len).       */
 /* workspace: device scratch of >= pa_decode_workspace_size() bytes, 256-byte */
-/* aligned, owned by the caller; its contents need no initialisation.        */
+/* aligned, owned by the caller.  It must be zero-filled before its first    */
+/* use (its head holds per-context piece counters); every completed call     */
+/* leaves those counters at zero again, so it needs no clearing afterwards   */
+/* (a call that recorded PA_ERRBIT_TIMEOUT may leave them dirty: re-zero).  */
 /* Two calls that run at the same time must use different workspaces.        */
 int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
               int max_blocks_per_seq, const int32_t* context_lens, int batch, int num_q_heads,

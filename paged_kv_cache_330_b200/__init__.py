@@ -158,8 +158,8 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len: int
     if out is None:
         out = torch.empty_like(q)
     _, _, need = decode_plan(B, Hq, Hkv, D, max_context_len, num_partitions)
-    if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is None:  # zero-filled once; every call leaves it zeroed again
+        workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.pa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), int(block_tables.shape[1]),
                          _ptr(context_lens), B, Hq, Hkv, D, bs, NB, int(max_context_len), float(scale),

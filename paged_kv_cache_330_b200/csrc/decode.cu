@@ -20,7 +20,8 @@
 // of the context split on "In-depth analysis of vllm-ascend", section 3.1.
 //
 // Data movement.  One producer warp walks the CTA's chunk range, looks up each
-// chunk's physical block (one lookup ahead) and gathers 16-row K and V boxes
+// chunk's physical block (several stages ahead, cp.async into a plan ring) and
+// gathers 16-row K and V boxes
 // with TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast) into an
 // NSTAGES-deep shared-memory ring guarded by mbarriers, straight across piece
 // and segment boundaries (the pages' prefetch-depth / pipeline-stage lesson,
@@ -51,13 +52,17 @@ using namespace pa;
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kChunk = 16;  // tokens per chunk = rows per TMA box
+constexpr int kPlanRing = 8;  // producer plan ring slots
+constexpr int kMaxPieces = 32;  // pieces per segment the epilogue merges with precomputed weights
+constexpr int kLookahead = 6; // stages planned (block-table entries in flight) ahead of the one issued
+static_assert(kPlanRing > kLookahead, "plan ring must hold the stages in flight plus the one issued");
 
 struct DecodeParams {
   const void* q;
   void* out;
   const int32_t* block_tables;
   const int32_t* context_lens;
-  long long* ws_pre;  // [B+1] chunks before sequence b (written by CTA 0)
+  int* ws_cnt;        // [B*Hkv] pieces of each segment written so far (zero between calls)
   float* ws_m;        // [nslots][G] running max of a piece (log2 domain)
   float* ws_l;        // [nslots][G] sum of exp2(x - m)
   float* ws_o;        // [nslots][G][D] sum of exp2(x - m) * v
@@ -73,8 +78,11 @@ struct DecodeParams {
 
 enum : int { F_FIRST = 1, F_LAST = 2, F_DIRECT = 4, F_END = 8 };
 
+// One stage as the producer planned it.  c0/npieces (set on a piece's last
+// stage) name the first CTA holding a piece of this segment and how many
+// pieces the segment has, for the merge.
 struct StageMeta {
-  int b, g, tok0, ntok, flags, slot, nchunk, pad;
+  int b, g, tok0, ntok, flags, nchunk, c0, npieces;
 };
 
 template <int D, int G, int NW, int NSTAGES, bool MMA>
@@ -88,16 +96,26 @@ struct Layout {
   static constexpr int V_OFF = K_OFF + NSTAGES * STAGE_BYTES;
   static constexpr int QS_OFF = V_OFF + NSTAGES * STAGE_BYTES;
   static constexpr int META_OFF = QS_OFF + NSTAGES * QSLOT;
-  static constexpr int QF_OFF = META_OFF + NSTAGES * (int)sizeof(StageMeta);  // fp32 q per warp (CUDA-core path)
+  static constexpr int PLAN_OFF = META_OFF + NSTAGES * (int)sizeof(StageMeta);  // producer plan ring
+  static constexpr int PLAN_BYTES = kPlanRing * ((int)sizeof(StageMeta) + 8 * 4);
+  static constexpr int QF_OFF = PLAN_OFF + PLAN_BYTES;                        // fp32 q per warp (CUDA-core path)
   static constexpr int QF_BYTES = MMA ? 0 : NW * G * D * 4;
   static constexpr int P_OFF = QF_OFF + QF_BYTES;                             // fp32 p per warp (CUDA-core path)
   static constexpr int P_BYTES = MMA ? 0 : NW * 32 * G * 4;
-  static constexpr int M_OFF = P_OFF + P_BYTES;                               // merge: fp32 [NW][G][D]
-  static constexpr int ML_OFF = M_OFF + NW * G * D * 4;                       // merge: fp32 [NW][G][2]
-  static constexpr int BAR_OFF = ML_OFF + NW * G * 2 * 4;                     // full[NSTAGES], empty[NSTAGES]
-  static constexpr int BYTES = BAR_OFF + 2 * NSTAGES * 8;
+  // two merge buffers handed from the consumers to the epilogue warp:
+  // fp32 o [NW][G][D], fp32 (m, l) [NW][G][2], then the piece's descriptor
+  static constexpr int MB_O = 0;
+  static constexpr int MB_ML = NW * G * D * 4;
+  static constexpr int MB_DESC = MB_ML + NW * G * 2 * 4;
+  static constexpr int MB_BYTES = (MB_DESC + (int)sizeof(StageMeta) + 15) / 16 * 16;
+  static constexpr int M_OFF = P_OFF + P_BYTES;
+  static constexpr int WTS_OFF = M_OFF + 2 * MB_BYTES;                        // merge weights fp32 [G][kMaxPieces]
+  static constexpr int MISC_OFF = WTS_OFF + G * kMaxPieces * 4;               // int64 total chunks on the line
+  static constexpr int BAR_OFF = MISC_OFF + 16;  // full[NSTAGES], empty[NSTAGES], mfull[2], mempty[2]
+  static constexpr int BYTES = BAR_OFF + (2 * NSTAGES + 4) * 8;
   static constexpr int ALLOC = BYTES + 1024;                                  // slack for 1024-byte alignment
   static_assert(QS_OFF % 16 == 0 && QSLOT % 16 == 0 && BAR_OFF % 8 == 0, "alignment");
+  static_assert(CPS <= 8, "plan ring holds 8 block lookups per stage");
 };
 
 // Address of element (row r, column d) inside a stage buffer laid out as
@@ -187,6 +205,15 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint3
                : "memory");
 }
 
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ------------------------------------------------------------------ CUDA-core consumer (G <= 4)
 template <int DT, int D, int G, int NW, int NSTAGES>
 struct CoreConsumer {
@@ -218,10 +245,10 @@ struct CoreConsumer {
   // One 32-token tile: rows r0 .. r0+31 of the stage, nv of them valid.
   __device__ __forceinline__ void tile(uint32_t kbase, uint32_t vbase, uint32_t qbase, uint32_t pbase, int r0,
                                        int nv, int lane) {
-    // ---- scores: lane = token
-    float acc[G];
+    // ---- scores: lane = token; four partial sums per head keep the FMA chains short
+    float acc[G][4];
 #pragma unroll
-    for (int h = 0; h < G; ++h) acc[h] = 0.f;
+    for (int h = 0; h < G; ++h) acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
     const int r = r0 + lane;
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) {
@@ -232,23 +259,21 @@ struct CoreConsumer {
       for (int h = 0; h < G; ++h) {
         const uint4 qa = lds128(qbase + (h * D + c * 8) * 4);
         const uint4 qb = lds128(qbase + (h * D + c * 8 + 4) * 4);
-        float a = acc[h];
-        a = fmaf(k01.x, __uint_as_float(qa.x), a);
-        a = fmaf(k01.y, __uint_as_float(qa.y), a);
-        a = fmaf(k23.x, __uint_as_float(qa.z), a);
-        a = fmaf(k23.y, __uint_as_float(qa.w), a);
-        a = fmaf(k45.x, __uint_as_float(qb.x), a);
-        a = fmaf(k45.y, __uint_as_float(qb.y), a);
-        a = fmaf(k67.x, __uint_as_float(qb.z), a);
-        a = fmaf(k67.y, __uint_as_float(qb.w), a);
-        acc[h] = a;
+        acc[h][0] = fmaf(k01.x, __uint_as_float(qa.x), acc[h][0]);
+        acc[h][1] = fmaf(k01.y, __uint_as_float(qa.y), acc[h][1]);
+        acc[h][2] = fmaf(k23.x, __uint_as_float(qa.z), acc[h][2]);
+        acc[h][3] = fmaf(k23.y, __uint_as_float(qa.w), acc[h][3]);
+        acc[h][0] = fmaf(k45.x, __uint_as_float(qb.x), acc[h][0]);
+        acc[h][1] = fmaf(k45.y, __uint_as_float(qb.y), acc[h][1]);
+        acc[h][2] = fmaf(k67.x, __uint_as_float(qb.z), acc[h][2]);
+        acc[h][3] = fmaf(k67.y, __uint_as_float(qb.w), acc[h][3]);
       }
     }
     // ---- online softmax (log2 domain), fp32
     float p[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      const float s = lane < nv ? acc[h] : -INFINITY;
+      const float s = lane < nv ? (acc[h][0] + acc[h][1]) + (acc[h][2] + acc[h][3]) : -INFINITY;
       const float mn = fmaxf(m[h], warp_max(s));
       const float alpha = fast_exp2(m[h] - mn);
       p[h] = fast_exp2(s - mn);
@@ -270,6 +295,7 @@ struct CoreConsumer {
     __syncwarp();
     // ---- PV: lane = DPL consecutive columns
     const int d0 = lane * DPL;
+#pragma unroll 4
     for (int t = 0; t < nv; ++t) {
       float v[DPL];
       const uint32_t va = swz_addr<LY::TOK>(vbase, r0 + t, d0);
@@ -463,9 +489,19 @@ struct Walker {
   long long piece_start;      // first chunk of the current piece
   int b, g, L, nch;           // current segment: sequence, KV head, clamped length, chunks
   int win_base, win_len;      // lens window: lane i holds the clamped length of sequence win_base + i
-  int batch, hkv, cap;
+  int batch, hkv, cap, grid;
+  long long total;            // chunks on the whole line
   const int32_t* lens;
+  // sub-ranges still to walk after the current one, in order (at most two)
+  int nq;
+  long long q0_start, q0_end, q0_pre, q1_start, q1_end, q1_pre;
+  int q0_b, q1_b;
 };
+
+// CTA that owns chunk x of the line: the largest c with total*c/grid <= x.
+__device__ __forceinline__ long long owner_of(long long x, long long total, long long grid) {
+  return ((x + 1) * grid - 1) / total;
+}
 
 __device__ __forceinline__ int clamp_len(int L, int cap) { return L < 0 ? 0 : (L > cap ? cap : L); }
 
@@ -473,6 +509,66 @@ __device__ __forceinline__ void load_window(Walker& w, int base, int lane) {
   w.win_base = base;
   const int i = base + lane;
   w.win_len = i < w.batch ? clamp_len(__ldg(w.lens + i), w.cap) : 0;
+}
+
+// Sequence b holding chunk x of the line (x < total) and pre = chunks of all sequences before it.
+// Warp-cooperative scan over the lengths, 256 per pass.
+__device__ __forceinline__ void find_seq(const Walker& w, long long x, int lane, int& fb, long long& fpre) {
+  long long run = 0;
+  fb = -1;
+  fpre = 0;
+  for (int base = 0; base < w.batch; base += 256) {
+    int v[8];
+    long long s = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = base + lane * 8 + j;
+      v[j] = i < w.batch ? (clamp_len(__ldg(w.lens + i), w.cap) + kChunk - 1) / kChunk : 0;
+      s += v[j];
+    }
+    const long long incl = warp_incl_scan_ll(s, lane);
+    long long pre = run + incl - s;
+    int found = -1;
+    long long found_pre = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (v[j] > 0 && pre * w.hkv <= x && x < (pre + v[j]) * w.hkv) {
+        found = base + lane * 8 + j;
+        found_pre = pre;
+      }
+      pre += v[j];
+    }
+    const unsigned hit = __ballot_sync(0xffffffffu, found >= 0);
+    if (hit) {
+      const int src = __ffs(hit) - 1;
+      fb = __shfl_sync(0xffffffffu, found, src);
+      fpre = __shfl_sync(0xffffffffu, found_pre, src);
+      return;
+    }
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+}
+
+// Start walking chunks [x, end) from the segment that holds x (sequence b, pre chunks before it).
+__device__ __forceinline__ void walker_seek(Walker& w, long long x, long long end, int b, long long pre, int lane) {
+  if (b < w.win_base || b >= w.win_base + 32) load_window(w, b, lane);
+  w.b = b;
+  w.L = __shfl_sync(0xffffffffu, w.win_len, b - w.win_base);
+  w.nch = (w.L + kChunk - 1) / kChunk;
+  w.g = (int)((x - pre * w.hkv) / w.nch);
+  w.seg_start = pre * w.hkv + (long long)w.g * w.nch;
+  w.pos = x;
+  w.piece_start = x;
+  w.end = end;
+}
+
+__device__ __forceinline__ void walker_push(Walker& w, long long start, long long end, int b, long long pre) {
+  if (w.nq == 0) {
+    w.q0_start = start; w.q0_end = end; w.q0_b = b; w.q0_pre = pre;
+  } else {
+    w.q1_start = start; w.q1_end = end; w.q1_b = b; w.q1_pre = pre;
+  }
+  ++w.nq;
 }
 
 // Move to the next sequence with at least one chunk (b must stay < batch while chunks remain).
@@ -490,9 +586,14 @@ __device__ __forceinline__ void next_sequence(Walker& w, int lane) {
 template <int CPS>
 __device__ __forceinline__ StageMeta walker_next(Walker& w, int cta, int lane) {
   StageMeta d;
+  if (w.pos >= w.end && w.nq > 0) {  // next sub-range
+    walker_seek(w, w.q0_start, w.q0_end, w.q0_b, w.q0_pre, lane);
+    w.q0_start = w.q1_start; w.q0_end = w.q1_end; w.q0_b = w.q1_b; w.q0_pre = w.q1_pre;
+    --w.nq;
+  }
   if (w.pos >= w.end) {
     d.flags = F_END;
-    d.b = d.g = d.tok0 = d.ntok = d.slot = d.nchunk = d.pad = 0;
+    d.b = d.g = d.tok0 = d.ntok = d.nchunk = d.c0 = d.npieces = 0;
     return d;
   }
   const long long seg_end = w.seg_start + w.nch;
@@ -507,8 +608,18 @@ __device__ __forceinline__ StageMeta walker_next(Walker& w, int cta, int lane) {
   d.nchunk = (int)(stop - w.pos);
   d.flags = (w.pos == w.piece_start ? F_FIRST : 0) | (stop == piece_end ? F_LAST : 0) |
             (w.piece_start == w.seg_start && piece_end == seg_end ? F_DIRECT : 0);
-  d.slot = w.b * w.hkv + w.g + cta;
-  d.pad = 0;
+  d.c0 = cta;
+  d.npieces = 1;
+  if ((d.flags & F_LAST) && !(d.flags & F_DIRECT)) {
+    const long long c0 = owner_of(w.seg_start, w.total, w.grid), c1 = owner_of(seg_end - 1, w.total, w.grid);
+    int n = (int)(c1 - c0 + 1);
+    if (w.total < w.grid) {  // some CTAs have an empty range and hold no piece
+      n = 0;
+      for (long long c = c0; c <= c1; ++c) n += (w.total * c / w.grid != w.total * (c + 1) / w.grid);
+    }
+    d.c0 = (int)c0;
+    d.npieces = n;
+  }
   w.pos = stop;
   if (stop == piece_end && stop < w.end) {  // next piece starts a new segment
     w.piece_start = stop;
@@ -523,7 +634,7 @@ __device__ __forceinline__ StageMeta walker_next(Walker& w, int cta, int lane) {
 
 // ------------------------------------------------------------------ decode kernel
 template <int DT, int D, int G, int NW, int NSTAGES, bool MMA>
-__global__ void __launch_bounds__((NW + 1) * 32) decode_kernel(const __grid_constant__ CUtensorMap kmap,
+__global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_constant__ CUtensorMap kmap,
                                                                const __grid_constant__ CUtensorMap vmap,
                                                                const DecodeParams p) {
   using LY = Layout<D, G, NW, NSTAGES, MMA>;
@@ -533,6 +644,8 @@ __global__ void __launch_bounds__((NW + 1) * 32) decode_kernel(const __grid_cons
   const uint32_t sbase = smem_u32(smem);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + LY::BAR_OFF);
   uint64_t* empty = full + NSTAGES;
+  uint64_t* mfull = empty + NSTAGES;   // merge buffer j filled by the NW consumer warps
+  uint64_t* mempty = mfull + 2;        // merge buffer j released by the epilogue warp
   StageMeta* meta = reinterpret_cast<StageMeta*>(smem + LY::META_OFF);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
@@ -542,6 +655,10 @@ __global__ void __launch_bounds__((NW + 1) * 32) decode_kernel(const __grid_cons
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], NW);
     }
+    for (int j = 0; j < 2; ++j) {  // every lane arrives, so each lane's own smem writes/reads are ordered
+      mbar_init(&mfull[j], NW * 32);
+      mbar_init(&mempty[j], 32);
+    }
     fence_mbar_init();
   }
   __syncthreads();
@@ -550,7 +667,7 @@ __global__ void __launch_bounds__((NW + 1) * 32) decode_kernel(const __grid_cons
     // ================================================= producer warp
     const int B = p.batch, Hkv = p.num_kv_heads;
     const int cap = p.max_blocks_per_seq * p.block_size;
-    // pass 1: total chunks over all sequences
+    // pass 1: total chunks over all sequences (CTA 0 also writes out = 0 for empty sequences)
     long long tot = 0;
     bool clamped = false;
     for (int base = 0; base < B; base += 256) {
@@ -562,81 +679,74 @@ __global__ void __launch_bounds__((NW + 1) * 32) decode_kernel(const __grid_cons
           const int L = __ldg(p.context_lens + i);
           clamped |= (L < 0 || L > cap);
           s += (clamp_len(L, cap) + kChunk - 1) / kChunk;
+          if (cta == 0 && clamp_len(L, cap) == 0) {
+            uint4* o4 = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.out) + (size_t)i * p.num_q_heads * D);
+            for (int e = 0; e < p.num_q_heads * D * 2 / 16; ++e) o4[e] = make_uint4(0, 0, 0, 0);
+          }
         }
       }
       tot += warp_sum_ll(s);
     }
     if (clamped && cta == 0 && lane == 0) PA_RECORD_ERROR(PA_ERRBIT_INDEX);
     const long long C = tot * Hkv;
+    if (lane == 0) *reinterpret_cast<long long*>(smem + LY::MISC_OFF) = C;  // published by the first full barrier
     const long long x0 = C * cta / p.grid, x1 = C * (cta + 1) / p.grid;
-    // pass 2: the sequence holding chunk x0 (CTA 0 also publishes the prefix sums for the reduce)
+    // Walk order: the first piece, then the last piece, then the whole segments between.  Only
+    // those two pieces can be partial, so both halves of every segment cut between two CTAs
+    // finish early and its merge overlaps the rest of the stream instead of trailing it.
     Walker w;
-    w.pos = x0;
-    w.end = x1;
+    w.pos = w.end = 0;
     w.batch = B;
     w.hkv = Hkv;
     w.cap = cap;
+    w.grid = p.grid;
+    w.total = C;
     w.lens = p.context_lens;
-    int fb = -1;
-    long long fpre = 0;
-    {
-      long long run = 0;
-      for (int base = 0; base < B; base += 256) {
-        int v[8];
-        long long s = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int i = base + lane * 8 + j;
-          v[j] = i < B ? (clamp_len(__ldg(p.context_lens + i), cap) + kChunk - 1) / kChunk : 0;
-          s += v[j];
-        }
-        const long long incl = warp_incl_scan_ll(s, lane);
-        long long pre = run + incl - s;
-        int found = -1;
-        long long found_pre = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int i = base + lane * 8 + j;
-          if (i < B) {
-            if (cta == 0) p.ws_pre[i] = pre;
-            if (v[j] > 0 && pre * Hkv <= x0 && x0 < (pre + v[j]) * Hkv) {
-              found = i;
-              found_pre = pre;
-            }
-          }
-          pre += v[j];
-        }
-        const unsigned hit = __ballot_sync(0xffffffffu, found >= 0);
-        if (hit && fb < 0) {
-          const int src = __ffs(hit) - 1;
-          fb = __shfl_sync(0xffffffffu, found, src);
-          fpre = __shfl_sync(0xffffffffu, found_pre, src);
-        }
-        run += __shfl_sync(0xffffffffu, incl, 31);
-        if (fb >= 0 && cta != 0) break;
-      }
-      if (cta == 0 && lane == 0) p.ws_pre[B] = tot;
-    }
+    w.win_base = -64;
+    w.nq = 0;
     if (x0 < x1) {
-      load_window(w, fb, lane);
-      w.b = fb;
-      w.L = __shfl_sync(0xffffffffu, w.win_len, 0);
-      w.nch = (w.L + kChunk - 1) / kChunk;
-      w.g = (int)((x0 - fpre * Hkv) / w.nch);
-      w.seg_start = fpre * Hkv + (long long)w.g * w.nch;
-      w.piece_start = x0;
+      int b0, bl;
+      long long p0, pl;
+      find_seq(w, x0, lane, b0, p0);
+      find_seq(w, x1 - 1, lane, bl, pl);
+      walker_seek(w, x0, x1, b0, p0, lane);
+      const long long s0 = w.seg_start, e0 = s0 + w.nch;
+      const int Ll = clamp_len(__ldg(p.context_lens + bl), cap), nl = (Ll + kChunk - 1) / kChunk;
+      const long long sl = pl * Hkv + ((x1 - 1 - pl * Hkv) / nl) * nl, el = sl + nl;
+      const bool last_sep = sl > s0 && x1 < el;
+      const long long first_end = e0 < x1 ? e0 : x1, mid_end = last_sep ? sl : x1;
+      w.end = first_end;
+      if (last_sep) walker_push(w, sl, x1, bl, pl);
+      if (first_end < mid_end) {
+        int bm;
+        long long pm;
+        find_seq(w, first_end, lane, bm, pm);
+        walker_push(w, first_end, mid_end, bm, pm);
+      }
     }
+    // The walk runs kLookahead stages ahead of the TMA issue: each planned
+    // stage's block-table entries are fetched with cp.async into the plan
+    // ring, so no lookup latency sits between a freed stage and its refill.
     const int32_t* bt_all = p.block_tables;
     const int mb = p.max_blocks_per_seq, bs = p.block_size;
-    auto lookup = [&](const StageMeta& d) -> int {
-      if (d.flags & F_END || lane >= d.nchunk) return 0;
-      return __ldg(bt_all + (size_t)d.b * mb + (d.tok0 + lane * kChunk) / bs);
+    StageMeta* plan = reinterpret_cast<StageMeta*>(smem + LY::PLAN_OFF);
+    int32_t* plan_phys = reinterpret_cast<int32_t*>(smem + LY::PLAN_OFF + kPlanRing * sizeof(StageMeta));
+    auto plan_push = [&](int j) {
+      const StageMeta dn = walker_next<LY::CPS>(w, cta, lane);
+      const int slot = j % kPlanRing;
+      if (lane == 0) plan[slot] = dn;
+      if (!(dn.flags & F_END) && lane < dn.nchunk)
+        cp_async4(plan_phys + slot * 8 + lane, bt_all + (size_t)dn.b * mb + (dn.tok0 + lane * kChunk) / bs);
+      cp_async_commit();
     };
-    StageMeta d = walker_next<LY::CPS>(w, cta, lane);
-    int phys = lookup(d);
+    for (int j = 0; j < kLookahead; ++j) plan_push(j);
     bool ok = true;
     int k = 0;
     for (;; ++k) {
+      cp_async_wait<kLookahead - 1>();  // this lane's lookups for stage k have landed
+      __syncwarp();
+      const StageMeta d = plan[k % kPlanRing];
+      const int phys = lane < d.nchunk ? plan_phys[(k % kPlanRing) * 8 + lane] : 0;
       const int st = k % NSTAGES;
       if (k >= NSTAGES && !mbar_wait(&empty[st], ((k / NSTAGES) - 1) & 1)) {
         ok = false;
@@ -668,15 +778,142 @@ __global__ void __launch_bounds__((NW + 1) * 32) decode_kernel(const __grid_cons
                               ((size_t)d.b * p.num_q_heads + (size_t)d.g * G) * D * 2;
         bulk_load(smem + LY::QS_OFF + st * LY::QSLOT, qsrc, LY::QSLOT, &full[st]);
       }
-      d = walker_next<LY::CPS>(w, cta, lane);
-      phys = lookup(d);
+      plan_push(k + kLookahead);
     }
+    cp_async_wait<0>();
     if (!ok && lane == 0) PA_RECORD_ERROR(PA_ERRBIT_TIMEOUT);
     // drain: every copy this CTA issued has landed before the warp leaves
     if (lane == 0) {
       for (int j = max(0, k - NSTAGES + 1); j < k; ++j)
         if (!mbar_wait(&full[j % NSTAGES], (j / NSTAGES) & 1)) PA_RECORD_ERROR(PA_ERRBIT_TIMEOUT);
     }
+    return;
+  }
+
+  if (warp == NW + 1) {
+    // ================================================= epilogue warp
+    // Per finished piece: merge the NW consumer warps' states, then write the
+    // output (whole segment) or an fp32 partial.  A partial is counted (atomic
+    // add after a fence, no waiting); the CTA that completes a segment's last
+    // piece merges all of its partials by the log-sum-exp rule and writes the
+    // output.  Only a CTA's first and last pieces can be partial, and the
+    // producer walks them first, so these merges overlap the stream.
+    const long long* line_total = reinterpret_cast<const long long*>(smem + LY::MISC_OFF);
+    bool ok = true;
+    for (int pc = 0;; ++pc) {
+      const int j = pc & 1;
+      if (!mbar_wait(&mfull[j], (pc >> 1) & 1)) {
+        ok = false;
+        break;
+      }
+      uint8_t* mb = smem + LY::M_OFF + j * LY::MB_BYTES;
+      const float* mo = reinterpret_cast<const float*>(mb + LY::MB_O);
+      const float* mml = reinterpret_cast<const float*>(mb + LY::MB_ML);
+      const StageMeta d = *reinterpret_cast<const StageMeta*>(mb + LY::MB_DESC);
+      if (d.flags & F_END) break;
+      const bool direct = d.flags & F_DIRECT;
+      const size_t slot = (size_t)d.b * p.num_kv_heads + d.g + cta;
+      T* outp = reinterpret_cast<T*>(p.out) + ((size_t)d.b * p.num_q_heads + (size_t)d.g * G) * D;
+      for (int i = lane; i < G * D; i += 32) {
+        const int h = i / D, dd = i - h * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w2 = 0; w2 < NW; ++w2) M = fmaxf(M, mml[(w2 * G + h) * 2]);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < NW; ++w2) {
+          const float sc = fast_exp2(mml[(w2 * G + h) * 2] - M);
+          num = fmaf(sc, mo[(w2 * G + h) * D + dd], num);
+          den = fmaf(sc, mml[(w2 * G + h) * 2 + 1], den);
+        }
+        if (direct) {
+          outp[i] = Elt<DT>::from_f(num / den);
+        } else {
+          const size_t srow = slot * G + h;
+          p.ws_o[srow * D + dd] = num;
+          if (dd == 0) {
+            p.ws_m[srow] = M;
+            p.ws_l[srow] = den;
+          }
+        }
+      }
+      mbar_arrive(&mempty[j]);  // this lane is done with the buffer
+      if (direct) continue;
+      __threadfence();  // this piece's partial is visible device-wide before it is counted
+      __syncwarp();
+      const long long C_s = *line_total;
+      {
+        const int sg = d.b * p.num_kv_heads + d.g;
+        int last = 0;
+        if (lane == 0) {
+          last = atomicAdd(p.ws_cnt + sg, 1) == d.npieces - 1;
+          if (last) atomicExch(p.ws_cnt + sg, 0);  // leave the counter at zero for the next call
+        }
+        if (!__shfl_sync(0xffffffffu, last, 0)) continue;  // another CTA finishes this segment
+        __threadfence();
+        // CTAs holding a piece of this segment: c0, c0+1, ... (when the line has fewer chunks than
+        // CTAs, some CTAs hold nothing and are skipped)
+        const bool dense = C_s >= p.grid;
+        auto piece_cta = [&](int n) -> long long {
+          if (dense) return d.c0 + n;
+          for (long long k2 = d.c0, m2 = 0;; ++k2)
+            if (C_s * k2 / p.grid != C_s * (k2 + 1) / p.grid && m2++ == n) return k2;
+        };
+        // Normalised weight of each piece per head, w[h][n] = 2^(m_n - M) / sum_n 2^(m_n - M) l_n;
+        // then out = sum_n w[h][n] o_n with every load independent, so the merge costs a few L2
+        // round trips instead of one per element.
+        float* wts = reinterpret_cast<float*>(smem + LY::WTS_OFF);
+        const int np = d.npieces;
+        if (np <= kMaxPieces) {
+          for (int h = lane; h < G; h += 32) {
+            float Mh = -INFINITY, den = 0.f;
+            for (int n = 0; n < np; ++n) Mh = fmaxf(Mh, __ldcg(p.ws_m + ((size_t)sg + piece_cta(n)) * G + h));
+            for (int n = 0; n < np; ++n) {
+              const size_t srow = ((size_t)sg + piece_cta(n)) * G + h;
+              const float w = fast_exp2(__ldcg(p.ws_m + srow) - Mh);
+              wts[h * np + n] = w;
+              den = fmaf(w, __ldcg(p.ws_l + srow), den);
+            }
+            const float inv = 1.f / den;
+            for (int n = 0; n < np; ++n) wts[h * np + n] *= inv;
+          }
+          __syncwarp();
+          T* outp = reinterpret_cast<T*>(p.out) + ((size_t)d.b * p.num_q_heads + (size_t)d.g * G) * D;
+#pragma unroll 4
+          for (int i0 = lane * 4; i0 < G * D; i0 += 128) {
+            const int h = i0 / D, dd = i0 - h * D;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int n = 0; n < np; ++n) {
+              const float w = wts[h * np + n];
+              const float4 o4 = __ldcg(reinterpret_cast<const float4*>(
+                  p.ws_o + (((size_t)sg + piece_cta(n)) * G + h) * D + dd));
+              acc.x = fmaf(w, o4.x, acc.x); acc.y = fmaf(w, o4.y, acc.y);
+              acc.z = fmaf(w, o4.z, acc.z); acc.w = fmaf(w, o4.w, acc.w);
+            }
+            uint2 pk;
+            pk.x = Elt<DT>::from_f2(acc.x, acc.y);
+            pk.y = Elt<DT>::from_f2(acc.z, acc.w);
+            *reinterpret_cast<uint2*>(outp + i0) = pk;
+          }
+          __syncwarp();
+        } else {  // more pieces than the weight area holds (only with far more CTAs than chunks)
+          T* outp = reinterpret_cast<T*>(p.out) + ((size_t)d.b * p.num_q_heads + (size_t)d.g * G) * D;
+          for (int i = lane; i < G * D; i += 32) {
+            const int h = i / D, dd = i - h * D;
+            float M = -INFINITY, num = 0.f, den = 0.f;
+            for (int n = 0; n < np; ++n) M = fmaxf(M, __ldcg(p.ws_m + ((size_t)sg + piece_cta(n)) * G + h));
+            for (int n = 0; n < np; ++n) {
+              const size_t srow = ((size_t)sg + piece_cta(n)) * G + h;
+              const float w = fast_exp2(__ldcg(p.ws_m + srow) - M);
+              num = fmaf(w, __ldcg(p.ws_o + srow * D + dd), num);
+              den = fmaf(w, __ldcg(p.ws_l + srow), den);
+            }
+            outp[i] = Elt<DT>::from_f(num / den);
+          }
+        }
+      }
+    }
+    if (!ok && lane == 0) PA_RECORD_ERROR(PA_ERRBIT_TIMEOUT);
     return;
   }
 
@@ -687,9 +924,24 @@ __global__ void __launch_bounds__((NW + 1) * 32) decode_kernel(const __grid_cons
   float* qf = reinterpret_cast<float*>(smem + LY::QF_OFF) + warp * G * D;
   const uint32_t qbase = smem_u32(qf);
   const uint32_t pbase = sbase + LY::P_OFF + warp * 32 * G * 4;
-  float* merge_o = reinterpret_cast<float*>(smem + LY::M_OFF);
-  float* merge_ml = reinterpret_cast<float*>(smem + LY::ML_OFF);
   bool ok = true;
+  int pc = 0;  // pieces handed to the epilogue warp
+  // Hand a finished piece (or the end marker) to the epilogue through merge buffer pc%2.
+  auto hand_over = [&](const StageMeta& d, bool end) -> bool {
+    const int j = pc & 1;
+    if (pc >= 2 && !mbar_wait(&mempty[j], ((pc >> 1) - 1) & 1)) return false;
+    uint8_t* mb = smem + LY::M_OFF + j * LY::MB_BYTES;
+    if (!end) c.stash(reinterpret_cast<float*>(mb + LY::MB_O) + warp * G * D,
+                      reinterpret_cast<float*>(mb + LY::MB_ML) + warp * G * 2, lane);
+    if (warp == 0 && lane == 0) {
+      StageMeta dd = d;
+      if (end) dd.flags = F_END;
+      *reinterpret_cast<StageMeta*>(mb + LY::MB_DESC) = dd;
+    }
+    mbar_arrive(&mfull[j]);
+    ++pc;
+    return true;
+  };
   for (int k = 0;; ++k) {
     const int st = k % NSTAGES;
     if (!mbar_wait(&full[st], (k / NSTAGES) & 1)) {
@@ -697,7 +949,10 @@ __global__ void __launch_bounds__((NW + 1) * 32) decode_kernel(const __grid_cons
       break;
     }
     const StageMeta d = meta[st];
-    if (d.flags & F_END) break;
+    if (d.flags & F_END) {
+      ok = hand_over(d, true);
+      break;
+    }
     if (d.flags & F_FIRST) {
       c.init();
       c.load_q(smem + LY::QS_OFF + st * LY::QSLOT, qf, p.scale_log2, lane);
@@ -713,106 +968,17 @@ __global__ void __launch_bounds__((NW + 1) * 32) decode_kernel(const __grid_cons
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
-    if (d.flags & F_LAST) {
-      // merge the NW warps' states of this piece; write out (whole segment) or a partial
-      c.stash(merge_o + warp * G * D, merge_ml + warp * G * 2, lane);
-      named_barrier_sync(1, NW * 32);
-      const int hq0 = d.g * G;
-      for (int i = threadIdx.x; i < G * D; i += NW * 32) {
-        const int h = i / D, dd = i - h * D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w2 = 0; w2 < NW; ++w2) M = fmaxf(M, merge_ml[(w2 * G + h) * 2]);
-        float num = 0.f, den = 0.f;
-#pragma unroll
-        for (int w2 = 0; w2 < NW; ++w2) {
-          const float sc = fast_exp2(merge_ml[(w2 * G + h) * 2] - M);
-          num = fmaf(sc, merge_o[(w2 * G + h) * D + dd], num);
-          den = fmaf(sc, merge_ml[(w2 * G + h) * 2 + 1], den);
-        }
-        if (d.flags & F_DIRECT) {
-          const size_t row = (size_t)d.b * p.num_q_heads + hq0 + h;
-          reinterpret_cast<T*>(p.out)[row * D + dd] = Elt<DT>::from_f(num / den);
-        } else {
-          const size_t srow = (size_t)d.slot * G + h;
-          p.ws_o[srow * D + dd] = num;
-          if (dd == 0) {
-            p.ws_m[srow] = M;
-            p.ws_l[srow] = den;
-          }
-        }
-      }
-      named_barrier_sync(1, NW * 32);
+    if ((d.flags & F_LAST) && !hand_over(d, false)) {
+      ok = false;
+      break;
     }
   }
   if (!ok && lane == 0) PA_RECORD_ERROR(PA_ERRBIT_TIMEOUT);
 }
 
-// ------------------------------------------------------------------ reduce
-// One warp per (b, h): merges the pieces of segment (b, h/G) written by CTAs
-// c0..c1 (out = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c), writes zeros
-// for empty sequences, and leaves whole-segment pieces (already written) alone.
-template <int DT, int D, int G>
-__global__ void __launch_bounds__(128) decode_reduce_kernel(const DecodeParams p) {
-  using T = typename Elt<DT>::T;
-  constexpr int DPL = D / 32;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 4 + warp;  // b * Hq + h
-  if (row >= p.batch * p.num_q_heads) return;
-  const int b = row / p.num_q_heads, h = row - b * p.num_q_heads;
-  const int g = h / G, j = h - g * G;
-  const long long pre = p.ws_pre[b];
-  const long long nch = p.ws_pre[b + 1] - pre;
-  T* out = reinterpret_cast<T*>(p.out) + (size_t)row * D + lane * DPL;
-  if (nch <= 0) {
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) out[e] = Elt<DT>::from_f(0.f);
-    return;
-  }
-  const long long Hkv = p.num_kv_heads, grid = p.grid;
-  const long long C = Hkv * p.ws_pre[p.batch];
-  const long long cs = Hkv * pre + g * nch, ce = cs + nch;
-  const long long c0 = ((cs + 1) * grid - 1) / C, c1 = (ce * grid - 1) / C;  // owners of the first and last chunk
-  if (c0 == c1) return;
-  float M = -INFINITY;
-  for (long long c = c0; c <= c1; ++c) {
-    if (C * c / grid == C * (c + 1) / grid) continue;  // a CTA with an empty range wrote nothing
-    const long long slot = (long long)b * p.num_kv_heads + g + c;
-    M = fmaxf(M, p.ws_m[slot * G + j]);
-  }
-  float acc[DPL];
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-  float den = 0.f;
-  for (long long c = c0; c <= c1; ++c) {
-    if (C * c / grid == C * (c + 1) / grid) continue;
-    const long long srow = ((long long)b * p.num_kv_heads + g + c) * G + j;
-    const float w = fast_exp2(p.ws_m[srow] - M);
-    den = fmaf(w, p.ws_l[srow], den);
-    const float* o = p.ws_o + srow * D + lane * DPL;
-    if constexpr (DPL == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(o);
-      acc[0] = fmaf(w, v.x, acc[0]); acc[1] = fmaf(w, v.y, acc[1]);
-      acc[2] = fmaf(w, v.z, acc[2]); acc[3] = fmaf(w, v.w, acc[3]);
-    } else {
-      const float2 v = *reinterpret_cast<const float2*>(o);
-      acc[0] = fmaf(w, v.x, acc[0]); acc[1] = fmaf(w, v.y, acc[1]);
-    }
-  }
-  const float inv = 1.f / den;
-  if constexpr (DPL == 4) {
-    uint2 wv;
-    wv.x = Elt<DT>::from_f2(acc[0] * inv, acc[1] * inv);
-    wv.y = Elt<DT>::from_f2(acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<uint2*>(out) = wv;
-  } else {
-    *reinterpret_cast<uint32_t*>(out) = Elt<DT>::from_f2(acc[0] * inv, acc[1] * inv);
-  }
-}
-
 // ------------------------------------------------------------------ host side
 constexpr int kNW = 2;       // consumer warps per CTA (64-token stages)
-constexpr int kStages = 3;   // ring depth
+constexpr int kStages = 2;   // ring depth (three CTAs per SM)
 
 template <int D, int G>
 constexpr int alloc_bytes() {
@@ -838,7 +1004,7 @@ int smem_per_cta(int D, int G) {
 struct Plan {
   int grid;
   size_t ws_bytes;
-  size_t off_m, off_l, off_o;
+  size_t off_m, off_l, off_o;  // the piece counters sit at offset 0
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -860,7 +1026,7 @@ bool make_plan(int batch, int Hq, int Hkv, int D, int num_partitions, Plan* pl) 
   }
   pl->grid = grid;
   const size_t slots = (size_t)batch * Hkv + grid;
-  pl->off_m = align256((size_t)(batch + 1) * 8);
+  pl->off_m = align256((size_t)batch * Hkv * 4);
   pl->off_l = pl->off_m + align256(slots * G * 4);
   pl->off_o = pl->off_l + align256(slots * G * 4);
   pl->ws_bytes = pl->off_o + align256(slots * G * D * 4);
@@ -880,10 +1046,7 @@ int launch(const CUtensorMap& km, const CUtensorMap& vm, const DecodeParams& p, 
       return PA_ERR_CUDA;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  kern<<<p.grid, (kNW + 1) * 32, LY::ALLOC, st>>>(km, vm, p);
-  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  const int rows = p.batch * p.num_q_heads;
-  decode_reduce_kernel<DT, D, G><<<(rows + 3) / 4, 128, 0, st>>>(p);
+  kern<<<p.grid, (kNW + 2) * 32, LY::ALLOC, st>>>(km, vm, p);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   return PA_OK;
 }
@@ -955,7 +1118,7 @@ extern "C" int pa_decode(const void* q, const void* k_cache, const void* v_cache
   p.block_tables = block_tables;
   p.context_lens = context_lens;
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
-  p.ws_pre = reinterpret_cast<long long*>(ws);
+  p.ws_cnt = reinterpret_cast<int*>(ws);
   p.ws_m = reinterpret_cast<float*>(ws + pl.off_m);
   p.ws_l = reinterpret_cast<float*>(ws + pl.off_l);
   p.ws_o = reinterpret_cast<float*>(ws + pl.off_o);

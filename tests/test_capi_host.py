@@ -97,7 +97,7 @@ def test_decode_plan():
         grid, maxp, ws = pa.decode_plan(B, Hq, Hkv, D, 1000)
         assert grid >= 1 and maxp == B * Hkv + grid
         G = Hq // Hkv
-        assert ws >= (B + 1) * 8 + maxp * G * (D + 2) * 4
+        assert ws >= B * Hkv * 4 + maxp * G * (D + 2) * 4
         assert pa.lib.pa_decode_workspace_size(B, Hq, Hkv, D, 1000, 0) == ws
     grid, maxp, ws = pa.decode_plan(4, 8, 2, 128, 1000, num_partitions=7)
     assert grid == 7 and maxp == 4 * 2 + 7

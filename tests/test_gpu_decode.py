@@ -169,3 +169,20 @@ def test_decode_large_logits():
     got = out.float().cpu().numpy()
     assert np.isfinite(got).all()
     assert_close(got, ref, "q x10")
+
+
+def test_decode_workspace_reuse_across_calls():
+    """The piece counters at the head of the workspace return to zero after every call, so one workspace
+    serves many calls (different partition counts and batches) without clearing."""
+    wl = make_workload("qwen_decode")
+    ref = _oracle_decode(wl)
+    out0, kc, vc, bt, lens, bt_h, lens_h = gpu_step(wl)
+    maxL = int(lens_h.max())
+    need = max(pa.decode_plan(wl.batch, 16, 8, 128, maxL, n)[2] for n in (0, 3, 1000))
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    q = wl.q.cuda()
+    for n in (0, 3, 1000, 0, 3):
+        out = pa.decode(q, kc, vc, bt, lens, maxL, wl.scale, workspace=ws, num_partitions=n)
+        assert_close(out.float().cpu().numpy(), ref, f"reuse partitions={n}")
+    torch.cuda.synchronize()
+    assert int(ws[: wl.batch * 8 * 4].view(torch.int32).abs().sum().item()) == 0
