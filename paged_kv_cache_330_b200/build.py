@@ -1,6 +1,6 @@
 """Build libpaged_attn.so in-tree with nvcc for sm_100a.
 
-    python -m paged_kv_cache_330_b200.build [--debug-ptxas]
+    python paged_kv_cache_330_b200/build.py [--debug-ptxas]
 
 Each source compiles to an object under ``_build/`` (in parallel), then nvcc
 links the shared library next to this file.  Nothing is JIT-compiled at

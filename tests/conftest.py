@@ -12,11 +12,10 @@ def pytest_configure(config):
 
 
 def pytest_sessionstart(session):
-    """Build libpaged_attn.so in-tree if it is missing (the binding refuses to import without it)."""
-    lib = os.path.join(ROOT, "paged_kv_cache_330_b200", "libpaged_attn.so")
-    if not os.path.exists(lib):
-        import importlib.util
-        spec = importlib.util.spec_from_file_location("_pa_build", os.path.join(ROOT, "paged_kv_cache_330_b200", "build.py"))
-        mod = importlib.util.module_from_spec(spec)
-        spec.loader.exec_module(mod)
-        mod.build()
+    """(Re)build libpaged_attn.so in-tree when it is missing or older than its sources (incremental; the
+    binding refuses to import without it)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("_pa_build", os.path.join(ROOT, "paged_kv_cache_330_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
