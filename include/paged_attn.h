@@ -144,6 +144,29 @@ int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int
               void* out, void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Decode with library-owned scratch (no counterpart on the source pages).   */
+/* Same computation, arguments and results as pa_decode, but without a      */
+/* workspace argument: for callers that cannot allocate device memory where */
+/* they run decode (inside CUDA graph capture, under a fixed memory pool,   */
+/* or on a serving path that must not block on an allocation).  The scratch */
+/* is one static device array of PA_DECODE_STATIC_SCRATCH_BYTES, reserved   */
+/* on every GPU that loads the library until the process exits.  Calls that */
+/* would need more (pa_decode_workspace_size() larger than that) return     */
+/* PA_ERR_WORKSPACE.  Nothing is allocated: the call only clears the piece */
+/* counters at the head of the array (cudaMemsetAsync on `stream`) and runs */
+/* the decode kernel.  The first call on a device looks up the array's     */
+/* device address (cudaGetSymbolAddress) with that device current; make     */
+/* that first call before any stream capture.  All calls share the one      */
+/* array and it keeps the last call's contents, so calls whose work overlaps */
+/* on the GPU (other streams, other threads) race: serialise them.          */
+/* ------------------------------------------------------------------------ */
+#define PA_DECODE_STATIC_SCRATCH_BYTES (8u << 20)
+int pa_decode_static_scratch(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                             int max_blocks_per_seq, const int32_t* context_lens, int batch, int num_q_heads,
+                             int num_kv_heads, int head_dim, int block_size, int num_blocks, int max_context_len,
+                             float scale, int dtype, int num_partitions_or_0, void* out, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* Chunked prefill (P3 s1.1 / s3.1 PCP: prefill cut into chunks on one       */
 /* device).  Sequence b appends C_b = query_start_loc[b+1]-query_start_loc[b]*/
 /* query tokens whose K/V were already written (pa_write_kv) so that the    */

@@ -22,12 +22,13 @@ import os
 import numpy as np
 
 __all__ = ["PagedAttnError", "PoolOutOfBlocks", "BlockPool", "write_kv", "copy_blocks", "decode", "decode_plan",
+           "decode_static_scratch",
            "prefill_chunk", "device_error", "lib", "LIB_PATH", "replay_ops", "version"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpaged_attn.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is not built; run `python -m paged_kv_cache_330_b200.build` "
+    raise ImportError(f"{LIB_PATH} is not built; run `python paged_kv_cache_330_b200/build.py` "
                       "(there is no fallback path)")
 
 lib = ctypes.CDLL(LIB_PATH)
@@ -52,6 +53,7 @@ _SIGS = {
     "pa_decode_plan": (_i, [_i, _i, _i, _i, _i, _i, _ip, _ip, ctypes.POINTER(_sz)]),
     "pa_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "pa_decode": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _sz, _i, _vp, _vp]),
+    "pa_decode_static_scratch": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp, _vp]),
     "pa_prefill_chunk": (_i, [_vp, _vp, _i, _i, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _vp]),
     "pa_device_error": (_i, [_ip]),
     "pa_pool_create": (_vp, [_i, _i, _i32p]),
@@ -165,6 +167,23 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len: int
                          _ptr(context_lens), B, Hq, Hkv, D, bs, NB, int(max_context_len), float(scale),
                          _dtype_code(q), _ptr(workspace), ws_bytes, int(num_partitions), _ptr(out),
                          _stream_handle(stream)), "pa_decode")
+    return out
+
+
+def decode_static_scratch(q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,
+                          out=None, num_partitions: int = 0, stream=None):
+    """pa_decode without a workspace argument: the library's static device scratch is used instead (for callers
+    that must not allocate where they run decode).  Calls overlapping on the GPU race on that scratch."""
+    torch = _torch()
+    _contig(q, k_cache, v_cache, block_tables, context_lens, out)
+    B, Hq, D = q.shape
+    NB, bs, Hkv, _ = k_cache.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib.pa_decode_static_scratch(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                        int(block_tables.shape[1]), _ptr(context_lens), B, Hq, Hkv, D, bs, NB,
+                                        int(max_context_len), float(scale), _dtype_code(q), int(num_partitions),
+                                        _ptr(out), _stream_handle(stream)), "pa_decode_static_scratch")
     return out
 
 

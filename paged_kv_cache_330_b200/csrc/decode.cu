@@ -39,6 +39,7 @@
 //     keeps it exact to about 2^-17 instead of the 2^-9 of one bf16 rounding.
 
 #include <algorithm>
+#include <mutex>
 #include <type_traits>
 
 #include "common.cuh"
@@ -1142,4 +1143,56 @@ extern "C" int pa_decode(const void* q, const void* k_cache, const void* v_cache
   if (dtype == PA_BF16)
     return head_dim == 128 ? dispatch_g<PA_BF16, 128>(G, km, vm, p, st) : dispatch_g<PA_BF16, 64>(G, km, vm, p, st);
   return head_dim == 128 ? dispatch_g<PA_F16, 128>(G, km, vm, p, st) : dispatch_g<PA_F16, 64>(G, km, vm, p, st);
+}
+
+// ------------------------------------------------------------------ decode with library-owned scratch
+// Some callers cannot allocate device memory at the point where they run
+// decode: code that runs while a CUDA graph is being captured (cudaMalloc is
+// not allowed there), engines that hand out memory only from a pool fixed at
+// start-up, or hosts that forbid allocation on the serving path because an
+// allocation can block on the device.  For them the scratch lives in a static
+// array of this file, set aside once per GPU when the library is loaded.
+static __device__ __align__(256) unsigned char g_decode_scratch[PA_DECODE_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of g_decode_scratch on the current device, looked up once per
+// device (the array's host-side name is not a device address).
+int static_scratch_ptr(void** out) {
+  static std::mutex mu;
+  static void* ptrs[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return PA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return PA_ERR_CUDA;
+    ptrs[dev] = p;
+  }
+  *out = ptrs[dev];
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" int pa_decode_static_scratch(const void* q, const void* k_cache, const void* v_cache,
+                                        const int32_t* block_tables, int max_blocks_per_seq,
+                                        const int32_t* context_lens, int batch, int num_q_heads, int num_kv_heads,
+                                        int head_dim, int block_size, int num_blocks, int max_context_len, float scale,
+                                        int dtype, int num_partitions_or_0, void* out, void* stream) {
+  size_t need = 0;
+  int s = pa_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_partitions_or_0, nullptr,
+                         nullptr, &need);
+  if (s != PA_OK) return s;
+  if (need > PA_DECODE_STATIC_SCRATCH_BYTES) return PA_ERR_WORKSPACE;  // batch too large for the static scratch
+  void* scratch = nullptr;
+  if ((s = static_scratch_ptr(&scratch)) != PA_OK) return s;
+  // The head of the scratch holds the per-segment piece counters, which must start at zero.  A
+  // completed call leaves them at zero, but clear them anyway so an earlier failed call cannot leak in.
+  if (batch > 0 && num_kv_heads > 0 &&
+      cudaMemsetAsync(scratch, 0, (size_t)batch * num_kv_heads * sizeof(int), (cudaStream_t)stream) != cudaSuccess)
+    return PA_ERR_CUDA;
+  return pa_decode(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch, num_q_heads,
+                   num_kv_heads, head_dim, block_size, num_blocks, max_context_len, scale, dtype, scratch,
+                   PA_DECODE_STATIC_SCRATCH_BYTES, num_partitions_or_0, out, stream);
 }
