@@ -50,7 +50,10 @@ WORKLOAD_TEXT = {
 
 # DRAM bytes (read + write) per launch of the decode split kernel from one ncu capture of this workload,
 # valid only for the kernel source it was taken on (sha256 prefix of decode.cu + common.cuh).
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    "qwen_decode": {"bytes": 316_989_184, "src": "27d8eb8781511c66"},
+    "llama70b_long": {"bytes": 1_588_751_424, "src": "27d8eb8781511c66"},
+}
 
 
 def kernel_source_hash() -> str:
