@@ -46,6 +46,8 @@ WORKLOAD_TEXT = {
     "prefix_sweep": "prefix-shared decode: batch 256 = 8 groups x 32 sharing a 2048-token prefix, suffix uniform[0,512], "
                     "16 q / 8 kv heads, head_dim 128, bf16",
     "tiny": "tiny decode: 4 seqs, 4/4 heads, head_dim 64, fp16, block_size 16",
+    "prefill": "chunked prefill: 8 seqs, each a 512-token causal chunk appended to an 8192-token paged context, "
+               "32 q / 8 kv heads, head_dim 128, bf16, block_size 16",
 }
 
 # DRAM bytes (read + write) per launch of the decode split kernel from one ncu capture of this workload,
@@ -62,6 +64,28 @@ def kernel_source_hash() -> str:
         with open(os.path.join(ROOT, "paged_kv_cache_330_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+def measured_bf16_peak():
+    """(burst, sustained) dense bf16 TFLOP/s measured on this machine, or the fallback figure."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            d = json.load(fh)
+        return float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return 1590.0, 1400.0, "fallback"
+
+
+def prefill_flops(wl) -> float:
+    """4*D flops per visible (query, key) pair: query i of a C-token chunk on L tokens sees L-C+i+1 keys."""
+    c = wl.cfg
+    tot = 0
+    for b in range(wl.batch):
+        C = int(wl.query_start_loc[b + 1] - wl.query_start_loc[b])
+        L = int(wl.context_lens[b])
+        tot += C * (L - C) + C * (C + 1) // 2
+    return float(tot) * c["num_q_heads"] * 4 * c["head_dim"]
 
 
 def measured_hbm_peak():
@@ -419,6 +443,78 @@ def run_ours(args):
     return 0
 
 
+def run_prefill(args):
+    """Chunked-prefill step: pa_write_kv of every chunk token, then pa_prefill_chunk (tcgen05)."""
+    import torch
+    import paged_kv_cache_330_b200 as pa
+    from workloads import make_workload
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = make_workload("prefill")
+    c = wl.cfg
+    _, bt, lens, sm, _ = pa.replay_ops(wl.ops, wl.num_blocks, c["block_size"], wl.free_order, wl.batch)
+    kc, vc, q = wl.k_cache0.to(dev), wl.v_cache0.to(dev), wl.q.to(dev)
+    kn, vn, smd = wl.k_new.to(dev), wl.v_new.to(dev), torch.from_numpy(sm).to(dev)
+    btd, lensd = torch.from_numpy(bt).to(dev), torch.from_numpy(lens).to(dev)
+    qsl = torch.from_numpy(wl.query_start_loc).to(dev)
+    Cmax = int(np.diff(wl.query_start_loc).max())
+    out = torch.empty_like(q)
+    cs = torch.cuda.Stream(dev)
+    stream = torch.cuda.current_stream(dev)
+    wr = lambda st: pa.write_kv(kn, vn, smd, kc, vc, stream=st)
+    pf = lambda st: pa.prefill_chunk(q, qsl, kc, vc, btd, lensd, Cmax, wl.scale, out=out, stream=st)
+    for _ in range(args.warmup):
+        wr(stream)
+        pf(stream)
+    torch.cuda.synchronize(dev)
+    assert pa.device_error() == 0
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cs):
+            fn()
+        return g
+
+    g_step = capture(lambda: (wr(cs), pf(cs)))
+    g_pf = capture(lambda: pf(cs))
+    K = args.steps
+    for _ in range(3):
+        g_step.replay()
+    torch.cuda.synchronize(dev)
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    with ClockSampler(0) as clk:
+        e[0].record(stream)
+        for _ in range(K):
+            g_step.replay()
+        e[1].record(stream)
+        e[2].record(stream)
+        for _ in range(K):
+            g_pf.replay()
+        e[3].record(stream)
+        torch.cuda.synchronize(dev)
+    assert pa.device_error() == 0
+    ms_step = e[0].elapsed_time(e[1]) / K
+    ms_pf = e[2].elapsed_time(e[3]) / K
+    fl = prefill_flops(wl)
+    burst, sustained, kind = measured_bf16_peak()
+    line = {
+        "metric": "chunked prefill TFLOP/s (bf16, causal, paged context)", "value": fl / (ms_step * 1e-3) / 1e12,
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": K, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": str(c["dtype"]),
+        "data": "synthetic", "config": {"workload": WORKLOAD_TEXT["prefill"], "flops_per_step": fl},
+        "roofline": {"bound": "tensor", "kernel": "pa_prefill_chunk (tcgen05/TMEM, TMA)",
+                     "achieved": fl / (ms_pf * 1e-3) / 1e12, "peak": burst, "peak_kind": kind + " burst",
+                     "unit": "TFLOP/s", "frac": fl / (ms_pf * 1e-3) / 1e12 / burst,
+                     "frac_of_sustained": fl / (ms_pf * 1e-3) / 1e12 / sustained, "traffic": None,
+                     "avg_launch_ms": ms_pf},
+        "gpu_launches": 2 * K,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -436,6 +532,8 @@ def main():
         if args.steps * args.ref_budget > 120:
             args.ref_budget = max(1.0, 120.0 / max(1, args.steps + args.warmup))
         return run_reference(args)
+    if args.workload == "prefill":
+        return run_prefill(args)
     return run_ours(args)
 
 
