@@ -8,28 +8,32 @@
 // that it now holds L_b tokens; query i sits at position p = L_b - C_b + i and
 //   out[i][h] = sum_{t <= p} softmax_t(scale <q[i][h], K_b[t][h/G]>) V_b[t][h/G].
 //
-// One CTA per (128 query rows, query head, sequence).  Keys are walked in
-// tiles of 128 (the only dense contraction on the path, so it runs on the
-// 5th-generation tensor cores):
-//   * a TMA producer warp loads the Q tile once and, per key tile, 16-row K
-//     and V boxes gathered through the block table (128-byte swizzle, no
-//     multicast) into a two-stage ring;
-//   * one thread of the MMA warp issues S = Q K^T (M 128, N 128, K 128) into
-//     one of two TMEM buffers and O += P V into a TMEM accumulator
-//     (tcgen05.mma kind::f16, fp32 accumulate), completions signalled with
+// This is the one dense contraction on the path, so it runs on the
+// 5th-generation tensor cores.  One CTA owns two 128-row query tiles that read
+// the same keys: two query heads of one KV group over the same rows (or, when
+// a group has one head, two consecutive row tiles of it).  Keys are walked in
+// tiles of 64:
+//   * a TMA producer warp loads both query tiles once and, per key tile, 16-row
+//     K and V boxes gathered through the block table (128-byte swizzle, no
+//     multicast) into separate three-stage K and V rings shared by both query
+//     tiles (a K slot frees after the S products, a V slot after the PVs, so
+//     K runs ahead);
+//   * one thread of the MMA warp issues, per key tile, S_t = Q_t K^T for both
+//     query tiles (M 128, N 64, K 128) into per-tile double-buffered TMEM, then
+//     O_t += P_t V for the previous key tile (M 128, N 128, K 64), with fp32
+//     accumulation (tcgen05.mma kind::f16) and completions signalled with
 //     tcgen05.commit on mbarriers;
-//   * four softmax warps (thread r = query row r = TMEM lane r) read S with
-//     tcgen05.ld, apply the causal mask, keep fp32 running max / sum (the
-//     vLLM-Ascend page, section 3.1, keeps softmax out of fp16), rescale O in
-//     TMEM only when the running max grows by more than 2^8 (exact: O and the
-//     sum always share the same reference max), and write P as bf16/f16 into
-//     shared memory in the operand layout.  A key tile in which some row gets
-//     at least 1/16 of its running mass (always the first tile, and tiles
-//     with dominant keys) issues P as two 16-bit terms (hi + lo), exact to
-//     ~2^-17; other tiles use one term, whose rounding then moves each output
-//     by at most 2^-9 |v| / 16.
-// S is double-buffered so S_{j+1} = Q K_{j+1}^T runs while the softmax warps
-// work on tile j.
+//   * two softmax warpgroups, one per query tile (thread r = row r = TMEM lane
+//     r), read S with tcgen05.ld, apply the causal mask, keep fp32 running max
+//     and sum (the vLLM-Ascend page, section 3.1, keeps softmax out of fp16),
+//     rescale O in TMEM only when the running max grows by more than 2^8
+//     (exact: O and the sum always share one reference max), and write P in
+//     the operand layout into shared memory.  A key tile in which some row of
+//     the tile gets at least 1/16 of its running mass (always the first one,
+//     and tiles with dominant keys) also issues P's low 16-bit term, exact to
+//     ~2^-17; elsewhere one term moves an output by at most 2^-9 |v| / 16.
+// With two query tiles and double-buffered S, the tensor core always has an
+// S or a PV product to run while either warpgroup is in its softmax.
 
 #include <algorithm>
 
@@ -43,34 +47,37 @@ namespace {
 using namespace pa;
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int BM = 128;                 // query rows per CTA (TMEM lanes)
-constexpr int BN = 128;                 // keys per tile
+constexpr int BM = 128;                 // query rows per query tile (TMEM lanes)
+constexpr int BN = 64;                  // keys per key tile
 constexpr int HD = 128;                 // head_dim
-constexpr int kStages = 2;              // K/V ring depth
+constexpr int kStages = 3;              // K and V ring depth (separate rings)
 constexpr float kRescaleLog2 = 8.f;     // rescale O only when the max grows by more than 2^8
-// A key tile whose P carries at least 1/16 of some row's running softmax mass also issues P's low
-// 16-bit term: its one-term rounding error (2^-9 relative) would otherwise reach ~2^-9 |v| of that
-// row's output.  The first tile always qualifies (it holds all the mass so far).
 constexpr float kLoFraction = 1.f / 16.f;
 
-// shared memory map (offsets from a 1024-byte aligned base)
-constexpr int TILE_HALF = BM * 128;                     // 128 rows x 128 bytes = 16 KB (64 columns)
-constexpr int TILE = 2 * TILE_HALF;                     // 128 x 128 16-bit values = 32 KB
-constexpr int Q_OFF = 0;
-constexpr int K_OFF = Q_OFF + TILE;
-constexpr int V_OFF = K_OFF + kStages * TILE;
-constexpr int P_OFF = V_OFF + kStages * TILE;    // P, high 16-bit term
-constexpr int PL_OFF = P_OFF + TILE;             // P, low 16-bit term (tiles that need it)
-constexpr int BAR_OFF = PL_OFF + TILE;
-// barriers: q_full, k_full[2], v_full[2], kv_empty[2], s_full[2], s_free[2], p_full, o_done
-constexpr int NBAR = 1 + 2 * kStages + kStages + 2 + 2 + 2;
-constexpr int TMEM_SLOT_OFF = BAR_OFF + NBAR * 8;
-constexpr int LOFLAG_OFF = TMEM_SLOT_OFF + 4;    // int [2]: tile index + 1 when that tile needs the low term
-constexpr int SMEM_BYTES = LOFLAG_OFF + 8 + 4;
-static_assert(SMEM_BYTES + 1024 <= 232448, "shared memory budget");
+// shared memory map (offsets from a 1024-byte aligned base).  Operand tiles have rows of
+// 128 bytes (64 16-bit values) with the 128-byte swizzle; wider tiles are split into
+// 64-column "halves" placed one after the other.
+constexpr int QHALF = BM * 128;                 // 16 KB: 128 rows x 64 columns
+constexpr int QTILE = 2 * QHALF;                // 32 KB: 128 rows x 128 columns (head_dim)
+constexpr int KVHALF = BN * 128;                // 8 KB: 64 keys x 64 columns
+constexpr int KVTILE = 2 * KVHALF;              // 16 KB: 64 keys x 128 columns
+constexpr int PTILE = BM * 128;                 // 16 KB: 128 rows x 64 keys
+constexpr int Q_OFF = 0;                        // Q[2]
+constexpr int K_OFF = Q_OFF + 2 * QTILE;        // K[kStages]
+constexpr int V_OFF = K_OFF + kStages * KVTILE; // V[kStages]
+constexpr int P_OFF = V_OFF + kStages * KVTILE; // P high term [2 query tiles]
+constexpr int PL_OFF = P_OFF + 2 * PTILE;       // P low term [2 query tiles]
+constexpr int BAR_OFF = PL_OFF + 2 * PTILE;
+// barriers: q_full, k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2][2], s_free[2][2], p_full[2],
+// o_done[2][2]
+constexpr int NBAR = 1 + 4 * kStages + 4 + 4 + 2 + 4;
+constexpr int MISC_OFF = BAR_OFF + NBAR * 8;    // tmem base (4 B), lo flags int[2][2]
+constexpr int SMEM_BYTES = MISC_OFF + 4 + 16 + 12;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
-constexpr int TMEM_COLS = 512;  // S0 [0,128), S1 [128,256), O [256,384)
+// TMEM columns: S_t buffers [t*128 + buf*64, +64), O_t [256 + t*128, +128)
+constexpr int TMEM_COLS = 512;
 constexpr int O_COL = 256;
 
 struct PrefillParams {
@@ -85,6 +92,7 @@ struct PrefillParams {
   int block_size;
   int num_blocks;
   int mtiles;         // ceil(max_chunk_len / BM)
+  int units;          // query-tile pairs per (sequence, KV head)
   float scale_log2;
 };
 
@@ -94,19 +102,20 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo_bytes, uin
   return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
-// K-major operand (rows of 128 bytes, 8-row groups 1024 bytes apart): k-step ks of 16 elements.
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int ks) {
-  return sdesc(tile + (ks >> 2) * TILE_HALF + (ks & 3) * 32, 16, 1024);
+// K-major operand whose 64-column halves are `half` bytes apart (rows 128 bytes, 8-row groups
+// 1024 bytes apart): k-step ks of 16 elements.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int half, int ks) {
+  return sdesc(tile + (ks >> 2) * half + (ks & 3) * 32, 16, 1024);
 }
-// MN-major operand (V: key rows of 128 bytes = 64 head_dim values; the two 64-column halves
-// 16 KB apart): k-step ks covers keys 16*ks .. 16*ks+15.
-__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile, int ks) {
-  return sdesc(tile + ks * 16 * 128, TILE_HALF, 1024);
+// MN-major V tile (key rows of 128 bytes = 64 head_dim values; the two halves KVHALF apart):
+// k-step ks covers keys 16*ks .. 16*ks+15.
+__device__ __forceinline__ uint64_t v_desc(uint32_t tile, int ks) {
+  return sdesc(tile + ks * 16 * 128, KVHALF, 1024);
 }
-// Instruction descriptor, kind::f16: fp32 accumulate, A/B 16-bit (0 = f16, 1 = bf16), M 128, N 128.
-__host__ __device__ constexpr uint32_t idesc(int fmt, bool b_mn_major) {
+// Instruction descriptor, kind::f16: fp32 accumulate, A/B 16-bit (0 = f16, 1 = bf16), M 128.
+__host__ __device__ constexpr uint32_t idesc(int fmt, bool b_mn_major, int n) {
   return (1u << 4) | ((uint32_t)fmt << 7) | ((uint32_t)fmt << 10) | ((b_mn_major ? 1u : 0u) << 16) |
-         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id, uint32_t accumulate) {
@@ -160,15 +169,15 @@ __device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint3
   asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
 }
 
-// Byte offset of (row r, column c) in a 128 x 128 tile stored as two 64-column halves with the
-// 128-byte swizzle (16-byte chunk index XOR row % 8).
-__device__ __forceinline__ uint32_t tile_off(int r, int c) {
-  return (c >> 6) * TILE_HALF + r * 128 + ((((c >> 3) & 7) ^ (r & 7)) << 4) + ((c & 7) << 1);
+// Byte offset of (row r, 16-bit column c) in a tile of 128-byte rows split into 64-column halves
+// `half` bytes apart, with the 128-byte swizzle (16-byte chunk index XOR row % 8).
+__device__ __forceinline__ uint32_t tile_off(int r, int c, int half) {
+  return (c >> 6) * half + r * 128 + ((((c >> 3) & 7) ^ (r & 7)) << 4) + ((c & 7) << 1);
 }
 
 // --------------------------------------------------------------- kernel
 template <int DT>
-__global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__ CUtensorMap qmap,
+__global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__ CUtensorMap qmap,
                                                           const __grid_constant__ CUtensorMap kmap,
                                                           const __grid_constant__ CUtensorMap vmap,
                                                           const PrefillParams p) {
@@ -180,58 +189,70 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
   uint64_t* v_full = k_full + kStages;
-  uint64_t* kv_empty = v_full + kStages;
-  uint64_t* s_full = kv_empty + kStages;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_free + 2;
-  uint64_t* o_done = p_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + TMEM_SLOT_OFF);
-  volatile int* lo_flag = reinterpret_cast<volatile int*>(smem + LOFLAG_OFF);
+  uint64_t* k_empty = v_full + kStages;    // K slot free: both S products of its key tile are done
+  uint64_t* v_empty = k_empty + kStages;   // V slot free: both PV products of its key tile are done
+  uint64_t* s_full = v_empty + kStages;    // [t][buf] at s_full[t * 2 + buf]
+  uint64_t* s_free = s_full + 4;           // [t][buf]
+  uint64_t* p_full = s_free + 4;           // [t]
+  uint64_t* o_done = p_full + 2;           // [t][key tile & 1]: O_t += P_t V of that key tile is complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + MISC_OFF);
+  volatile int* lo_flag = reinterpret_cast<volatile int*>(smem + MISC_OFF + 4);  // [t][j & 1]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.num_q_heads / p.num_kv_heads;
-  // CTA -> (query head, m-tile, sequence); the G heads of a KV group are adjacent so their K/V
-  // tiles are read from L2 by neighbouring CTAs.
+  // CTA -> (pair unit, KV head, sequence).  G >= 2: two heads of the group over the same 128 rows;
+  // G == 1: the group's single head over two consecutive 128-row tiles.
   int u = blockIdx.x;
-  const int j_in_group = u % G;
-  u /= G;
-  const int mt = u % p.mtiles;
-  u /= p.mtiles;
+  const int unit = u % p.units;
+  u /= p.units;
   const int g = u % p.num_kv_heads;
   const int b = u / p.num_kv_heads;
-  const int h = g * G + j_in_group;
+  int head[2], mrow[2];
+  if (G >= 2) {
+    const int pair = unit % (G / 2), mt = unit / (G / 2);
+    head[0] = g * G + 2 * pair;
+    head[1] = head[0] + 1;
+    mrow[0] = mrow[1] = mt * BM;
+  } else {
+    head[0] = head[1] = g;
+    mrow[0] = unit * 2 * BM;
+    mrow[1] = mrow[0] + BM;
+  }
 
   const int q0 = __ldg(p.query_start_loc + b), q1 = __ldg(p.query_start_loc + b + 1);
   const int C = q1 - q0;
-  const int m0 = mt * BM;
-  if (m0 >= C) return;
-  int L = __ldg(p.context_lens + b);
+  if (mrow[0] >= C) return;
+  const int L = __ldg(p.context_lens + b);
   const int cap = p.max_blocks_per_seq * p.block_size;
   if (L > cap || L < C) {  // broken caller invariant: record and produce nothing for this tile
     if (threadIdx.x == 0) PA_RECORD_ERROR(PA_ERRBIT_INDEX);
     return;
   }
-  const int pos0 = L - C + m0;                              // position of this tile's first query row
-  const int kend = min(L, pos0 + BM);                       // keys [0, kend) are visible to some row
+  // keys [0, kend) are visible to some row of either tile
+  const int kend = min(L, L - C + max(mrow[0], mrow[1]) + BM);
   const int nkv = (kend + BN - 1) / BN;
 
   if (threadIdx.x == 0) {
-    lo_flag[0] = lo_flag[1] = 0;
+    lo_flag[0] = lo_flag[1] = lo_flag[2] = lo_flag[3] = 0;
     mbar_init(q_full, 1);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], BM);
     }
-    mbar_init(p_full, BM);
-    mbar_init(o_done, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&p_full[t], BM);
+      mbar_init(&o_done[t * 2], 1);
+      mbar_init(&o_done[t * 2 + 1], 1);
+    }
     fence_mbar_init();
   }
-  if (warp == 5) {  // TMEM: S0, S1, O
+  if (warp == 9) {  // TMEM: S_0 x2, S_1 x2, O_0, O_1
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(TMEM_COLS)
                  : "memory");
@@ -243,51 +264,78 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
 
-  if (warp == 4) {
-    // ============================================ producer: Q once, then K/V tiles through the block table
+  if (warp == 8) {
+    // ============================================ producer: both Q tiles once, then K/V tiles
     if (lane == 0) {
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
-      mbar_arrive_expect_tx(q_full, TILE);
-      for (int hf = 0; hf < 2; ++hf)
-        tma_load_2d(smem + Q_OFF + hf * TILE_HALF, &qmap, h * HD + hf * 64, q0 + m0, q_full);
+      mbar_arrive_expect_tx(q_full, 2 * QTILE);
+      for (int t = 0; t < 2; ++t)
+        for (int hf = 0; hf < 2; ++hf)
+          tma_load_2d(smem + Q_OFF + t * QTILE + hf * QHALF, &qmap, head[t] * HD + hf * 64, q0 + mrow[t], q_full);
     }
     const int32_t* bt = p.block_tables + (size_t)b * p.max_blocks_per_seq;
     auto lookup = [&](int j) -> int {
       const int key = j * BN + lane * 16;
-      return (j < nkv && lane < 8 && key < kend) ? __ldg(bt + key / p.block_size) : 0;
+      return (j < nkv && lane < BN / 16 && key < kend) ? __ldg(bt + key / p.block_size) : 0;
     };
-    int phys = lookup(0);
-    for (int j = 0; j < nkv && ok; ++j) {
+    // K and V tiles are issued as their own slots free up: K slots early (after the S products),
+    // V slots late (after the PV products), so K runs ahead of V.
+    int jk = 0, jv = 0;
+    int physk = lookup(0), physv = physk;
+    auto issue = [&](int j, int phys, uint64_t* full, const CUtensorMap* map, int off) {
       const int st = j % kStages;
-      if (j >= kStages && !mbar_wait(&kv_empty[st], ((j / kStages) - 1) & 1)) {
-        ok = false;
-        break;
-      }
-      const int nbox = min(8, (kend - j * BN + 15) / 16);
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&k_full[st], nbox * 16 * HD * 2);
-        mbar_arrive_expect_tx(&v_full[st], nbox * 16 * HD * 2);
-      }
+      const int nbox = min(BN / 16, (kend - j * BN + 15) / 16);
+      if (lane == 0) mbar_arrive_expect_tx(&full[st], nbox * 16 * HD * 2);
       __syncwarp();
       if (lane < nbox) {
         if (phys < 0 || phys >= p.num_blocks) PA_RECORD_ERROR(PA_ERRBIT_INDEX);  // TMA zero-fills out of range
         const int key = j * BN + lane * 16;
         const int y = phys * p.block_size + key % p.block_size;
-        for (int hf = 0; hf < 2; ++hf) {
-          tma_load_2d(smem + K_OFF + st * TILE + hf * TILE_HALF + lane * 16 * 128, &kmap, g * HD + hf * 64, y,
-                      &k_full[st]);
-          tma_load_2d(smem + V_OFF + st * TILE + hf * TILE_HALF + lane * 16 * 128, &vmap, g * HD + hf * 64, y,
-                      &v_full[st]);
+        for (int hf = 0; hf < 2; ++hf)
+          tma_load_2d(smem + off + st * KVTILE + hf * KVHALF + lane * 16 * 128, map, g * HD + hf * 64, y, &full[st]);
+      }
+    };
+    // lane 0 polls both rings and broadcasts, so the warp never splits on a wait; the time spent with
+    // neither ring ready is bounded like every other wait
+    uint64_t idle_since = 0;
+    while (jk < nkv || jv < nkv) {
+      int go = 0;  // 1: issue K, 2: issue V
+      if (lane == 0) {
+        if (jk < nkv && (jk < kStages || mbar_try_wait(&k_empty[jk % kStages], ((jk / kStages) - 1) & 1)))
+          go = 1;
+        else if (jv < jk && (jv < kStages || mbar_try_wait(&v_empty[jv % kStages], ((jv / kStages) - 1) & 1)))
+          go = 2;
+      }
+      go = __shfl_sync(0xffffffffu, go, 0);
+      if (go == 1) {
+        issue(jk, physk, k_full, &kmap, K_OFF);
+        ++jk;
+        physk = lookup(jk);
+        idle_since = 0;
+      } else if (go == 2) {
+        issue(jv, physv, v_full, &vmap, V_OFF);
+        ++jv;
+        physv = lookup(jv);
+        idle_since = 0;
+      } else {
+        int late = 0;
+        if (lane == 0) {
+          const uint64_t now = global_ns();
+          if (idle_since == 0) idle_since = now;
+          late = now - idle_since > PA_WAIT_LIMIT_NS;
+        }
+        if (__shfl_sync(0xffffffffu, late, 0)) {
+          ok = false;
+          break;
         }
       }
-      phys = lookup(j + 1);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ============================================ MMA issuer (one thread issues; the warp zeroes V tails)
-    const uint32_t id_s = idesc(DT == PA_BF16 ? 1 : 0, false);
-    const uint32_t id_pv = idesc(DT == PA_BF16 ? 1 : 0, true);
+    const uint32_t id_s = idesc(DT == PA_BF16 ? 1 : 0, false, BN);
+    const uint32_t id_pv = idesc(DT == PA_BF16 ? 1 : 0, true, HD);
     auto issue_pv = [&](int i) -> bool {
       const int st = i % kStages;
       if (!mbar_wait(&v_full[st], (i / kStages) & 1)) return false;
@@ -295,95 +343,119 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
       if (valid < BN) {  // keys past the end: zero their V rows (their bytes may be anything, even NaN)
         for (int idx = lane; idx < (BN - valid) * 16; idx += 32) {
           const int r = valid + idx / 16, c = (idx % 16) * 8;
-          sts128(sb + V_OFF + st * TILE + tile_off(r, c), 0, 0, 0, 0);
+          sts128(sb + V_OFF + st * KVTILE + tile_off(r, c, KVHALF), 0, 0, 0, 0);
         }
         fence_proxy_async_smem();
         __syncwarp();
       }
-      if (!mbar_wait(p_full, i & 1)) return false;
-      tc_fence_after();
-      const bool lo = lo_flag[i & 1] == i + 1;
-      if (lane == 0) {
-        for (int ks = 0; ks < BN / 16; ++ks)
-          mma_f16(tmem + O_COL, kmajor_desc(sb + P_OFF, ks), mnmajor_desc(sb + V_OFF + st * TILE, ks), id_pv,
-                  (i > 0 || ks > 0) ? 1u : 0u);
-        if (lo)
+      for (int t = 0; t < 2; ++t) {
+        if (!mbar_wait(&p_full[t], i & 1)) return false;
+        tc_fence_after();
+        const bool lo = lo_flag[t * 2 + (i & 1)] == i + 1;
+        if (lane == 0) {
+          const uint32_t od = tmem + O_COL + t * HD;
           for (int ks = 0; ks < BN / 16; ++ks)
-            mma_f16(tmem + O_COL, kmajor_desc(sb + PL_OFF, ks), mnmajor_desc(sb + V_OFF + st * TILE, ks), id_pv, 1u);
-        mma_commit(o_done);
-        mma_commit(&kv_empty[st]);
+            mma_f16(od, kmajor_desc(sb + P_OFF + t * PTILE, 0, ks), v_desc(sb + V_OFF + st * KVTILE, ks), id_pv,
+                    (i > 0 || ks > 0) ? 1u : 0u);
+          if (lo)
+            for (int ks = 0; ks < BN / 16; ++ks)
+              mma_f16(od, kmajor_desc(sb + PL_OFF + t * PTILE, 0, ks), v_desc(sb + V_OFF + st * KVTILE, ks), id_pv,
+                      1u);
+          mma_commit(&o_done[t * 2 + (i & 1)]);
+          if (t == 1) mma_commit(&v_empty[st]);
+        }
+        __syncwarp();
       }
-      __syncwarp();
       return true;
     };
     if (!mbar_wait(q_full, 0)) ok = false;
     for (int j = 0; j < nkv && ok; ++j) {
-      const int st = j % kStages, s2 = j & 1;
-      if (!mbar_wait(&k_full[st], (j / kStages) & 1) || (j >= 2 && !mbar_wait(&s_free[s2], ((j >> 1) - 1) & 1))) {
+      const int st = j % kStages, buf = j & 1;
+      if (!mbar_wait(&k_full[st], (j / kStages) & 1)) {
         ok = false;
         break;
       }
-      tc_fence_after();
-      if (lane == 0) {
-        for (int ks = 0; ks < HD / 16; ++ks)
-          mma_f16(tmem + s2 * BN, kmajor_desc(sb + Q_OFF, ks), kmajor_desc(sb + K_OFF + st * TILE, ks), id_s,
-                  ks > 0 ? 1u : 0u);
-        mma_commit(&s_full[s2]);
+      for (int t = 0; t < 2; ++t) {
+        if (j >= 2 && !mbar_wait(&s_free[t * 2 + buf], ((j >> 1) - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          for (int ks = 0; ks < HD / 16; ++ks)
+            mma_f16(tmem + t * 128 + buf * BN, kmajor_desc(sb + Q_OFF + t * QTILE, QHALF, ks),
+                    kmajor_desc(sb + K_OFF + st * KVTILE, KVHALF, ks), id_s, ks > 0 ? 1u : 0u);
+          mma_commit(&s_full[t * 2 + buf]);
+          if (t == 1) mma_commit(&k_empty[st]);
+        }
+        __syncwarp();
       }
-      __syncwarp();
+      if (!ok) break;
       if (j >= 1 && !issue_pv(j - 1)) ok = false;
     }
     if (ok && !issue_pv(nkv - 1)) ok = false;
   } else {
-    // ============================================ softmax warps: thread r owns query row m0 + r
-    const int r = threadIdx.x;
-    const int pos = pos0 + r;                                 // this row's position (keys 0..pos visible)
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lane quarter
-    float m_ref = -INFINITY;                                  // reference max (log2 units) shared by O and l
+    // ============================================ softmax warpgroups: warpgroup t, thread r owns row mrow[t] + r
+    const int t = warp >> 2;
+    const int r = threadIdx.x & 127;
+    const int pos = L - C + mrow[t] + r;                      // this row's position (keys 0..pos visible)
+    const int last_key = min(pos, L - 1);
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;  // this warp's TMEM lane quarter
+    const uint32_t p_lo = sb + PL_OFF + t * PTILE;
+    float m_ref = -INFINITY;  // reference max (log2 units) shared by O and l
     float l = 0.f;
     float s[BN];
     for (int j = 0; j < nkv && ok; ++j) {
-      const int s2 = j & 1;
-      if (!mbar_wait(&s_full[s2], (j >> 1) & 1)) {
+      const int buf = j & 1;
+      if (!mbar_wait(&s_full[t * 2 + buf], (j >> 1) & 1)) {
         ok = false;
         break;
       }
       tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < BN; c += 32) tmem_ld32(tmem + lane_base + s2 * BN + c, s + c);
+      tmem_ld32(tmem + lane_base + t * 128 + buf * BN, s);
+      tmem_ld32(tmem + lane_base + t * 128 + buf * BN + 32, s + 32);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(&s_free[s2]);
-      // causal mask: key k visible iff k <= pos (and k < L)
-      const int k0 = j * BN;
-      const int lim = min(pos, L - 1) - k0;  // last visible column of this tile
-      float mx = -INFINITY;
+      mbar_arrive(&s_free[t * 2 + buf]);
+      const int lim = last_key - j * BN;  // last visible column of this key tile
+      if (lim < BN - 1) {
 #pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        s[c] = c <= lim ? s[c] * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < BN; ++c) s[c] = c <= lim ? s[c] : -INFINITY;
       }
+      // eight independent partial maxima: short dependency chains
+      float pm[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) pm[e] = s[e];
+#pragma unroll
+      for (int c = 8; c < BN; ++c) pm[c & 7] = fmaxf(pm[c & 7], s[c]);
+      float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      mx *= p.scale_log2;
       float alpha = 1.f;
       bool rescale = false;
-      if (mx > m_ref + kRescaleLog2 || m_ref == -INFINITY) {
+      if (mx > m_ref + kRescaleLog2 || (m_ref == -INFINITY && mx != -INFINITY)) {
         alpha = m_ref == -INFINITY ? 0.f : fast_exp2(m_ref - mx);
         rescale = m_ref != -INFINITY;
         m_ref = mx;
       }
-      float rs = 0.f;
+      const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
+      float ps[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ps[e] = 0.f;
 #pragma unroll
       for (int c = 0; c < BN; ++c) {
-        s[c] = fast_exp2(s[c] - m_ref);
-        rs += s[c];
+        s[c] = fast_exp2(fmaf(s[c], p.scale_log2, neg_m));
+        ps[c & 7] += s[c];
       }
+      const float rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       l = l * alpha + rs;
-      // does this tile carry a large share of some row's mass?  (CTA-wide decision: tile j needs
-      // the low term iff lo_flag[j&1] == j+1 after the softmax warps have all voted)
-      if (__any_sync(0xffffffffu, rs >= kLoFraction * l) && lane == 0) lo_flag[j & 1] = j + 1;
-      named_barrier_sync(1, BM);
-      const bool lo = lo_flag[j & 1] == j + 1;
-      // the previous tile's PV must be done (P buffers free, O complete) before we touch either
-      if (j > 0 && !mbar_wait(o_done, (j - 1) & 1)) {
+      // does this key tile carry a large share of some row's mass?  (decided per query tile:
+      // tile j needs the low term iff lo_flag[t][j&1] == j+1 once the warpgroup has voted)
+      if (__any_sync(0xffffffffu, rs >= kLoFraction * l) && lane == 0) lo_flag[t * 2 + (j & 1)] = j + 1;
+      named_barrier_sync(1 + t, BM);
+      const bool lo = lo_flag[t * 2 + (j & 1)] == j + 1;
+      const uint32_t p_hi = sb + P_OFF + t * PTILE;
+      // the P buffers and O are touched only after the PV of key tile j-1 is complete
+      if (j >= 1 && !mbar_wait(&o_done[t * 2 + ((j - 1) & 1)], ((j - 1) >> 1) & 1)) {
         ok = false;
         break;
       }
@@ -392,41 +464,44 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
 #pragma unroll
         for (int c = 0; c < HD; c += 32) {
           float o[32];
-          tmem_ld32(tmem + lane_base + O_COL + c, o);
+          tmem_ld32(tmem + lane_base + O_COL + t * HD + c, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] *= alpha;
-          tmem_st32(tmem + lane_base + O_COL + c, o);
+          tmem_st32(tmem + lane_base + O_COL + t * HD + c, o);
         }
         tmem_wait_st();
       }
 #pragma unroll
       for (int c = 0; c < BN; c += 8) {
-        uint32_t w[4], wl[4];
+        uint32_t w[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = s[c + 2 * e], bb = s[c + 2 * e + 1];
-          w[e] = Elt<DT>::from_f2(a, bb);
-          const float2 hv = Elt<DT>::to_f2(w[e]);
-          wl[e] = Elt<DT>::from_f2(a - hv.x, bb - hv.y);
+        for (int e = 0; e < 4; ++e) w[e] = Elt<DT>::from_f2(s[c + 2 * e], s[c + 2 * e + 1]);
+        sts128(p_hi + tile_off(r, c, 0), w[0], w[1], w[2], w[3]);
+        if (lo) {
+          uint32_t wl[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 hv = Elt<DT>::to_f2(w[e]);
+            wl[e] = Elt<DT>::from_f2(s[c + 2 * e] - hv.x, s[c + 2 * e + 1] - hv.y);
+          }
+          sts128(p_lo + tile_off(r, c, 0), wl[0], wl[1], wl[2], wl[3]);
         }
-        sts128(sb + P_OFF + tile_off(r, c), w[0], w[1], w[2], w[3]);
-        if (lo) sts128(sb + PL_OFF + tile_off(r, c), wl[0], wl[1], wl[2], wl[3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[t]);
     }
     // epilogue: O / l -> out
-    if (ok && mbar_wait(o_done, (nkv - 1) & 1)) {
+    if (ok && mbar_wait(&o_done[t * 2 + ((nkv - 1) & 1)], ((nkv - 1) >> 1) & 1)) {
       tc_fence_after();
-      const int row = m0 + r;
-      T* orow = reinterpret_cast<T*>(p.out) + ((size_t)(q0 + row) * p.num_q_heads + h) * HD;
+      const int row = mrow[t] + r;
+      T* orow = reinterpret_cast<T*>(p.out) + ((size_t)(q0 + row) * p.num_q_heads + head[t]) * HD;
       const float inv = 1.f / l;
 #pragma unroll
       for (int c = 0; c < HD; c += 32) {
         float o[32];
-        tmem_ld32(tmem + lane_base + O_COL + c, o);
+        tmem_ld32(tmem + lane_base + O_COL + t * HD + c, o);
         tmem_wait_ld();
         if (row < C) {
 #pragma unroll
@@ -448,13 +523,8 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5)
+  if (warp == 9)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
-}
-
-int encode_q_map(CUtensorMap* map, const void* q, int total_q, int Hq) {
-  return pa::encode_2d_sw128(map, q, (uint64_t)Hq * HD, (uint64_t)std::max(total_q, 1), (uint64_t)Hq * HD * 2, 64,
-                             BM);
 }
 
 }  // namespace
@@ -469,7 +539,8 @@ extern "C" int pa_prefill_chunk(const void* q, const int32_t* query_start_loc, i
     return PA_ERR_INVALID;
   if (!pa::valid_dtype(dtype) || head_dim != HD || !pa::valid_block_size(block_size)) return PA_ERR_UNSUPPORTED;
   if (num_q_heads % num_kv_heads) return PA_ERR_INVALID;
-  if (!pa::valid_group(num_q_heads / num_kv_heads)) return PA_ERR_UNSUPPORTED;
+  const int G = num_q_heads / num_kv_heads;
+  if (!pa::valid_group(G)) return PA_ERR_UNSUPPORTED;
   if (batch == 0 || total_q_tokens == 0 || max_chunk_len == 0) return PA_OK;
   if (!q || !query_start_loc || !k_cache || !v_cache || !block_tables || !context_lens || !out) return PA_ERR_INVALID;
   if (!pa::aligned16(q) || !pa::aligned16(k_cache) || !pa::aligned16(v_cache) || !pa::aligned16(out) ||
@@ -479,7 +550,8 @@ extern "C" int pa_prefill_chunk(const void* q, const int32_t* query_start_loc, i
   if (num_blocks == 0) return PA_ERR_INVALID;
   if ((long)num_blocks * block_size >= (1L << 31)) return PA_ERR_UNSUPPORTED;
   const int mtiles = (max_chunk_len + BM - 1) / BM;
-  const long grid = (long)batch * num_kv_heads * mtiles * (num_q_heads / num_kv_heads);
+  const int units = G >= 2 ? (G / 2) * mtiles : (mtiles + 1) / 2;
+  const long grid = (long)batch * num_kv_heads * units;
   if (grid > 0x7fffffffL) return PA_ERR_UNSUPPORTED;
 
   PrefillParams p;
@@ -494,12 +566,15 @@ extern "C" int pa_prefill_chunk(const void* q, const int32_t* query_start_loc, i
   p.block_size = block_size;
   p.num_blocks = num_blocks;
   p.mtiles = mtiles;
+  p.units = units;
   p.scale_log2 = scale * kLog2e;
 
   CUtensorMap qm, km, vm;
   const uint64_t rows = (uint64_t)num_blocks * block_size;
   const uint64_t cols = (uint64_t)num_kv_heads * HD;
-  if (encode_q_map(&qm, q, total_q_tokens, num_q_heads) != PA_OK) return PA_ERR_CUDA;
+  if (pa::encode_2d_sw128(&qm, q, (uint64_t)num_q_heads * HD, (uint64_t)total_q_tokens, (uint64_t)num_q_heads * HD * 2,
+                          64, BM) != PA_OK)
+    return PA_ERR_CUDA;
   if (pa::encode_2d_sw128(&km, k_cache, cols, rows, cols * 2, 64, 16) != PA_OK) return PA_ERR_CUDA;
   if (pa::encode_2d_sw128(&vm, v_cache, cols, rows, cols * 2, 64, 16) != PA_OK) return PA_ERR_CUDA;
 
@@ -513,6 +588,6 @@ extern "C" int pa_prefill_chunk(const void* q, const int32_t* query_start_loc, i
       return PA_ERR_CUDA;
     if (dev >= 0 && dev < 64) attr_set[di][dev] = true;
   }
-  kern<<<(unsigned)grid, 192, SMEM_ALLOC, (cudaStream_t)stream>>>(qm, km, vm, p);
+  kern<<<(unsigned)grid, 320, SMEM_ALLOC, (cudaStream_t)stream>>>(qm, km, vm, p);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
