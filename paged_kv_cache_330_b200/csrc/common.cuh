@@ -100,6 +100,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (global_ns() - start > PA_WAIT_LIMIT_NS) return false;
   }
 }
+// The bounded wait taken by every lane of a warp, which then agrees on the outcome: a timeout
+// seen by one lane cannot split the warp.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity)) != 0;
+}
 
 // ---------------------------------------------------------------- TMA
 // 2-D tiled bulk tensor load global -> shared, completion counted in bytes on

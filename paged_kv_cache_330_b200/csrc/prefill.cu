@@ -9,31 +9,36 @@
 //   out[i][h] = sum_{t <= p} softmax_t(scale <q[i][h], K_b[t][h/G]>) V_b[t][h/G].
 //
 // This is the one dense contraction on the path, so it runs on the
-// 5th-generation tensor cores.  One CTA owns two 128-row query tiles that read
-// the same keys: two query heads of one KV group over the same rows (or, when
-// a group has one head, two consecutive row tiles of it).  Keys are walked in
-// tiles of 64:
-//   * a TMA producer warp loads both query tiles once and, per key tile, 16-row
-//     K and V boxes gathered through the block table (128-byte swizzle, no
-//     multicast) into separate three-stage K and V rings shared by both query
-//     tiles (a K slot frees after the S products, a V slot after the PVs, so
-//     K runs ahead);
-//   * one thread of the MMA warp issues, per key tile, S_t = Q_t K^T for both
-//     query tiles (M 128, N 64, K 128) into per-tile double-buffered TMEM, then
-//     O_t += P_t V for the previous key tile (M 128, N 128, K 64), with fp32
-//     accumulation (tcgen05.mma kind::f16) and completions signalled with
-//     tcgen05.commit on mbarriers;
-//   * two softmax warpgroups, one per query tile (thread r = row r = TMEM lane
-//     r), read S with tcgen05.ld, apply the causal mask, keep fp32 running max
-//     and sum (the vLLM-Ascend page, section 3.1, keeps softmax out of fp16),
-//     rescale O in TMEM only when the running max grows by more than 2^8
-//     (exact: O and the sum always share one reference max), and write P in
-//     the operand layout into shared memory.  A key tile in which some row of
-//     the tile gets at least 1/16 of its running mass (always the first one,
-//     and tiles with dominant keys) also issues P's low 16-bit term, exact to
-//     ~2^-17; elsewhere one term moves an output by at most 2^-9 |v| / 16.
-// With two query tiles and double-buffered S, the tensor core always has an
-// S or a PV product to run while either warpgroup is in its softmax.
+// 5th-generation tensor cores, as CTA pairs (a cluster of two CTAs on one
+// TPC).  Each CTA owns 128 query rows: two heads of one KV group over the same
+// rows, or, when a group has one head, two consecutive row tiles of it.  The
+// pair walks the keys in tiles of 128 and the even CTA issues every product for
+// both (tcgen05.mma cta_group::2, M = 256):
+//   * S = Q K^T (N 128, K 128): A = the CTA's query tile in its own TMEM
+//     (64 columns of packed 16-bit pairs), B = K split by key: each CTA holds
+//     64 of the tile's 128 keys;
+//   * O += P V (N 128, K 128): A = P, written by the softmax over its own S
+//     buffer in TMEM, B = V split by head_dim: each CTA holds 64 columns.
+// So each CTA streams half of every K and V tile from L2 (the bound of the
+// one-CTA form) and the paired product runs at ~0.8 of the tensor peak where a
+// one-CTA 128 x 128 x 16 product with A in TMEM stops near 0.6.
+// A TMA producer warp per CTA gathers its 16-row K and V boxes through the
+// block table (128-byte swizzle, no multicast) into four-stage K and V rings;
+// the copies of both CTAs complete on the even CTA's barriers (TMA
+// .cta_group::2), slots are released by a multicast tcgen05.commit, and the
+// last, partial V tile is loaded against a local barrier and zero-filled past
+// the end before it is signalled.  The MMA thread issues S(j) and then
+// O += P(j-1) V, so the tensor core runs PV(j-1) and S(j+1) while the softmax
+// works on S(j).  In each CTA two softmax warpgroups split every key tile in
+// halves (keys 0-63 and 64-127; thread r = row r = TMEM lane r): they swap
+// their half-tile maxima through shared memory, keep fp32 running sums per
+// half (added at the end), rescale O in TMEM only when the running max grows
+// by more than 2^8 (exact: O and the sums always share one reference max), and
+// write P as a high and a low 16-bit term.  The low term's product is issued
+// for a half-tile only when some row of either CTA puts at least 1/16 of that
+// half's running mass there (always the first tile, and tiles with dominant
+// keys): exact to ~2^-17 there; elsewhere the high term alone moves an output
+// by at most 2^-9 |v| / 16.
 
 #include <algorithm>
 
@@ -47,40 +52,42 @@ namespace {
 using namespace pa;
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int BM = 128;                 // query rows per query tile (TMEM lanes)
-constexpr int BN = 64;                  // keys per key tile
+constexpr int BM = 128;                 // query rows per CTA (TMEM lanes); the pair covers 256
+constexpr int BN = 128;                 // keys per key tile
 constexpr int HD = 128;                 // head_dim
-constexpr int kStages = 3;              // K and V ring depth (separate rings)
+constexpr int KS = 4;                   // K ring depth
+constexpr int VS = 4;                   // V ring depth
 constexpr float kRescaleLog2 = 8.f;     // rescale O only when the max grows by more than 2^8
 constexpr float kLoFraction = 1.f / 16.f;
 
-// shared memory map (offsets from a 1024-byte aligned base).  Operand tiles have rows of
-// 128 bytes (64 16-bit values) with the 128-byte swizzle; wider tiles are split into
-// 64-column "halves" placed one after the other.
-constexpr int QHALF = BM * 128;                 // 16 KB: 128 rows x 64 columns
-constexpr int QTILE = 2 * QHALF;                // 32 KB: 128 rows x 128 columns (head_dim)
-constexpr int KVHALF = BN * 128;                // 8 KB: 64 keys x 64 columns
-constexpr int KVTILE = 2 * KVHALF;              // 16 KB: 64 keys x 128 columns
-constexpr int PTILE = BM * 128;                 // 16 KB: 128 rows x 64 keys
-constexpr int Q_OFF = 0;                        // Q[2]
-constexpr int K_OFF = Q_OFF + 2 * QTILE;        // K[kStages]
-constexpr int V_OFF = K_OFF + kStages * KVTILE; // V[kStages]
-constexpr int P_OFF = V_OFF + kStages * KVTILE; // P high term [2 query tiles]
-constexpr int PL_OFF = P_OFF + 2 * PTILE;       // P low term [2 query tiles]
-constexpr int BAR_OFF = PL_OFF + 2 * PTILE;
-// barriers: q_full, k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2][2], s_free[2][2], p_full[2],
-// o_done[2][2]
-constexpr int NBAR = 1 + 4 * kStages + 4 + 4 + 2 + 4;
-constexpr int MISC_OFF = BAR_OFF + NBAR * 8;    // tmem base (4 B), lo flags int[2][2]
-constexpr int SMEM_BYTES = MISC_OFF + 4 + 16 + 12;
+// shared memory map (offsets from a 1024-byte aligned base).  Tiles have rows of 128 bytes
+// (64 16-bit values) with the 128-byte swizzle.
+constexpr int KHALF = (BN / 2) * 128;           // 8 KB: this CTA's 64 keys x 64 head_dim columns
+constexpr int KTILE = 2 * KHALF;                // 16 KB: this CTA's 64 keys x 128 columns
+constexpr int VTILE = BN * 128;                 // 16 KB: 128 keys x this CTA's 64 columns
+constexpr int K_OFF = 0;                        // K[KS]
+constexpr int V_OFF = K_OFF + KS * KTILE;       // V[VS]
+constexpr int XCH_OFF = V_OFF + VS * VTILE;     // float m_part[2][2][128], l_part[2][128]
+constexpr int BAR_OFF = XCH_OFF + 6 * BM * 4;
+// barriers: q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], v_tail, s_full[2], p_full[2],
+// o_done[2], drain.  The full barriers, q_full, p_full and drain are used in the even CTA only.
+constexpr int NBAR = 1 + 2 * KS + 2 * VS + 1 + 2 + 2 + 2 + 1;
+constexpr int MISC_OFF = BAR_OFF + NBAR * 8;    // tmem base (4 B), lo flags int[2 ranks][2][2 halves]
+constexpr int SMEM_BYTES = MISC_OFF + 4 + 32 + 28;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
-// TMEM columns: S_t buffers [t*128 + buf*64, +64), O_t [256 + t*128, +128)
+// TMEM columns (both CTAs): Q [0, 64) (packed pairs), S buffers [128, 256) and [256, 384),
+// O [384, 512).  Within an S buffer, P of key half h sits at h*64 (high term, 32 columns) and
+// h*64 + 32 (low term), inside the columns that half's own S values occupied.
 constexpr int TMEM_COLS = 512;
-constexpr int O_COL = 256;
+constexpr int Q_COL = 0;
+constexpr int S_COL = 128;
+constexpr int O_COL = 384;
+constexpr int kSoftmaxWarps = 8;        // per CTA; q_full and p_full count one arrival per warp of the pair
 
 struct PrefillParams {
+  const void* q;
   void* out;
   const int32_t* query_start_loc;
   const int32_t* block_tables;
@@ -92,49 +99,98 @@ struct PrefillParams {
   int block_size;
   int num_blocks;
   int mtiles;         // ceil(max_chunk_len / BM)
-  int units;          // query-tile pairs per (sequence, KV head)
+  int units;          // CTA pairs per (sequence, KV head)
   float scale_log2;
 };
 
-// --------------------------------------------------------------- tcgen05 helpers
+// --------------------------------------------------------------- cluster / tcgen05 helpers
+__device__ __forceinline__ uint32_t cta_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// The address of this CTA's shared variable `local` in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_rank(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+// All threads of both CTAs.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive on a barrier of the other CTA.  The release form publishes this thread's earlier
+// shared-memory writes to the pair and costs ~1-2 us, so it is kept for the few arrivals that
+// follow generic writes; the relaxed form serves arrivals whose data is already ordered (TMA bytes
+// counted by the barrier itself, TMEM stores completed by tcgen05.wait::st).
+__device__ __forceinline__ void arrive_cluster_release(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void arrive_cluster_relaxed(uint32_t bar) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void st_cluster(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+// 2-D tiled load into this CTA's shared memory whose completion is counted on a barrier of
+// either CTA of the pair (`bar` is a shared::cluster address).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(dst),
+      "l"(map), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), version 1.
 __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
   return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
-// K-major operand whose 64-column halves are `half` bytes apart (rows 128 bytes, 8-row groups
-// 1024 bytes apart): k-step ks of 16 elements.
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int half, int ks) {
-  return sdesc(tile + (ks >> 2) * half + (ks & 3) * 32, 16, 1024);
+// This CTA's K half-tile as the K-major B operand of S (64 key rows of 128 bytes per head_dim
+// half, the halves KHALF apart, 8-row groups 1024 bytes apart): k-step ks of 16 head_dim values.
+__device__ __forceinline__ uint64_t k_desc(uint32_t tile, int ks) {
+  return sdesc(tile + (ks >> 2) * KHALF + (ks & 3) * 32, 16, 1024);
 }
-// MN-major V tile (key rows of 128 bytes = 64 head_dim values; the two halves KVHALF apart):
-// k-step ks covers keys 16*ks .. 16*ks+15.
+// This CTA's V tile as the MN-major B operand of PV (128 key rows of 128 bytes = its 64
+// head_dim columns): k-step ks covers keys 16*ks .. 16*ks+15.
 __device__ __forceinline__ uint64_t v_desc(uint32_t tile, int ks) {
-  return sdesc(tile + ks * 16 * 128, KVHALF, 1024);
+  return sdesc(tile + ks * 16 * 128, VTILE, 1024);
 }
-// Instruction descriptor, kind::f16: fp32 accumulate, A/B 16-bit (0 = f16, 1 = bf16), M 128.
+// Instruction descriptor, kind::f16: fp32 accumulate, A/B 16-bit (0 = f16, 1 = bf16), A K-major,
+// M 256 (the pair).
 __host__ __device__ constexpr uint32_t idesc(int fmt, bool b_mn_major, int n) {
   return (1u << 4) | ((uint32_t)fmt << 7) | ((uint32_t)fmt << 10) | ((b_mn_major ? 1u : 0u) << 16) |
-         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)((2 * BM) >> 4) << 24);
 }
-
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id, uint32_t accumulate) {
+// D (TMEM of both CTAs) [+]= A (TMEM of both CTAs, 128 lanes x 16 elements each as 8 columns of
+// packed pairs) * B (shared memory of both CTAs, split along N).
+__device__ __forceinline__ void mma_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t id,
+                                         uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(id), "r"(accumulate), "r"(0u)
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(id), "r"(accumulate)
       : "memory");
 }
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+// Arrive once on the barrier at this offset in both CTAs when every product issued so far is done.
+__device__ __forceinline__ void commit_both(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"((uint16_t)3)
+      : "memory");
+}
+// ... on this CTA's barrier only.
+__device__ __forceinline__ void commit_local(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-  uint32_t r[32];
+// 32 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
       "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
@@ -143,293 +199,369 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
         "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
         "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
       "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
-      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
-      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
-      "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
-      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
-      "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
-      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
-      "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
-      "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
-      "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
-  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
-}
-
-// Byte offset of (row r, 16-bit column c) in a tile of 128-byte rows split into 64-column halves
-// `half` bytes apart, with the 128-byte swizzle (16-byte chunk index XOR row % 8).
-__device__ __forceinline__ uint32_t tile_off(int r, int c, int half) {
-  return (c >> 6) * half + r * 128 + ((((c >> 3) & 7) ^ (r & 7)) << 4) + ((c & 7) << 1);
-}
-
 // --------------------------------------------------------------- kernel
 template <int DT>
-__global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__ CUtensorMap qmap,
-                                                          const __grid_constant__ CUtensorMap kmap,
-                                                          const __grid_constant__ CUtensorMap vmap,
-                                                          const PrefillParams p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                   const PrefillParams p) {
   using T = typename Elt<DT>::T;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
-  uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
-  uint64_t* v_full = k_full + kStages;
-  uint64_t* k_empty = v_full + kStages;    // K slot free: both S products of its key tile are done
-  uint64_t* v_empty = k_empty + kStages;   // V slot free: both PV products of its key tile are done
-  uint64_t* s_full = v_empty + kStages;    // [t][buf] at s_full[t * 2 + buf]
-  uint64_t* s_free = s_full + 4;           // [t][buf]
-  uint64_t* p_full = s_free + 4;           // [t]
-  uint64_t* o_done = p_full + 2;           // [t][key tile & 1]: O_t += P_t V of that key tile is complete
+  uint64_t* q_full = bars;                 // [even CTA] queries in TMEM, one arrival per softmax warp
+  uint64_t* k_full = bars + 1;             // [even CTA] both K halves landed
+  uint64_t* k_empty = k_full + KS;         // K slot free: S of its key tile is done
+  uint64_t* v_full = k_empty + KS;         // [even CTA] both V halves landed (two producer arrivals)
+  uint64_t* v_empty = v_full + VS;         // V slot free: PV of its key tile is done
+  uint64_t* v_tail = v_empty + VS;         // this CTA's partial last V tile landed
+  uint64_t* s_full = v_tail + 1;           // [key tile & 1]
+  uint64_t* p_full = s_full + 2;           // [even CTA][key tile & 1]: P written, one arrival per softmax warp
+  uint64_t* o_done = p_full + 2;           // [key tile & 1]: O += P V of that key tile is complete
+  uint64_t* drain = o_done + 2;            // [even CTA] every issued product has completed
+  float* m_part = reinterpret_cast<float*>(smem + XCH_OFF);  // [key tile & 1][half][row]
+  float* l_part = m_part + 4 * BM;                            // [half][row]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + MISC_OFF);
-  volatile int* lo_flag = reinterpret_cast<volatile int*>(smem + MISC_OFF + 4);  // [t][j & 1]
+  volatile int* lo_flag = reinterpret_cast<volatile int*>(smem + MISC_OFF + 4);  // [rank][j & 1][half], even CTA
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cta_rank();
+  const bool leader = rank == 0;
   const int G = p.num_q_heads / p.num_kv_heads;
-  // CTA -> (pair unit, KV head, sequence).  G >= 2: two heads of the group over the same 128 rows;
-  // G == 1: the group's single head over two consecutive 128-row tiles.
-  int u = blockIdx.x;
+  // pair -> (unit, KV head, sequence); the pairs reading the same K/V are adjacent
+  int u = blockIdx.x >> 1;
   const int unit = u % p.units;
   u /= p.units;
   const int g = u % p.num_kv_heads;
   const int b = u / p.num_kv_heads;
-  int head[2], mrow[2];
+  int head, mrow, mrow_lo, mrow_hi;  // this CTA's head and first row; the pair's first and last row tiles
   if (G >= 2) {
-    const int pair = unit % (G / 2), mt = unit / (G / 2);
-    head[0] = g * G + 2 * pair;
-    head[1] = head[0] + 1;
-    mrow[0] = mrow[1] = mt * BM;
+    const int hp = unit % (G / 2), mt = unit / (G / 2);
+    head = g * G + 2 * hp + (int)rank;
+    mrow = mrow_lo = mrow_hi = mt * BM;
   } else {
-    head[0] = head[1] = g;
-    mrow[0] = unit * 2 * BM;
-    mrow[1] = mrow[0] + BM;
+    head = g;
+    mrow = (2 * unit + (int)rank) * BM;
+    mrow_lo = 2 * unit * BM;
+    mrow_hi = mrow_lo + BM;
   }
 
   const int q0 = __ldg(p.query_start_loc + b), q1 = __ldg(p.query_start_loc + b + 1);
   const int C = q1 - q0;
-  if (mrow[0] >= C) return;
+  // both CTAs of a pair take the same early exits (they depend on the pair only)
+  if (mrow_lo >= C) return;
   const int L = __ldg(p.context_lens + b);
   const int cap = p.max_blocks_per_seq * p.block_size;
-  if (L > cap || L < C) {  // broken caller invariant: record and produce nothing for this tile
+  if (L > cap || L < C) {  // broken caller invariant: record and produce nothing for this pair
     if (threadIdx.x == 0) PA_RECORD_ERROR(PA_ERRBIT_INDEX);
     return;
   }
-  // keys [0, kend) are visible to some row of either tile
-  const int kend = min(L, L - C + max(mrow[0], mrow[1]) + BM);
+  // keys [0, kend) are visible to some row of the pair
+  const int kend = L - C + min(mrow_hi + BM, C);
   const int nkv = (kend + BN - 1) / BN;
 
   if (threadIdx.x == 0) {
-    lo_flag[0] = lo_flag[1] = lo_flag[2] = lo_flag[3] = 0;
-    mbar_init(q_full, 1);
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < 8; ++i) lo_flag[i] = 0;
+    mbar_init(q_full, 2 * kSoftmaxWarps);
+    for (int i = 0; i < KS; ++i) {
       mbar_init(&k_full[i], 1);
-      mbar_init(&v_full[i], 1);
       mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < VS; ++i) {
+      mbar_init(&v_full[i], 2);
       mbar_init(&v_empty[i], 1);
     }
-    for (int i = 0; i < 4; ++i) {
+    mbar_init(v_tail, 1);
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], BM);
+      mbar_init(&p_full[i], 2 * kSoftmaxWarps);
+      mbar_init(&o_done[i], 1);
     }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(&p_full[t], BM);
-      mbar_init(&o_done[t * 2], 1);
-      mbar_init(&o_done[t * 2 + 1], 1);
-    }
+    mbar_init(drain, 1);
     fence_mbar_init();
   }
-  if (warp == 9) {  // TMEM: S_0 x2, S_1 x2, O_0, O_1
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+  if (warp == 9) {  // the same warp in both CTAs allocates the pair's TMEM
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(TMEM_COLS)
                  : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
 
   if (warp == 8) {
-    // ============================================ producer: both Q tiles once, then K/V tiles
+    // ============================================ producer: this CTA's K and V halves
     if (lane == 0) {
-      tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
-      mbar_arrive_expect_tx(q_full, 2 * QTILE);
-      for (int t = 0; t < 2; ++t)
-        for (int hf = 0; hf < 2; ++hf)
-          tma_load_2d(smem + Q_OFF + t * QTILE + hf * QHALF, &qmap, head[t] * HD + hf * 64, q0 + mrow[t], q_full);
     }
     const int32_t* bt = p.block_tables + (size_t)b * p.max_blocks_per_seq;
-    auto lookup = [&](int j) -> int {
-      const int key = j * BN + lane * 16;
-      return (j < nkv && lane < BN / 16 && key < kend) ? __ldg(bt + key / p.block_size) : 0;
+    const uint32_t kfull0 = map_rank(smem_u32(k_full), 0), vfull0 = map_rank(smem_u32(v_full), 0);
+    // first key of box i of key tile j: K boxes cover this CTA's 64 keys, V boxes all 128
+    auto kbox_key = [&](int j, int i) { return j * BN + (int)rank * (BN / 2) + i * 16; };
+    auto vbox_key = [&](int j, int i) { return j * BN + i * 16; };
+    auto nbox = [&](int key0, int maxb) { return max(0, min(maxb, (kend - key0 + 15) / 16)); };
+    auto phys_of = [&](int key) -> int { return key < kend ? __ldg(bt + key / p.block_size) : 0; };
+    auto wait1 = [&](uint64_t* bar, uint32_t parity) -> bool {
+      int r = 1;
+      if (lane == 0) r = mbar_wait(bar, parity) ? 1 : 0;
+      return __shfl_sync(0xffffffffu, r, 0) != 0;
     };
-    // K and V tiles are issued as their own slots free up: K slots early (after the S products),
-    // V slots late (after the PV products), so K runs ahead of V.
-    int jk = 0, jv = 0;
-    int physk = lookup(0), physv = physk;
-    auto issue = [&](int j, int phys, uint64_t* full, const CUtensorMap* map, int off) {
-      const int st = j % kStages;
-      const int nbox = min(BN / 16, (kend - j * BN + 15) / 16);
-      if (lane == 0) mbar_arrive_expect_tx(&full[st], nbox * 16 * HD * 2);
+    auto put_k = [&](int j) -> bool {
+      const int st = j % KS;
+      if (j >= KS && !wait1(&k_empty[st], ((j / KS) - 1) & 1)) return false;
+      const int mine = nbox(kbox_key(j, 0), 4);
+      if (leader && lane == 0) {  // bytes of both CTAs' boxes
+        const int peer = nbox(j * BN + BN / 2, 4);
+        mbar_arrive_expect_tx(&k_full[st], (mine + peer) * 2 * 16 * 128);
+      }
       __syncwarp();
-      if (lane < nbox) {
+      if (lane < mine) {
+        const int key = kbox_key(j, lane);
+        const int phys = phys_of(key);
         if (phys < 0 || phys >= p.num_blocks) PA_RECORD_ERROR(PA_ERRBIT_INDEX);  // TMA zero-fills out of range
-        const int key = j * BN + lane * 16;
         const int y = phys * p.block_size + key % p.block_size;
         for (int hf = 0; hf < 2; ++hf)
-          tma_load_2d(smem + off + st * KVTILE + hf * KVHALF + lane * 16 * 128, map, g * HD + hf * 64, y, &full[st]);
+          tma_load_2d_pair(sb + K_OFF + st * KTILE + hf * KHALF + lane * 16 * 128, &kmap, g * HD + hf * 64, y,
+                           kfull0 + 8 * st);
       }
+      __syncwarp();
+      return true;
     };
-    // lane 0 polls both rings and broadcasts, so the warp never splits on a wait; the time spent with
-    // neither ring ready is bounded like every other wait
-    uint64_t idle_since = 0;
-    while (jk < nkv || jv < nkv) {
-      int go = 0;  // 1: issue K, 2: issue V
-      if (lane == 0) {
-        if (jk < nkv && (jk < kStages || mbar_try_wait(&k_empty[jk % kStages], ((jk / kStages) - 1) & 1)))
-          go = 1;
-        else if (jv < jk && (jv < kStages || mbar_try_wait(&v_empty[jv % kStages], ((jv / kStages) - 1) & 1)))
-          go = 2;
+    auto put_v = [&](int j) -> bool {
+      const int st = j % VS;
+      if (j >= VS && !wait1(&v_empty[st], ((j / VS) - 1) & 1)) return false;
+      const int nb = nbox(vbox_key(j, 0), 8);
+      const int valid = kend - j * BN;  // keys of this tile that exist
+      const int x = g * HD + (int)rank * 64;
+      auto box = [&](int i, bool pair_bar) {
+        const int key = vbox_key(j, i);
+        const int phys = phys_of(key);
+        if (phys < 0 || phys >= p.num_blocks) PA_RECORD_ERROR(PA_ERRBIT_INDEX);
+        const int y = phys * p.block_size + key % p.block_size;
+        if (pair_bar)
+          tma_load_2d_pair(sb + V_OFF + st * VTILE + i * 16 * 128, &vmap, x, y, vfull0 + 8 * st);
+        else
+          tma_load_2d(smem + V_OFF + st * VTILE + i * 16 * 128, &vmap, x, y, v_tail);
+      };
+      if (valid >= BN) {
+        if (leader && lane == 0) mbar_arrive_expect_tx(&v_full[st], 2 * nb * 16 * 128);
+        __syncwarp();
+        if (lane < nb) box(lane, true);
+        __syncwarp();
+        if (!leader && lane == 0) arrive_cluster_relaxed(vfull0 + 8 * st);
+        return true;
       }
-      go = __shfl_sync(0xffffffffu, go, 0);
-      if (go == 1) {
-        issue(jk, physk, k_full, &kmap, K_OFF);
-        ++jk;
-        physk = lookup(jk);
-        idle_since = 0;
-      } else if (go == 2) {
-        issue(jv, physv, v_full, &vmap, V_OFF);
-        ++jv;
-        physv = lookup(jv);
-        idle_since = 0;
-      } else {
-        int late = 0;
-        if (lane == 0) {
-          const uint64_t now = global_ns();
-          if (idle_since == 0) idle_since = now;
-          late = now - idle_since > PA_WAIT_LIMIT_NS;
-        }
-        if (__shfl_sync(0xffffffffu, late, 0)) {
+      // last, partial tile: land it here, zero the rows past the end (their bytes may be anything,
+      // even NaN, and P is 0 there), then signal the even CTA
+      if (lane == 0) mbar_arrive_expect_tx(v_tail, nb * 16 * 128);
+      __syncwarp();
+      if (lane < nb) box(lane, false);
+      __syncwarp();
+      if (!wait1(v_tail, 0)) return false;
+      uint8_t* vt = smem + V_OFF + st * VTILE;
+      for (int off = valid * 128 + lane * 16; off < VTILE; off += 32 * 16)
+        *reinterpret_cast<uint4*>(vt + off) = make_uint4(0u, 0u, 0u, 0u);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(&v_full[st]);
+        else
+          arrive_cluster_release(vfull0 + 8 * st);
+      }
+      __syncwarp();
+      return true;
+    };
+    // tiles go out in the order the products take them: K(0), then K(j+1), V(j)
+    int jk = 0, jv = 0;
+    if (put_k(0))
+      jk = 1;
+    else
+      ok = false;
+    while (ok && jv < nkv) {
+      if (jk < nkv) {
+        if (!put_k(jk)) {
           ok = false;
           break;
         }
+        ++jk;
       }
-    }
-  } else if (warp == 9) {
-    // ============================================ MMA issuer (one thread issues; the warp zeroes V tails)
-    const uint32_t id_s = idesc(DT == PA_BF16 ? 1 : 0, false, BN);
-    const uint32_t id_pv = idesc(DT == PA_BF16 ? 1 : 0, true, HD);
-    auto issue_pv = [&](int i) -> bool {
-      const int st = i % kStages;
-      if (!mbar_wait(&v_full[st], (i / kStages) & 1)) return false;
-      const int valid = kend - i * BN;
-      if (valid < BN) {  // keys past the end: zero their V rows (their bytes may be anything, even NaN)
-        for (int idx = lane; idx < (BN - valid) * 16; idx += 32) {
-          const int r = valid + idx / 16, c = (idx % 16) * 8;
-          sts128(sb + V_OFF + st * KVTILE + tile_off(r, c, KVHALF), 0, 0, 0, 0);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-      }
-      for (int t = 0; t < 2; ++t) {
-        if (!mbar_wait(&p_full[t], i & 1)) return false;
-        tc_fence_after();
-        const bool lo = lo_flag[t * 2 + (i & 1)] == i + 1;
-        if (lane == 0) {
-          const uint32_t od = tmem + O_COL + t * HD;
-          for (int ks = 0; ks < BN / 16; ++ks)
-            mma_f16(od, kmajor_desc(sb + P_OFF + t * PTILE, 0, ks), v_desc(sb + V_OFF + st * KVTILE, ks), id_pv,
-                    (i > 0 || ks > 0) ? 1u : 0u);
-          if (lo)
-            for (int ks = 0; ks < BN / 16; ++ks)
-              mma_f16(od, kmajor_desc(sb + PL_OFF + t * PTILE, 0, ks), v_desc(sb + V_OFF + st * KVTILE, ks), id_pv,
-                      1u);
-          mma_commit(&o_done[t * 2 + (i & 1)]);
-          if (t == 1) mma_commit(&v_empty[st]);
-        }
-        __syncwarp();
-      }
-      return true;
-    };
-    if (!mbar_wait(q_full, 0)) ok = false;
-    for (int j = 0; j < nkv && ok; ++j) {
-      const int st = j % kStages, buf = j & 1;
-      if (!mbar_wait(&k_full[st], (j / kStages) & 1)) {
+      if (!put_v(jv)) {
         ok = false;
         break;
       }
-      for (int t = 0; t < 2; ++t) {
-        if (j >= 2 && !mbar_wait(&s_free[t * 2 + buf], ((j >> 1) - 1) & 1)) {
+      ++jv;
+    }
+    // the even CTA's full barriers count both CTAs' bytes: wait there for the last copies to land
+    // before the pair can exit (bounded)
+    if (leader) {
+      for (int j = max(0, jk - KS); j < jk; ++j)
+        if (!wait1(&k_full[j % KS], (j / KS) & 1)) ok = false;
+      for (int j = max(0, jv - VS); j < jv; ++j)
+        if (!wait1(&v_full[j % VS], (j / VS) & 1)) ok = false;
+    }
+  } else if (warp == 9) {
+    // ============================================ MMA issuer: one thread of the even CTA
+    if (leader) {
+      const uint32_t id_s = idesc(DT == PA_BF16 ? 1 : 0, false, BN);
+      const uint32_t id_pv = idesc(DT == PA_BF16 ? 1 : 0, true, HD);
+      bool issued = false;
+      auto issue_pv = [&](int i) -> bool {
+        const int st = i % VS, buf = i & 1;
+        if (!mbar_wait_warp(&v_full[st], (i / VS) & 1)) return false;
+        if (!mbar_wait_warp(&p_full[buf], (i >> 1) & 1)) return false;
+        tc_fence_after();
+        bool lo[2];
+        for (int h = 0; h < 2; ++h)
+          lo[h] = lo_flag[0 * 4 + buf * 2 + h] == i + 1 || lo_flag[1 * 4 + buf * 2 + h] == i + 1;
+        if (lane == 0) {
+          const uint32_t pb = tmem + S_COL + buf * BN;
+          for (int ks = 0; ks < BN / 16; ++ks)
+            mma_pair(tmem + O_COL, pb + (ks >> 2) * 64 + (ks & 3) * 8, v_desc(sb + V_OFF + st * VTILE, ks), id_pv,
+                     (i > 0 || ks > 0) ? 1u : 0u);
+          for (int ks = 0; ks < BN / 16; ++ks)
+            if (lo[ks >> 2])
+              mma_pair(tmem + O_COL, pb + (ks >> 2) * 64 + 32 + (ks & 3) * 8, v_desc(sb + V_OFF + st * VTILE, ks),
+                       id_pv, 1u);
+          commit_both(&o_done[buf]);
+          commit_both(&v_empty[st]);
+        }
+        __syncwarp();
+        return true;
+      };
+      if (!mbar_wait_warp(q_full, 0)) ok = false;
+      tc_fence_after();
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int st = j % KS, buf = j & 1;
+        // S buffer j&1 last held P(j-2), whose PV was issued before this point (the tensor core
+        // runs its products in issue order)
+        if (!mbar_wait_warp(&k_full[st], (j / KS) & 1)) {
           ok = false;
           break;
         }
         tc_fence_after();
         if (lane == 0) {
           for (int ks = 0; ks < HD / 16; ++ks)
-            mma_f16(tmem + t * 128 + buf * BN, kmajor_desc(sb + Q_OFF + t * QTILE, QHALF, ks),
-                    kmajor_desc(sb + K_OFF + st * KVTILE, KVHALF, ks), id_s, ks > 0 ? 1u : 0u);
-          mma_commit(&s_full[t * 2 + buf]);
-          if (t == 1) mma_commit(&k_empty[st]);
+            mma_pair(tmem + S_COL + buf * BN, tmem + Q_COL + ks * 8, k_desc(sb + K_OFF + st * KTILE, ks), id_s,
+                     ks > 0 ? 1u : 0u);
+          commit_both(&s_full[buf]);
+          commit_both(&k_empty[st]);
         }
+        issued = true;
         __syncwarp();
+        if (j >= 1 && !issue_pv(j - 1)) ok = false;
       }
-      if (!ok) break;
-      if (j >= 1 && !issue_pv(j - 1)) ok = false;
+      if (ok && !issue_pv(nkv - 1)) ok = false;
+      // every product issued here completes before the pair releases its TMEM (bounded)
+      if (issued) {
+        if (lane == 0) commit_local(drain);
+        __syncwarp();
+        if (!mbar_wait_warp(drain, 0)) ok = false;
+      }
     }
-    if (ok && !issue_pv(nkv - 1)) ok = false;
   } else {
-    // ============================================ softmax warpgroups: warpgroup t, thread r owns row mrow[t] + r
-    const int t = warp >> 2;
+    // ============================================ softmax warpgroups: half hf = warp / 4, thread r = row r
+    const int hf = warp >> 2;
     const int r = threadIdx.x & 127;
-    const int pos = L - C + mrow[t] + r;                      // this row's position (keys 0..pos visible)
+    const int row = mrow + r;
+    const int pos = L - C + row;                              // this row's position (keys 0..pos visible)
     const int last_key = min(pos, L - 1);
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;  // this warp's TMEM lane quarter
-    const uint32_t p_lo = sb + PL_OFF + t * PTILE;
+    const int pair_bar = 3 + (warp & 3);                      // the two warps that own rows 32*(warp&3)..
+    const uint32_t qfull0 = map_rank(smem_u32(q_full), 0), pfull0 = map_rank(smem_u32(p_full), 0);
+    const uint32_t flag0 = map_rank(smem_u32((const void*)lo_flag), 0) + 4u * (rank * 4 + hf);
+    // one arrival per warp on the even CTA's barrier, after every lane's TMEM stores are complete
+    // (the even CTA arrives locally; the odd CTA releases only after it wrote a low-term flag)
+    auto warp_arrive = [&](uint64_t* bar, uint32_t bar0, bool wrote_flag) {
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(bar);
+        else if (wrote_flag)
+          arrive_cluster_release(bar0);
+        else
+          arrive_cluster_relaxed(bar0);
+      }
+    };
+    // the query row's half hf of head_dim into TMEM (packed pairs: the low half holds the even element)
+    {
+      uint32_t w[32];
+      if (row < C) {
+        const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.q) +
+                                                           ((size_t)(q0 + row) * p.num_q_heads + head) * HD + hf * 64);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 v = __ldg(src + i);
+          w[4 * i] = v.x;
+          w[4 * i + 1] = v.y;
+          w[4 * i + 2] = v.z;
+          w[4 * i + 3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) w[i] = 0u;
+      }
+      tmem_st32(tmem + lane_base + Q_COL + hf * 32, w);
+      warp_arrive(q_full, qfull0, false);
+    }
     float m_ref = -INFINITY;  // reference max (log2 units) shared by O and l
-    float l = 0.f;
-    float s[BN];
+    float l = 0.f;            // running sum over this half's keys
+    float s[64];
     for (int j = 0; j < nkv && ok; ++j) {
       const int buf = j & 1;
-      if (!mbar_wait(&s_full[t * 2 + buf], (j >> 1) & 1)) {
+      const uint32_t sbuf = tmem + lane_base + S_COL + buf * BN + hf * 64;
+      if (!mbar_wait_warp(&s_full[buf], (j >> 1) & 1)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      tmem_ld32(tmem + lane_base + t * 128 + buf * BN, s);
-      tmem_ld32(tmem + lane_base + t * 128 + buf * BN + 32, s + 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&s_free[t * 2 + buf]);
-      const int lim = last_key - j * BN;  // last visible column of this key tile
-      if (lim < BN - 1) {
+      {
+        uint32_t raw[32];
+        tmem_ld32(sbuf, raw);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < BN; ++c) s[c] = c <= lim ? s[c] : -INFINITY;
+        for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(raw[c]);
+        tmem_ld32(sbuf + 32, raw);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) s[32 + c] = __uint_as_float(raw[c]);
       }
-      // eight independent partial maxima: short dependency chains
+      const int lim = last_key - (j * BN + hf * 64);  // last visible column of this half-tile
+      if (lim < 63) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) s[c] = c <= lim ? s[c] : -INFINITY;
+      }
       float pm[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) pm[e] = s[e];
 #pragma unroll
-      for (int c = 8; c < BN; ++c) pm[c & 7] = fmaxf(pm[c & 7], s[c]);
+      for (int c = 8; c < 64; ++c) pm[c & 7] = fmaxf(pm[c & 7], s[c]);
       float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-      mx *= p.scale_log2;
+      // swap half-tile maxima with the warp that owns the same rows; the barrier also orders both
+      // warps' S reads before either writes P over its half of the buffer
+      m_part[(buf * 2 + hf) * BM + r] = mx;
+      named_barrier_sync(pair_bar, 64);
+      mx = fmaxf(mx, m_part[(buf * 2 + (hf ^ 1)) * BM + r]) * p.scale_log2;
       float alpha = 1.f;
       bool rescale = false;
       if (mx > m_ref + kRescaleLog2 || (m_ref == -INFINITY && mx != -INFINITY)) {
@@ -442,75 +574,74 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
 #pragma unroll
       for (int e = 0; e < 8; ++e) ps[e] = 0.f;
 #pragma unroll
-      for (int c = 0; c < BN; ++c) {
+      for (int c = 0; c < 64; ++c) {
         s[c] = fast_exp2(fmaf(s[c], p.scale_log2, neg_m));
         ps[c & 7] += s[c];
       }
       const float rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       l = l * alpha + rs;
-      // does this key tile carry a large share of some row's mass?  (decided per query tile:
-      // tile j needs the low term iff lo_flag[t][j&1] == j+1 once the warpgroup has voted)
-      if (__any_sync(0xffffffffu, rs >= kLoFraction * l) && lane == 0) lo_flag[t * 2 + (j & 1)] = j + 1;
-      named_barrier_sync(1 + t, BM);
-      const bool lo = lo_flag[t * 2 + (j & 1)] == j + 1;
-      const uint32_t p_hi = sb + P_OFF + t * PTILE;
-      // the P buffers and O are touched only after the PV of key tile j-1 is complete
-      if (j >= 1 && !mbar_wait(&o_done[t * 2 + ((j - 1) & 1)], ((j - 1) >> 1) & 1)) {
-        ok = false;
-        break;
+      // does this half-tile carry a large share of some row's mass in this half?  Any warp of
+      // either CTA that says so makes the even CTA issue the low term's product for the half (the
+      // low term is always written, so every row's is there)
+      const bool flag = __any_sync(0xffffffffu, rs >= kLoFraction * l);
+      if (flag && lane == 0) {
+        if (leader)
+          lo_flag[rank * 4 + buf * 2 + hf] = j + 1;
+        else
+          st_cluster(flag0 + 8u * buf, (uint32_t)(j + 1));
       }
       if (__any_sync(0xffffffffu, rescale)) {
+        // O must hold PV(j-1) before it is scaled; PV(j) waits for this tile's P
+        if (j >= 1 && !mbar_wait_warp(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < HD; c += 32) {
-          float o[32];
-          tmem_ld32(tmem + lane_base + O_COL + t * HD + c, o);
+        for (int c = 0; c < 64; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_base + O_COL + hf * 64 + c, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= alpha;
-          tmem_st32(tmem + lane_base + O_COL + t * HD + c, o);
-        }
-        tmem_wait_st();
-      }
-#pragma unroll
-      for (int c = 0; c < BN; c += 8) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) w[e] = Elt<DT>::from_f2(s[c + 2 * e], s[c + 2 * e + 1]);
-        sts128(p_hi + tile_off(r, c, 0), w[0], w[1], w[2], w[3]);
-        if (lo) {
-          uint32_t wl[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 hv = Elt<DT>::to_f2(w[e]);
-            wl[e] = Elt<DT>::from_f2(s[c + 2 * e] - hv.x, s[c + 2 * e + 1] - hv.y);
-          }
-          sts128(p_lo + tile_off(r, c, 0), wl[0], wl[1], wl[2], wl[3]);
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tmem + lane_base + O_COL + hf * 64 + c, o);
         }
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&p_full[t]);
+      {
+        uint32_t w[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) w[e] = Elt<DT>::from_f2(s[2 * e], s[2 * e + 1]);
+        tmem_st32(sbuf, w);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float2 hv = Elt<DT>::to_f2(w[e]);
+          w[e] = Elt<DT>::from_f2(s[2 * e] - hv.x, s[2 * e + 1] - hv.y);
+        }
+        tmem_st32(sbuf + 32, w);
+      }
+      warp_arrive(&p_full[buf], pfull0 + 8u * buf, flag);
     }
-    // epilogue: O / l -> out
-    if (ok && mbar_wait(&o_done[t * 2 + ((nkv - 1) & 1)], ((nkv - 1) >> 1) & 1)) {
+    // epilogue: O / (l_0 + l_1) -> out
+    l_part[hf * BM + r] = l;
+    named_barrier_sync(pair_bar, 64);
+    const float lsum = l + l_part[(hf ^ 1) * BM + r];
+    if (ok && mbar_wait_warp(&o_done[(nkv - 1) & 1], ((nkv - 1) >> 1) & 1)) {
       tc_fence_after();
-      const int row = mrow[t] + r;
-      T* orow = reinterpret_cast<T*>(p.out) + ((size_t)(q0 + row) * p.num_q_heads + head[t]) * HD;
-      const float inv = 1.f / l;
+      T* orow = reinterpret_cast<T*>(p.out) + ((size_t)(q0 + row) * p.num_q_heads + head) * HD + hf * 64;
+      const float inv = 1.f / lsum;
 #pragma unroll
-      for (int c = 0; c < HD; c += 32) {
-        float o[32];
-        tmem_ld32(tmem + lane_base + O_COL + t * HD + c, o);
+      for (int c = 0; c < 64; c += 32) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_base + O_COL + hf * 64 + c, o);
         tmem_wait_ld();
         if (row < C) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
             uint4 v;
-            v.x = Elt<DT>::from_f2(o[e] * inv, o[e + 1] * inv);
-            v.y = Elt<DT>::from_f2(o[e + 2] * inv, o[e + 3] * inv);
-            v.z = Elt<DT>::from_f2(o[e + 4] * inv, o[e + 5] * inv);
-            v.w = Elt<DT>::from_f2(o[e + 6] * inv, o[e + 7] * inv);
+            v.x = Elt<DT>::from_f2(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
+            v.y = Elt<DT>::from_f2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+            v.z = Elt<DT>::from_f2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
+            v.w = Elt<DT>::from_f2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
             *reinterpret_cast<uint4*>(orow + c + e) = v;
           }
         }
@@ -520,11 +651,12 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
     }
   }
   if (!ok && lane == 0) PA_RECORD_ERROR(PA_ERRBIT_TIMEOUT);
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // no product, copy or remote arrival of the pair is still in flight
   tc_fence_after();
   if (warp == 9)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
 }
 
 }  // namespace
@@ -551,10 +683,11 @@ extern "C" int pa_prefill_chunk(const void* q, const int32_t* query_start_loc, i
   if ((long)num_blocks * block_size >= (1L << 31)) return PA_ERR_UNSUPPORTED;
   const int mtiles = (max_chunk_len + BM - 1) / BM;
   const int units = G >= 2 ? (G / 2) * mtiles : (mtiles + 1) / 2;
-  const long grid = (long)batch * num_kv_heads * units;
+  const long grid = 2L * batch * num_kv_heads * units;
   if (grid > 0x7fffffffL) return PA_ERR_UNSUPPORTED;
 
   PrefillParams p;
+  p.q = q;
   p.out = out;
   p.query_start_loc = query_start_loc;
   p.block_tables = block_tables;
@@ -569,12 +702,9 @@ extern "C" int pa_prefill_chunk(const void* q, const int32_t* query_start_loc, i
   p.units = units;
   p.scale_log2 = scale * kLog2e;
 
-  CUtensorMap qm, km, vm;
+  CUtensorMap km, vm;
   const uint64_t rows = (uint64_t)num_blocks * block_size;
   const uint64_t cols = (uint64_t)num_kv_heads * HD;
-  if (pa::encode_2d_sw128(&qm, q, (uint64_t)num_q_heads * HD, (uint64_t)total_q_tokens, (uint64_t)num_q_heads * HD * 2,
-                          64, BM) != PA_OK)
-    return PA_ERR_CUDA;
   if (pa::encode_2d_sw128(&km, k_cache, cols, rows, cols * 2, 64, 16) != PA_OK) return PA_ERR_CUDA;
   if (pa::encode_2d_sw128(&vm, v_cache, cols, rows, cols * 2, 64, 16) != PA_OK) return PA_ERR_CUDA;
 
@@ -588,6 +718,6 @@ extern "C" int pa_prefill_chunk(const void* q, const int32_t* query_start_loc, i
       return PA_ERR_CUDA;
     if (dev >= 0 && dev < 64) attr_set[di][dev] = true;
   }
-  kern<<<(unsigned)grid, 320, SMEM_ALLOC, (cudaStream_t)stream>>>(qm, km, vm, p);
+  kern<<<(unsigned)grid, 320, SMEM_ALLOC, (cudaStream_t)stream>>>(km, vm, p);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
