@@ -22,23 +22,26 @@
 // So each CTA streams half of every K and V tile from L2 (the bound of the
 // one-CTA form) and the paired product runs at ~0.8 of the tensor peak where a
 // one-CTA 128 x 128 x 16 product with A in TMEM stops near 0.6.
-// A TMA producer warp per CTA gathers its 16-row K and V boxes through the
-// block table (128-byte swizzle, no multicast) into four-stage K and V rings;
+// Two TMA producer warps per CTA (one for K, one for V: a TMA issue stalls
+// while the unit is busy) gather its 16-row K and V boxes through the block
+// table (128-byte swizzle, no multicast) into four-stage K and V rings;
 // the copies of both CTAs complete on the even CTA's barriers (TMA
 // .cta_group::2), slots are released by a multicast tcgen05.commit, and the
 // last, partial V tile is loaded against a local barrier and zero-filled past
-// the end before it is signalled.  The MMA thread issues S(j) and then
-// O += P(j-1) V, so the tensor core runs PV(j-1) and S(j+1) while the softmax
-// works on S(j).  In each CTA two softmax warpgroups split every key tile in
+// the end before it is signalled.  Two threads of the even CTA issue the
+// products, one S(j) and one O += P(j) V, so the tensor core runs PV(j-1) and
+// S(j+1) while the softmax works on S(j).  In each CTA two softmax warpgroups split every key tile in
 // halves (keys 0-63 and 64-127; thread r = row r = TMEM lane r): they swap
 // their half-tile maxima through shared memory, keep fp32 running sums per
 // half (added at the end), rescale O in TMEM only when the running max grows
 // by more than 2^8 (exact: O and the sums always share one reference max), and
-// write P as a high and a low 16-bit term.  The low term's product is issued
-// for a half-tile only when some row of either CTA puts at least 1/16 of that
-// half's running mass there (always the first tile, and tiles with dominant
-// keys): exact to ~2^-17 there; elsewhere the high term alone moves an output
-// by at most 2^-9 |v| / 16.
+// write P's high 16-bit term.  A warp in which some row puts at least 1/16 of
+// that half's running mass in the half-tile (always the first tile, and tiles
+// with dominant keys) also writes P's low term, exact to ~2^-17, and the
+// other warps write zeros there; the even CTA issues the low term's product
+// for a half when any warp of the pair asked.  Without it the high term alone
+// moves an output by at most 2^-9 |v| / 16.  3 of every 8 exponentials run
+// as a polynomial on the FMA pipe to relieve the MUFU unit.
 
 #include <algorithm>
 
@@ -70,8 +73,8 @@ constexpr int V_OFF = K_OFF + KS * KTILE;       // V[VS]
 constexpr int XCH_OFF = V_OFF + VS * VTILE;     // float m_part[2][2][128], l_part[2][128]
 constexpr int BAR_OFF = XCH_OFF + 6 * BM * 4;
 // barriers: q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], v_tail, s_full[2], p_full[2],
-// o_done[2], drain.  The full barriers, q_full, p_full and drain are used in the even CTA only.
-constexpr int NBAR = 1 + 2 * KS + 2 * VS + 1 + 2 + 2 + 2 + 1;
+// o_done[2], drain[2].  The full barriers, q_full, p_full and drain are used in the even CTA only.
+constexpr int NBAR = 1 + 2 * KS + 2 * VS + 1 + 2 + 2 + 2 + 2;
 constexpr int MISC_OFF = BAR_OFF + NBAR * 8;    // tmem base (4 B), lo flags int[2 ranks][2][2 halves]
 constexpr int SMEM_BYTES = MISC_OFF + 4 + 32 + 28;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
@@ -85,6 +88,9 @@ constexpr int Q_COL = 0;
 constexpr int S_COL = 128;
 constexpr int O_COL = 384;
 constexpr int kSoftmaxWarps = 8;        // per CTA; q_full and p_full count one arrival per warp of the pair
+// warps 0-7 softmax, 8 K producer, 9 S issuer (even CTA) and TMEM allocator, 10 V producer,
+// 11 PV issuer (even CTA)
+constexpr int kThreads = 12 * 32;
 
 struct PrefillParams {
   const void* q;
@@ -213,9 +219,63 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* v) {
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// ---------------------------------------------------------------- softmax arithmetic
+// Packed pairs of fp32 (Blackwell's f32x2 FMA/add issue two lanes' worth in one instruction).
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// 2^x for a pair, on the FMA pipe instead of the MUFU unit (which issues 16 exp2 per clock per SM
+// and bounds the softmax otherwise).  x is clamped to [-125, +inf) (every x here is <= 8), split
+// as x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in the low mantissa bits) and
+// f in [-1/2, 1/2]; 2^f is a degree-4 polynomial fitted here for minimal relative error on that
+// interval (weighted least squares driven toward equioscillation; max relative error 2.7e-6,
+// below the 2^-17 of the two-term P), and 2^n enters as n added to the exponent field.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float x0, x1;
+  upk2(x2, x0, x1);
+  x2 = pk2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t one = pk2(1.f, 1.f), neg_one = pk2(-1.f, -1.f);
+  const uint64_t magic = pk2(12582912.f, 12582912.f), neg_magic = pk2(-12582912.f, -12582912.f);
+  const uint64_t t = fma2(x2, one, magic);       // n in the low mantissa bits
+  const uint64_t n = fma2(t, one, neg_magic);    // n as a float
+  const uint64_t f = fma2(n, neg_one, x2);       // x - n
+  uint64_t q = pk2(9.570068680e-03f, 9.570068680e-03f);
+  q = fma2(q, f, pk2(5.591780692e-02f, 5.591780692e-02f));
+  q = fma2(q, f, pk2(2.402474433e-01f, 2.402474433e-01f));
+  q = fma2(q, f, pk2(6.931218505e-01f, 6.931218505e-01f));
+  q = fma2(q, f, pk2(9.999992847e-01f, 9.999992847e-01f));
+  float q0, q1, t0, t1;
+  upk2(q, q0, q1);
+  upk2(t, t0, t1);
+  // the bits of t are 0x4B400000 + n, so (bits << 23) is n << 23 modulo 2^32
+  return pk2(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
+             __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
+}
+constexpr int kPolyPairs = 3;  // of every 8 pairs of a row's half-tile, this many take exp2_poly2
+
 // --------------------------------------------------------------- kernel
 template <int DT>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                    const PrefillParams p) {
   using T = typename Elt<DT>::T;
@@ -232,7 +292,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
   uint64_t* s_full = v_tail + 1;           // [key tile & 1]
   uint64_t* p_full = s_full + 2;           // [even CTA][key tile & 1]: P written, one arrival per softmax warp
   uint64_t* o_done = p_full + 2;           // [key tile & 1]: O += P V of that key tile is complete
-  uint64_t* drain = o_done + 2;            // [even CTA] every issued product has completed
+  uint64_t* drain = o_done + 2;            // [even CTA][issuer] every product it issued has completed
   float* m_part = reinterpret_cast<float*>(smem + XCH_OFF);  // [key tile & 1][half][row]
   float* l_part = m_part + 4 * BM;                            // [half][row]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + MISC_OFF);
@@ -291,7 +351,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       mbar_init(&p_full[i], 2 * kSoftmaxWarps);
       mbar_init(&o_done[i], 1);
     }
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     fence_mbar_init();
   }
   if (warp == 9) {  // the same warp in both CTAs allocates the pair's TMEM
@@ -306,8 +367,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
 
-  if (warp == 8) {
-    // ============================================ producer: this CTA's K and V halves
+  if (warp == 8 || warp == 10) {
+    // ============================================ producers: this CTA's K halves (warp 8) and V
+    // halves (warp 10); a TMA issue stalls while the unit is busy, so K and V get a warp each
     if (lane == 0) {
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
@@ -390,25 +452,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       __syncwarp();
       return true;
     };
-    // tiles go out in the order the products take them: K(0), then K(j+1), V(j)
     int jk = 0, jv = 0;
-    if (put_k(0))
-      jk = 1;
-    else
-      ok = false;
-    while (ok && jv < nkv) {
-      if (jk < nkv) {
+    if (warp == 8) {
+      for (; jk < nkv; ++jk)
         if (!put_k(jk)) {
           ok = false;
           break;
         }
-        ++jk;
-      }
-      if (!put_v(jv)) {
-        ok = false;
-        break;
-      }
-      ++jv;
+    } else {
+      for (; jv < nkv; ++jv)
+        if (!put_v(jv)) {
+          ok = false;
+          break;
+        }
     }
     // the even CTA's full barriers count both CTAs' bytes: wait there for the last copies to land
     // before the pair can exit (bounded)
@@ -418,63 +474,70 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       for (int j = max(0, jv - VS); j < jv; ++j)
         if (!wait1(&v_full[j % VS], (j / VS) & 1)) ok = false;
     }
-  } else if (warp == 9) {
-    // ============================================ MMA issuer: one thread of the even CTA
+  } else if (warp == 9 || warp == 11) {
+    // ============================================ MMA issuers, even CTA: S products from warp 9, PV
+    // products from warp 11.  tcgen05.commit holds its thread until the products ahead of it have
+    // gone to the tensor core, so one thread issuing both would leave the tensor core idle around
+    // every commit; with two, S(j+1) runs while PV(j) is being issued.  The two streams are not
+    // ordered with each other, so S(j) waits for PV(j-2) (which read P(j-2) from the same TMEM
+    // buffer) to complete.
     if (leader) {
       const uint32_t id_s = idesc(DT == PA_BF16 ? 1 : 0, false, BN);
       const uint32_t id_pv = idesc(DT == PA_BF16 ? 1 : 0, true, HD);
       bool issued = false;
-      auto issue_pv = [&](int i) -> bool {
-        const int st = i % VS, buf = i & 1;
-        if (!mbar_wait_warp(&v_full[st], (i / VS) & 1)) return false;
-        if (!mbar_wait_warp(&p_full[buf], (i >> 1) & 1)) return false;
-        tc_fence_after();
-        bool lo[2];
-        for (int h = 0; h < 2; ++h)
-          lo[h] = lo_flag[0 * 4 + buf * 2 + h] == i + 1 || lo_flag[1 * 4 + buf * 2 + h] == i + 1;
-        if (lane == 0) {
-          const uint32_t pb = tmem + S_COL + buf * BN;
-          for (int ks = 0; ks < BN / 16; ++ks)
-            mma_pair(tmem + O_COL, pb + (ks >> 2) * 64 + (ks & 3) * 8, v_desc(sb + V_OFF + st * VTILE, ks), id_pv,
-                     (i > 0 || ks > 0) ? 1u : 0u);
-          for (int ks = 0; ks < BN / 16; ++ks)
-            if (lo[ks >> 2])
-              mma_pair(tmem + O_COL, pb + (ks >> 2) * 64 + 32 + (ks & 3) * 8, v_desc(sb + V_OFF + st * VTILE, ks),
-                       id_pv, 1u);
-          commit_both(&o_done[buf]);
-          commit_both(&v_empty[st]);
+      uint64_t* my_drain = drain + (warp == 9 ? 0 : 1);
+      if (warp == 9) {
+        if (!mbar_wait_warp(q_full, 0)) ok = false;
+        for (int j = 0; j < nkv && ok; ++j) {
+          const int st = j % KS, buf = j & 1;
+          if (!mbar_wait_warp(&k_full[st], (j / KS) & 1) ||
+              (j >= 2 && !mbar_wait_warp(&o_done[buf], ((j - 2) >> 1) & 1))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (lane == 0) {
+            for (int ks = 0; ks < HD / 16; ++ks)
+              mma_pair(tmem + S_COL + buf * BN, tmem + Q_COL + ks * 8, k_desc(sb + K_OFF + st * KTILE, ks), id_s,
+                       ks > 0 ? 1u : 0u);
+            commit_both(&s_full[buf]);
+            commit_both(&k_empty[st]);
+          }
+          issued = true;
+          __syncwarp();
         }
-        __syncwarp();
-        return true;
-      };
-      if (!mbar_wait_warp(q_full, 0)) ok = false;
-      tc_fence_after();
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int st = j % KS, buf = j & 1;
-        // S buffer j&1 last held P(j-2), whose PV was issued before this point (the tensor core
-        // runs its products in issue order)
-        if (!mbar_wait_warp(&k_full[st], (j / KS) & 1)) {
-          ok = false;
-          break;
+      } else {
+        for (int i = 0; i < nkv && ok; ++i) {
+          const int st = i % VS, buf = i & 1;
+          if (!mbar_wait_warp(&v_full[st], (i / VS) & 1) || !mbar_wait_warp(&p_full[buf], (i >> 1) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          bool lo[2];
+          for (int h = 0; h < 2; ++h)
+            lo[h] = lo_flag[0 * 4 + buf * 2 + h] == i + 1 || lo_flag[1 * 4 + buf * 2 + h] == i + 1;
+          if (lane == 0) {
+            const uint32_t pb = tmem + S_COL + buf * BN;
+            for (int ks = 0; ks < BN / 16; ++ks)
+              mma_pair(tmem + O_COL, pb + (ks >> 2) * 64 + (ks & 3) * 8, v_desc(sb + V_OFF + st * VTILE, ks), id_pv,
+                       (i > 0 || ks > 0) ? 1u : 0u);
+            for (int ks = 0; ks < BN / 16; ++ks)
+              if (lo[ks >> 2])
+                mma_pair(tmem + O_COL, pb + (ks >> 2) * 64 + 32 + (ks & 3) * 8, v_desc(sb + V_OFF + st * VTILE, ks),
+                         id_pv, 1u);
+            commit_both(&o_done[buf]);
+            commit_both(&v_empty[st]);
+          }
+          issued = true;
+          __syncwarp();
         }
-        tc_fence_after();
-        if (lane == 0) {
-          for (int ks = 0; ks < HD / 16; ++ks)
-            mma_pair(tmem + S_COL + buf * BN, tmem + Q_COL + ks * 8, k_desc(sb + K_OFF + st * KTILE, ks), id_s,
-                     ks > 0 ? 1u : 0u);
-          commit_both(&s_full[buf]);
-          commit_both(&k_empty[st]);
-        }
-        issued = true;
-        __syncwarp();
-        if (j >= 1 && !issue_pv(j - 1)) ok = false;
       }
-      if (ok && !issue_pv(nkv - 1)) ok = false;
-      // every product issued here completes before the pair releases its TMEM (bounded)
+      // every product this thread issued completes before the pair releases its TMEM (bounded)
       if (issued) {
-        if (lane == 0) commit_local(drain);
+        if (lane == 0) commit_local(my_drain);
         __syncwarp();
-        if (!mbar_wait_warp(drain, 0)) ok = false;
+        if (!mbar_wait_warp(my_drain, 0)) ok = false;
       }
     }
   } else {
@@ -547,16 +610,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
         for (int c = 0; c < 32; ++c) s[32 + c] = __uint_as_float(raw[c]);
       }
       const int lim = last_key - (j * BN + hf * 64);  // last visible column of this half-tile
-      if (lim < 63) {
+      const bool diag = lim < 63;
+      if (diag) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) s[c] = c <= lim ? s[c] : -INFINITY;
       }
       float pm[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) pm[e] = s[e];
+      for (int e = 0; e < 8; ++e) pm[e] = max3(s[e], s[8 + e], s[16 + e]);
 #pragma unroll
-      for (int c = 8; c < 64; ++c) pm[c & 7] = fmaxf(pm[c & 7], s[c]);
-      float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      for (int c = 24; c < 64; c += 16)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pm[e] = max3(pm[e], s[c + e], s[c + 8 + e]);
+      float mx = max3(max3(pm[0], pm[1], pm[2]), max3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
       // swap half-tile maxima with the warp that owns the same rows; the barrier also orders both
       // warps' S reads before either writes P over its half of the buffer
       m_part[(buf * 2 + hf) * BM + r] = mx;
@@ -570,19 +636,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
         m_ref = mx;
       }
       const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
-      float ps[8];
+      // P = 2^(s * scale_log2 - m_ref), pairwise: 5 of every 8 pairs on the MUFU unit, 3 on the
+      // FMA pipe; exact zeros where the causal mask applies
+      const uint64_t sc2 = pk2(p.scale_log2, p.scale_log2), nm2 = pk2(neg_m, neg_m);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ps[e] = 0.f;
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        s[c] = fast_exp2(fmaf(s[c], p.scale_log2, neg_m));
-        ps[c & 7] += s[c];
+      for (int e = 0; e < 32; ++e) {
+        const uint64_t x2 = fma2(pk2(s[2 * e], s[2 * e + 1]), sc2, nm2);
+        uint64_t p2;
+        if ((e & 7) < kPolyPairs) {
+          p2 = exp2_poly2(x2);
+        } else {
+          float x0, x1;
+          upk2(x2, x0, x1);
+          p2 = pk2(fast_exp2(x0), fast_exp2(x1));
+        }
+        upk2(p2, s[2 * e], s[2 * e + 1]);
       }
-      const float rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      if (diag) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) s[c] = c <= lim ? s[c] : 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 32; ++e) acc[e & 3] = add2(acc[e & 3], pk2(s[2 * e], s[2 * e + 1]));
+      float a0, a1, a2, a3;
+      upk2(add2(acc[0], acc[1]), a0, a1);
+      upk2(add2(acc[2], acc[3]), a2, a3);
+      const float rs = (a0 + a2) + (a1 + a3);
       l = l * alpha + rs;
-      // does this half-tile carry a large share of some row's mass in this half?  Any warp of
-      // either CTA that says so makes the even CTA issue the low term's product for the half (the
-      // low term is always written, so every row's is there)
+      // does this half-tile carry a large share of some row's mass in this half?  Such a warp
+      // writes P's low term and flags the half, which makes the even CTA issue the low term's
+      // product for it; every other warp writes zeros there, so each row gets its low term or none
       const bool flag = __any_sync(0xffffffffu, rs >= kLoFraction * l);
       if (flag && lane == 0) {
         if (leader)
@@ -612,10 +696,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) w[e] = Elt<DT>::from_f2(s[2 * e], s[2 * e + 1]);
         tmem_st32(sbuf, w);
+        if (flag) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float2 hv = Elt<DT>::to_f2(w[e]);
-          w[e] = Elt<DT>::from_f2(s[2 * e] - hv.x, s[2 * e + 1] - hv.y);
+          for (int e = 0; e < 32; ++e) {
+            const float2 hv = Elt<DT>::to_f2(w[e]);
+            w[e] = Elt<DT>::from_f2(s[2 * e] - hv.x, s[2 * e + 1] - hv.y);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) w[e] = 0u;
         }
         tmem_st32(sbuf + 32, w);
       }
@@ -718,6 +807,6 @@ extern "C" int pa_prefill_chunk(const void* q, const int32_t* query_start_loc, i
       return PA_ERR_CUDA;
     if (dev >= 0 && dev < 64) attr_set[di][dev] = true;
   }
-  kern<<<(unsigned)grid, 320, SMEM_ALLOC, (cudaStream_t)stream>>>(km, vm, p);
+  kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, (cudaStream_t)stream>>>(km, vm, p);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
