@@ -50,17 +50,20 @@ WORKLOAD_TEXT = {
                "32 q / 8 kv heads, head_dim 128, bf16, block_size 16",
 }
 
-# DRAM bytes (read + write) per launch of the decode split kernel from one ncu capture of this workload,
-# valid only for the kernel source it was taken on (sha256 prefix of decode.cu + common.cuh).
+# DRAM bytes (read + write) per launch of the workload's dominant kernel from one ncu capture,
+# valid only for the kernel source it was taken on (sha256 prefix of the listed csrc files).
+DECODE_SRC = ("decode.cu", "common.cuh")
+PREFILL_SRC = ("prefill.cu", "common.cuh")
 NCU_TRAFFIC = {
-    "qwen_decode": {"bytes": 316_989_184, "src": "27d8eb8781511c66"},
-    "llama70b_long": {"bytes": 1_588_751_424, "src": "27d8eb8781511c66"},
+    "qwen_decode": {"bytes": 316_989_184, "src": "27d8eb8781511c66", "files": DECODE_SRC},
+    "llama70b_long": {"bytes": 1_588_751_424, "src": "27d8eb8781511c66", "files": DECODE_SRC},
+    "prefill": {"bytes": 348_481_024, "src": "0a0c45baf16bf168", "files": PREFILL_SRC},
 }
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(files=DECODE_SRC) -> str:
     h = hashlib.sha256()
-    for f in ("decode.cu", "common.cuh"):
+    for f in files:
         with open(os.path.join(ROOT, "paged_kv_cache_330_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -408,7 +411,7 @@ def run_ours(args):
     alg = kvb + io_bytes(wl)
     achieved = alg / (dec_avg * 1e-3) / 1e9
     tr = NCU_TRAFFIC.get(args.workload)
-    traffic = tr["bytes"] if tr and tr.get("src") == kernel_source_hash() else None
+    traffic = tr["bytes"] if tr and tr.get("src") == kernel_source_hash(tr["files"]) else None
     launches_per_step = 2  # write_kv, decode (split-K merge inside)
     if rank == 0:
         cpu = None
@@ -497,6 +500,8 @@ def run_prefill(args):
     ms_step = e[0].elapsed_time(e[1]) / K
     ms_pf = e[2].elapsed_time(e[3]) / K
     fl = prefill_flops(wl)
+    tr = NCU_TRAFFIC["prefill"]
+    pf_traffic = tr["bytes"] if tr["src"] == kernel_source_hash(tr["files"]) else None
     burst, sustained, kind = measured_bf16_peak()
     line = {
         "metric": "chunked prefill TFLOP/s (bf16, causal, paged context)", "value": fl / (ms_step * 1e-3) / 1e12,
@@ -506,7 +511,7 @@ def run_prefill(args):
         "roofline": {"bound": "tensor", "kernel": "pa_prefill_chunk (tcgen05/TMEM, TMA)",
                      "achieved": fl / (ms_pf * 1e-3) / 1e12, "peak": burst, "peak_kind": kind + " burst",
                      "unit": "TFLOP/s", "frac": fl / (ms_pf * 1e-3) / 1e12 / burst,
-                     "frac_of_sustained": fl / (ms_pf * 1e-3) / 1e12 / sustained, "traffic": None,
+                     "frac_of_sustained": fl / (ms_pf * 1e-3) / 1e12 / sustained, "traffic": pf_traffic,
                      "avg_launch_ms": ms_pf},
         "gpu_launches": 2 * K,
         "clocks": clk.summary(),
