@@ -741,6 +741,10 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
       cp_async_commit();
     };
     for (int j = 0; j < kLookahead; ++j) plan_push(j);
+    // The cache rows read from here on may have just been written by pa_write_kv, which lets this
+    // kernel launch while it runs (programmatic dependent launch; q, the block tables and the lengths
+    // are not its outputs): wait for it to complete before the first load.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     bool ok = true;
     int k = 0;
     for (;; ++k) {
@@ -1047,7 +1051,19 @@ int launch(const CUtensorMap& km, const CUtensorMap& vm, const DecodeParams& p, 
       return PA_ERR_CUDA;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  kern<<<p.grid, (kNW + 2) * 32, LY::ALLOC, st>>>(km, vm, p);
+  // programmatic dependent launch: may start while the preceding pa_write_kv runs (it signals
+  // its dependents at entry); the producer waits for it before the first cache load
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.grid);
+  cfg.blockDim = dim3((kNW + 2) * 32);
+  cfg.dynamicSmemBytes = LY::ALLOC;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, km, vm, p) != cudaSuccess) return PA_ERR_CUDA;
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   return PA_OK;
 }

@@ -26,6 +26,9 @@ __global__ void __launch_bounds__(256) write_kv_kernel(const uint4* __restrict__
                                                        const int64_t* __restrict__ slot_mapping, int64_t total_vecs,
                                                        int vecs_per_row, int64_t num_slots, uint4* __restrict__ kc,
                                                        uint4* __restrict__ vc) {
+  // a decode launched after this may start its set-up now; it waits for this grid to complete
+  // before it reads the cache (programmatic dependent launch)
+  asm volatile("griddepcontrol.launch_dependents;");
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total_vecs;
        i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t t = i / vecs_per_row;
