@@ -55,8 +55,8 @@ WORKLOAD_TEXT = {
 DECODE_SRC = ("decode.cu", "common.cuh")
 PREFILL_SRC = ("prefill.cu", "common.cuh")
 NCU_TRAFFIC = {
-    "qwen_decode": {"bytes": 316_989_184, "src": "27d8eb8781511c66", "files": DECODE_SRC},
-    "llama70b_long": {"bytes": 1_588_751_424, "src": "27d8eb8781511c66", "files": DECODE_SRC},
+    "qwen_decode": {"bytes": 313_465_088, "src": "25100343f6ccb086", "files": DECODE_SRC},
+    "llama70b_long": {"bytes": 1_584_901_888, "src": "25100343f6ccb086", "files": DECODE_SRC},
     "prefill": {"bytes": 348_481_024, "src": "0a0c45baf16bf168", "files": PREFILL_SRC},
 }
 

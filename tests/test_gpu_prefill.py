@@ -52,7 +52,7 @@ def test_prefill_small_no_prefix():
     _compare(out, oracle_prefill(wl), wl, "no prefix")
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 4), (8, 2), (8, 1)])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 4), (8, 2), (8, 1), (16, 1)])
 @pytest.mark.parametrize("bs", [16, 64, 256])
 @pytest.mark.parametrize("dtype", ["bf16", "f16"])
 def test_prefill_ragged(Hq, Hkv, bs, dtype):
