@@ -258,6 +258,21 @@ def run_reference(args):
     return 0
 
 
+def reduce_over_ranks(times_ms, totals, world_size, device):
+    """Max over ranks of each timed duration, sum over ranks of each count (bytes, sequences).
+
+    The ranks are independent replicas, so the job takes its slowest rank's time and does every
+    rank's work; every rank makes the same two collective calls in the same order."""
+    import torch
+    import torch.distributed as dist
+    vals = torch.tensor([float(t) for t in times_ms], dtype=torch.float64, device=device)
+    tot = torch.tensor([float(t) for t in totals], dtype=torch.float64, device=device)
+    if world_size > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
+    return vals.tolist(), tot.tolist()
+
+
 # ------------------------------------------------------------------------------------------------ our arm
 def run_ours(args):
     import torch
@@ -397,13 +412,8 @@ def run_ours(args):
 
     # ---- max over ranks, totals
     kvb = kv_bytes(wl)
-    vals = torch.tensor([ms_step, e2e_ms, float(np.mean(dec_ms))], dtype=torch.float64, device=dev)
-    tot = torch.tensor([float(kvb), float(B)], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
-    ms_step, e2e_ms, dec_avg = vals.tolist()
-    kv_all, seqs_all = tot.tolist()
+    (ms_step, e2e_ms, dec_avg), (kv_all, seqs_all) = reduce_over_ranks(
+        [ms_step, e2e_ms, float(np.mean(dec_ms))], [kvb, B], ws, dev)
     value = kv_all / (ms_step * 1e-3) / 1e9
     e2e_value = kv_all / (e2e_ms * 1e-3) / 1e9
 
