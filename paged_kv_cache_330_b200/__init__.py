@@ -9,7 +9,7 @@ Calls (see the header for exact semantics):
 
 * ``write_kv``       - scatter new tokens' K/V into their cache slots
 * ``copy_blocks``    - copy whole blocks (copy-on-write of shared blocks)
-* ``decode``         - one-token paged attention, split-K with a reduce kernel
+* ``decode``         - one-token paged attention, split-K with the merge in the same kernel
 * ``prefill_chunk``  - causal chunked-prefill attention over the paged cache
 * ``BlockPool``      - host block pool: blocks, block tables, reference counts
 """
