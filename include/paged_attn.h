@@ -178,6 +178,17 @@ int pa_decode_static_scratch(const void* q, const void* k_cache, const void* v_c
 /* [batch+1] device, query_start_loc[0] = 0, non-decreasing, last =          */
 /* total_q_tokens; C_b <= max_chunk_len and C_b <= L_b.  Requires bf16 or   */
 /* f16 with head_dim 128 on the tensor-core path (tcgen05/TMEM).            */
+/* Runs as clusters of two CTAs on one TPC (tcgen05.mma cta_group::2), each  */
+/* CTA 128 query rows; needs no workspace; asynchronous on `stream`.         */
+/* Returns PA_OK (also for batch, total_q_tokens or max_chunk_len = 0),      */
+/* PA_ERR_INVALID (negative sizes, null pointers, num_q_heads not a multiple */
+/* of num_kv_heads, num_blocks = 0), PA_ERR_UNSUPPORTED (dtype, head_dim !=  */
+/* 128, block_size, group size not in {1,2,4,8,16}, caches of 2^31 rows or   */
+/* more), PA_ERR_ALIGN (q, caches, out not 16-byte aligned; int32 arrays not */
+/* 4-byte aligned) or PA_ERR_CUDA.  On the device, a sequence with L_b above */
+/* max_blocks_per_seq*block_size or below C_b, or a block id out of range,   */
+/* sets PA_ERRBIT_INDEX (read with pa_device_error); a pipeline wait past    */
+/* its 2 s bound sets PA_ERRBIT_TIMEOUT.  Nothing traps.                     */
 /* ------------------------------------------------------------------------ */
 int pa_prefill_chunk(const void* q, const int32_t* query_start_loc, int total_q_tokens, int max_chunk_len,
                      const void* k_cache, const void* v_cache, const int32_t* block_tables,
@@ -192,6 +203,8 @@ int pa_prefill_chunk(const void* q, const int32_t* query_start_loc, int total_q_
 /* synchronises the current device, copies the word to *out and clears it. */
 /* Bits: 1 = pipeline wait timed out, 2 = index out of range.               */
 /* ------------------------------------------------------------------------ */
+#define PA_ERRBIT_TIMEOUT 1u
+#define PA_ERRBIT_INDEX 2u
 int pa_device_error(int* out);
 
 /* ------------------------------------------------------------------------ */
