@@ -509,6 +509,38 @@ def run_prefill(args):
     assert pa.device_error() == 0
     ms_step = e[0].elapsed_time(e[1]) / K
     ms_pf = e[2].elapsed_time(e[3]) / K
+
+    # ---- end to end through the public API: pinned host inputs -> device, step, result -> host
+    pin = lambda t: t.pin_memory()
+    h_q, h_kn, h_vn, h_sm = pin(wl.q), pin(wl.k_new), pin(wl.v_new), pin(torch.from_numpy(sm))
+    h_bt, h_lens = pin(torch.from_numpy(bt)), pin(torch.from_numpy(lens))
+    h_qsl = pin(torch.from_numpy(wl.query_start_loc))
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_kn, h_vn, h_sm, h_bt, h_lens, h_qsl))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step(st):
+        for dst, src in ((q, h_q), (kn, h_kn), (vn, h_vn), (smd, h_sm), (btd, h_bt), (lensd, h_lens), (qsl, h_qsl)):
+            dst.copy_(src, non_blocking=True)
+        wr(st)
+        pf(st)
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step(stream)
+    torch.cuda.synchronize(dev)
+    g_e2e = capture(lambda: e2e_step(cs))
+    g_e2e.replay()
+    torch.cuda.synchronize(dev)
+    e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e4.record(stream)
+    for _ in range(K):
+        g_e2e.replay()
+    e5.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e4.elapsed_time(e5) / K
+    assert pa.device_error() == 0
+    del g_step, g_pf, g_e2e
     fl = prefill_flops(wl)
     tr = NCU_TRAFFIC["prefill"]
     pf_traffic = tr["bytes"] if tr["src"] == kernel_source_hash(tr["files"]) else None
@@ -523,6 +555,8 @@ def run_prefill(args):
                      "unit": "TFLOP/s", "frac": fl / (ms_pf * 1e-3) / 1e12 / burst,
                      "frac_of_sustained": fl / (ms_pf * 1e-3) / 1e12 / sustained, "traffic": pf_traffic,
                      "avg_launch_ms": ms_pf},
+        "e2e": {"value": fl / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": 2 * K,
         "clocks": clk.summary(),
     }
