@@ -99,3 +99,26 @@ def test_prefill_row_equals_decode():
     dec = pa.decode(q, kc, vc, btr, ctx, int(ctx.max()), wl.scale)
     diff = (dec.float() - out[rows].float()).abs().max().item()
     assert diff < 2e-2, diff
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (16, 8)])
+@pytest.mark.parametrize("bs", [32, 128])
+def test_prefill_pair_edges(Hq, Hkv, bs):
+    """CTA-pair edges: with one head per KV group a pair covers two consecutive 128-row tiles, so a
+    300-token chunk has three tiles and the second pair holds one tile past the chunk's end; chunks of
+    1, 127, 128 and 129 rows sit on tile boundaries; block sizes 32 and 128."""
+    lens = [300, 900, 129, 128, 60, 1]
+    chunks = [300, 299, 129, 127, 60, 1]
+    wl = make_custom(seed=bs + Hq, lens=lens, chunk_lens=chunks, kind="prefill", num_q_heads=Hq, num_kv_heads=Hkv,
+                     head_dim=128, block_size=bs)
+    out, *_ = gpu_prefill(wl)
+    _compare(out, oracle_prefill(wl), wl, f"pair edges G{Hq // Hkv} bs{bs}")
+
+
+def test_prefill_mixed_prefix_lengths():
+    """Sequences with and without earlier context in one batch: a chunk that is the whole sequence next to
+    chunks appended after long contexts (key tiles fully visible, diagonal tiles, fully masked tiles)."""
+    wl = make_custom(seed=23, lens=[128, 2048, 700, 4097], chunk_lens=[128, 64, 700, 257], kind="prefill",
+                     num_q_heads=8, num_kv_heads=2, head_dim=128, block_size=16, dtype="f16")
+    out, *_ = gpu_prefill(wl)
+    _compare(out, oracle_prefill(wl), wl, "mixed prefixes f16")
