@@ -20,15 +20,21 @@ source pages, in float64 with numpy:
   vLLM-Ascend page, section 3.1, moves softmax out of fp16 for accuracy); causal
   chunked prefill over the paged context (vllm-ascend page, section 1.1, PCP).
 * ``brute``       - a scalar pure-Python twin of ``attention`` for tiny cases.
+* ``rope``        - rotary position embedding of new tokens' queries and keys
+  fused with the KV write (Nano-vLLM-Ascend page, sections 3.1 and 5.1: the
+  rotary multiply by per-position cos/sin tables, inverted by negating sin).
 
-Parity pins (tests/test_oracle_pins.py): the pages' worked block arithmetic
+Parity pins (tests/test_oracle_pins.py, tests/test_oracle_rope.py): the pages' worked block arithmetic
 (tests/golden/), closed forms, torch's float64 scaled_dot_product_attention on
 dense inputs, the scalar twin, and invariants (block permutation, prefix
-sharing, prefill row i == decode of the first prefix+i+1 tokens).  No function
+sharing, prefill row i == decode of the first prefix+i+1 tokens); for the
+rotary step, rotation closed forms, the page's inverse rule, angle addition,
+the relative-position property and torch complex multiplication.  No function
 here is "parity unpinned".
 """
 
-from . import attention, block_pool, brute, kv_write  # noqa: F401
+from . import attention, block_pool, brute, kv_write, rope  # noqa: F401
 from .attention import decode_attention, gather_kv, prefill_attention, split_partials  # noqa: F401
 from .block_pool import OraclePool, replay  # noqa: F401
 from .kv_write import write_kv  # noqa: F401
+from .rope import rope_tokens, rope_write_kv, rotary  # noqa: F401
