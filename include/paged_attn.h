@@ -103,6 +103,42 @@ int pa_copy_blocks(const int32_t* pairs, int num_pairs, void* k_cache, void* v_c
                    int block_size, int num_kv_heads, int head_dim, int dtype, void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Rotary position embedding fused with the KV write (P1 s3.1: each model    */
+/* brings its rotary embedding; P1 s5.1: a rotary multiply of x by           */
+/* per-position cos/sin tables, whose inverse negates sin; P2 s2.2: the      */
+/* write into fixed-size blocks that follows it).                            */
+/*                                                                            */
+/* Pairing (rotate-half): element i of a head turns with element i + D/2 by  */
+/* the angle of column i of the token's table row p = positions[t]:          */
+/*   y[i]       = x[i] * cos[p][i] - x[i + D/2] * sin[p][i]                  */
+/*   y[i + D/2] = x[i + D/2] * cos[p][i] + x[i] * sin[p][i]                  */
+/* in fp32, rounded to nearest even.  For every token t:                     */
+/*   q_out[t][h] = y(q[t][h])                    (all num_q_heads heads)     */
+/* and, if slot = slot_mapping[t] >= 0 (slot -1: no cache write):            */
+/*   k_cache[slot / bs][slot % bs][h] = y(k[t][h]),                          */
+/*   v_cache[slot / bs][slot % bs][h] = v[t][h]  (bitwise)                   */
+/* q, q_out: [num_tokens][num_q_heads][head_dim] device; q_out may equal q   */
+/* (in place) but must not otherwise overlap any other argument.             */
+/* k, v: [num_tokens][num_kv_heads][head_dim] device, read only.             */
+/* positions, slot_mapping: int64 [num_tokens] device.                       */
+/* cos_table, sin_table: fp32 [max_position][head_dim / 2] device, 16-byte   */
+/* aligned, read only.  Caches as for pa_write_kv.  num_tokens == 0 is a     */
+/* no-op (only the caches are checked).  num_tokens * (num_q_heads +         */
+/* 3 * num_kv_heads) * head_dim / 16 must be below 2^31                      */
+/* (PA_ERR_UNSUPPORTED otherwise).  A position outside [0, max_position)    */
+/* leaves every row of that token unwritten and a slot >= num_blocks *       */
+/* block_size leaves its cache rows unwritten; both set PA_ERRBIT_INDEX in   */
+/* the device error word (pa_device_error).  One kernel launch; a          */
+/* pa_decode that follows on the stream may start its set-up early and      */
+/* waits for this kernel before it reads q_out or the cache.                 */
+/* ------------------------------------------------------------------------ */
+int pa_rope_write_kv(const void* q, void* q_out, const void* k, const void* v, const int64_t* positions,
+                     const float* cos_table, const float* sin_table, int max_position,
+                     const int64_t* slot_mapping, int num_tokens, int num_q_heads, void* k_cache,
+                     void* v_cache, int num_blocks, int block_size, int num_kv_heads, int head_dim,
+                     int dtype, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* Paged decode (P1 s2.2.1, s4.2; P2 s2.2, s3.1): one query token per        */
 /* sequence attends to all context_lens[b] tokens of its sequence:           */
 /*   out[b][h] = sum_t softmax_t(scale * <q[b][h], K_b[t][h/G]>) V_b[t][h/G] */

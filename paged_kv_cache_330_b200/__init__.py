@@ -9,6 +9,7 @@ Calls (see the header for exact semantics):
 
 * ``write_kv``       - scatter new tokens' K/V into their cache slots
 * ``copy_blocks``    - copy whole blocks (copy-on-write of shared blocks)
+* ``rope_write_kv``  - rotary embedding of new tokens' q and k, fused with the K/V cache write
 * ``decode``         - one-token paged attention, split-K with the merge in the same kernel
 * ``prefill_chunk``  - causal chunked-prefill attention over the paged cache
 * ``BlockPool``      - host block pool: blocks, block tables, reference counts
@@ -21,7 +22,8 @@ import os
 
 import numpy as np
 
-__all__ = ["PagedAttnError", "PoolOutOfBlocks", "BlockPool", "write_kv", "copy_blocks", "decode", "decode_plan",
+__all__ = ["PagedAttnError", "PoolOutOfBlocks", "BlockPool", "write_kv", "copy_blocks", "rope_write_kv", "decode",
+           "decode_plan",
            "decode_static_scratch",
            "prefill_chunk", "device_error", "lib", "LIB_PATH", "replay_ops", "version"]
 
@@ -50,6 +52,7 @@ _SIGS = {
     "pa_version": (ctypes.c_char_p, []),
     "pa_write_kv": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "pa_copy_blocks": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
+    "pa_rope_write_kv": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "pa_decode_plan": (_i, [_i, _i, _i, _i, _i, _i, _ip, _ip, ctypes.POINTER(_sz)]),
     "pa_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "pa_decode": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _sz, _i, _vp, _vp]),
@@ -140,6 +143,33 @@ def copy_blocks(pairs, k_cache, v_cache, stream=None) -> None:
     NB, bs, Hkv, D = k_cache.shape
     _check(lib.pa_copy_blocks(_ptr(pairs), int(pairs.shape[0]), _ptr(k_cache), _ptr(v_cache), NB, bs, Hkv, D,
                               _dtype_code(k_cache), _stream_handle(stream)), "pa_copy_blocks")
+
+
+def rope_write_kv(q, k, v, positions, cos_table, sin_table, slot_mapping, k_cache, v_cache, q_out=None,
+                  stream=None):
+    """Rotate q [T, Hq, D] and k [T, Hkv, D] by the rows positions (int64 [T]) of the fp32 tables
+    cos_table/sin_table [max_position, D/2]; write the rotated k and the unrotated v into the cache slots
+    (slot_mapping int64 [T], -1 = no cache write).  Returns q_out (a new tensor unless given; q_out=q
+    rotates in place)."""
+    torch = _torch()
+    if q_out is None:
+        q_out = torch.empty_like(q)
+    _contig(q, q_out, k, v, positions, cos_table, sin_table, slot_mapping, k_cache, v_cache)
+    if cos_table.dtype != torch.float32 or sin_table.dtype != torch.float32:
+        raise ValueError("cos/sin tables must be float32")
+    if q_out.shape != q.shape or q_out.dtype != q.dtype:
+        raise ValueError("q_out must match q")
+    NB, bs, Hkv, D = k_cache.shape
+    T, Hq = int(q.shape[0]), int(q.shape[1])
+    if tuple(k.shape) != (T, Hkv, D) or tuple(v.shape) != (T, Hkv, D) or q.shape[2] != D:
+        raise ValueError("q/k/v shapes do not match the cache")
+    if tuple(cos_table.shape) != tuple(sin_table.shape) or cos_table.shape[1] != D // 2:
+        raise ValueError("cos/sin tables must be [max_position, head_dim/2]")
+    _check(lib.pa_rope_write_kv(_ptr(q), _ptr(q_out), _ptr(k), _ptr(v), _ptr(positions), _ptr(cos_table),
+                                _ptr(sin_table), int(cos_table.shape[0]), _ptr(slot_mapping), T, Hq,
+                                _ptr(k_cache), _ptr(v_cache), NB, bs, Hkv, D, _dtype_code(k_cache),
+                                _stream_handle(stream)), "pa_rope_write_kv")
+    return q_out
 
 
 def decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_partitions=0):

@@ -9,6 +9,7 @@
 extern "C" int pa__err_write_kv(unsigned int* out);
 extern "C" int pa__err_decode(unsigned int* out);
 extern "C" int pa__err_prefill(unsigned int* out);
+extern "C" int pa__err_rope(unsigned int* out);
 
 extern "C" const char* pa_strerror(int status) {
   switch (status) {
@@ -30,12 +31,13 @@ extern "C" const char* pa_version(void) { return "0.1.0"; }
 extern "C" int pa_device_error(int* out) {
   if (!out) return PA_ERR_INVALID;
   if (cudaDeviceSynchronize() != cudaSuccess) return PA_ERR_CUDA;
-  unsigned int a = 0, b = 0, c = 0;
+  unsigned int a = 0, b = 0, c = 0, d = 0;
   int s;
   if ((s = pa__err_write_kv(&a)) != PA_OK) return s;
   if ((s = pa__err_decode(&b)) != PA_OK) return s;
   if ((s = pa__err_prefill(&c)) != PA_OK) return s;
-  *out = (int)(a | b | c);
+  if ((s = pa__err_rope(&d)) != PA_OK) return s;
+  *out = (int)(a | b | c | d);
   return PA_OK;
 }
 

@@ -56,6 +56,28 @@ def test_write_kv_validation():
     assert L.pa_write_kv(FAKE, FAKE, FAKE, 0, FAKE, FAKE, 8, 16, 2, 64, 1, NULL) == 0   # no-op, nothing launched
 
 
+def _rope(**kw):
+    a = dict(q=FAKE, qo=FAKE, k=FAKE, v=FAKE, pos=FAKE, cos=FAKE, sin=FAKE, maxpos=64, slots=FAKE, T=4, Hq=8,
+             kc=FAKE, vc=FAKE, NB=8, bs=16, Hkv=2, D=128, dt=1)
+    a.update(kw)
+    return pa.lib.pa_rope_write_kv(a["q"], a["qo"], a["k"], a["v"], a["pos"], a["cos"], a["sin"], a["maxpos"],
+                                   a["slots"], a["T"], a["Hq"], a["kc"], a["vc"], a["NB"], a["bs"], a["Hkv"],
+                                   a["D"], a["dt"], NULL)
+
+
+def test_rope_write_kv_validation():
+    assert _rope(dt=7) == -2 and _rope(D=96) == -2 and _rope(bs=24) == -2
+    assert _rope(T=-1) == -1 and _rope(maxpos=0) == -1 and _rope(Hq=0) == -1 and _rope(NB=-1) == -1
+    for name in ("q", "qo", "k", "v", "pos", "cos", "sin", "slots", "kc", "vc"):
+        assert _rope(**{name: NULL}) == -1, name
+    for name in ("q", "qo", "k", "v", "cos", "sin", "kc", "vc"):
+        assert _rope(**{name: MISALIGNED}) == -3, name
+    assert _rope(pos=ctypes.c_void_p(0x10004)) == -3 and _rope(slots=ctypes.c_void_p(0x10004)) == -3
+    assert _rope(T=0, q=NULL, k=NULL, v=NULL, pos=NULL, slots=NULL) == 0      # no-op: only the caches are checked
+    assert _rope(T=0, kc=MISALIGNED) == -3
+    assert _rope(T=1 << 26) == -2                                               # item count past 2^31
+
+
 def _dec(**kw):
     a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, mb=8, cl=FAKE, B=2, Hq=8, Hkv=2, D=128, bs=16, NB=16, maxL=100,
              scale=0.1, dt=1, ws=FAKE, wsb=1 << 30, ns=0, out=FAKE)

@@ -216,3 +216,76 @@ def make_custom(*, seed: int, lens, num_q_heads: int, num_kv_heads: int, head_di
     return Workload(name="custom", cfg=cfg, ops=ops, free_order=free_order, num_blocks=NB, context_lens=L, q=q,
                     k_new=k_new, v_new=v_new, k_cache0=k_cache0, v_cache0=v_cache0, query_start_loc=qsl,
                     scale=scale)
+
+
+def new_token_positions(wl: Workload) -> np.ndarray:
+    """int64 [T]: the index within its sequence of every token written this step, in the order of the
+    ``append_new`` entries (the row order of k_new/v_new).  Pool-script bookkeeping only."""
+    length: dict[int, int] = {}
+    out = []
+    for op in wl.ops:
+        if op[0] == "alloc":
+            length[op[1]] = op[2]
+        elif op[0] == "fork":
+            length[op[2]] = op[3]
+        elif op[0] == "append":
+            length[op[1]] += op[2]
+        elif op[0] == "append_new":
+            b, n = op[1], op[2]
+            out.extend(range(length[b], length[b] + n))
+            length[b] += n
+    return np.asarray(out, dtype=np.int64)
+
+
+def rope_tables(max_position: int, head_dim: int, base: float = 10000.0):
+    """fp32 cos/sin tables [max_position, head_dim/2] of the usual rotary frequency schedule,
+    angle(p, i) = p * base^(-2i/head_dim), evaluated in float64 and rounded to fp32.  The tables are data
+    handed to the rotary operator (it receives cos and sin, not a schedule)."""
+    inv = base ** (-np.arange(0, head_dim, 2, dtype=np.float64) / head_dim)
+    ang = np.outer(np.arange(max_position, dtype=np.float64), inv)
+    return torch.from_numpy(np.cos(ang).astype(np.float32)), torch.from_numpy(np.sin(ang).astype(np.float32))
+
+
+@dataclasses.dataclass
+class RopeCase:
+    q: torch.Tensor              # [T, Hq, D]
+    k: torch.Tensor              # [T, Hkv, D]
+    v: torch.Tensor
+    positions: torch.Tensor      # int64 [T]
+    cos: torch.Tensor            # fp32 [max_position, D/2]
+    sin: torch.Tensor
+    slots: torch.Tensor          # int64 [T], distinct, -1 = no cache write
+    k_cache0: torch.Tensor       # [NB, bs, Hkv, D]
+    v_cache0: torch.Tensor
+
+
+def make_rope_case(*, seed: int, num_tokens: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                   block_size: int, num_blocks: int, dtype: str = "bf16", max_position: int = 4096,
+                   skip_frac: float = 0.1, random_angles: bool = False) -> RopeCase:
+    """A standalone rotary + cache-write case: N(0,1) q/k/v and caches, positions uniform in
+    [0, max_position) with the first and last table rows always used (when T >= 2), distinct random slots
+    of the pool with a ``skip_frac`` share set to -1.  ``random_angles`` draws every table angle uniformly
+    in [-pi, pi) instead of the frequency schedule."""
+    g = torch.Generator().manual_seed(int(seed))
+    dt = TORCH_DTYPES[dtype]
+    T = int(num_tokens)
+    q = _randn(g, (T, num_q_heads, head_dim), dt)
+    k = _randn(g, (T, num_kv_heads, head_dim), dt)
+    v = _randn(g, (T, num_kv_heads, head_dim), dt)
+    pos = torch.randint(0, max_position, (T,), generator=g, dtype=torch.int64)
+    if T >= 2:
+        pos[0], pos[-1] = 0, max_position - 1
+    nslots = num_blocks * block_size
+    assert T <= nslots
+    slots = torch.randperm(nslots, generator=g)[:T].to(torch.int64)
+    skip = torch.rand(T, generator=g) < skip_frac
+    slots[skip] = -1
+    if random_angles:
+        ang = (torch.rand((max_position, head_dim // 2), generator=g, dtype=torch.float64) * 2 - 1) * math.pi
+        cos, sin = torch.cos(ang).to(torch.float32), torch.sin(ang).to(torch.float32)
+    else:
+        cos, sin = rope_tables(max_position, head_dim)
+    kc = _randn(g, (num_blocks, block_size, num_kv_heads, head_dim), dt)
+    vc = _randn(g, (num_blocks, block_size, num_kv_heads, head_dim), dt)
+    return RopeCase(q=q, k=k, v=v, positions=pos, cos=cos.contiguous(), sin=sin.contiguous(), slots=slots,
+                    k_cache0=kc, v_cache0=vc)
