@@ -48,16 +48,22 @@ WORKLOAD_TEXT = {
     "tiny": "tiny decode: 4 seqs, 4/4 heads, head_dim 64, fp16, block_size 16",
     "prefill": "chunked prefill: 8 seqs, each a 512-token causal chunk appended to an 8192-token paged context, "
                "32 q / 8 kv heads, head_dim 128, bf16, block_size 16",
+    "rope_write": "rotary embedding + KV cache write of the chunked-prefill step's 4096 new tokens (8 seqs x 512 at "
+                  "positions 8192..8703), 32 q / 8 kv heads, head_dim 128, bf16, block_size 16, fp32 cos/sin "
+                  "tables of 16384 positions; before every timed launch L2 is flushed by a 512 MB write followed by a 512 MB "
+                  "read of another buffer (the launch starts on a cold L2 that holds no dirty lines)",
 }
 
 # DRAM bytes (read + write) per launch of the workload's dominant kernel from one ncu capture,
 # valid only for the kernel source it was taken on (sha256 prefix of the listed csrc files).
 DECODE_SRC = ("decode.cu", "common.cuh")
 PREFILL_SRC = ("prefill.cu", "common.cuh")
+ROPE_SRC = ("rope_write_kv.cu", "common.cuh")
 NCU_TRAFFIC = {
     "qwen_decode": {"bytes": 313_465_088, "src": "25100343f6ccb086", "files": DECODE_SRC},
     "llama70b_long": {"bytes": 1_584_901_888, "src": "25100343f6ccb086", "files": DECODE_SRC},
     "prefill": {"bytes": 348_481_024, "src": "0a0c45baf16bf168", "files": PREFILL_SRC},
+    "rope_write": {"bytes": 55_164_160, "src": "9b1a5d7fb8331db7", "files": ROPE_SRC},
 }
 
 
@@ -564,6 +570,139 @@ def run_prefill(args):
     return 0
 
 
+def rope_bytes(T, Hq, Hkv, D, distinct_positions) -> int:
+    """Algorithmic bytes of one rotary + cache-write launch: q read and q_out written, k and v read and their
+    cache rows written (16-bit), the int64 position and slot of every token, and one fp32 cos and sin row
+    (D/2 entries each) per distinct position."""
+    return T * (Hq * D * 2 * 2 + Hkv * D * 2 * 4 + 16) + distinct_positions * D * 4
+
+
+def run_rope(args):
+    """Rotary + KV write step (pa_rope_write_kv) on the chunked-prefill step's new tokens, L2 flushed between
+    timed launches (its ~100 MB working set fits in L2).  The flush is a write of one buffer and a read of
+    another: a write alone would leave L2 full of dirty lines whose write-back the timed launch would pay."""
+    import torch
+    import paged_kv_cache_330_b200 as pa
+    from workloads import make_workload, new_token_positions, rope_tables
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = make_workload("prefill")
+    c = wl.cfg
+    T, Hq, Hkv, D = int(wl.k_new.shape[0]), c["num_q_heads"], c["num_kv_heads"], c["head_dim"]
+    _, bt, lens, sm, _ = pa.replay_ops(wl.ops, wl.num_blocks, c["block_size"], wl.free_order, wl.batch)
+    pos_h = new_token_positions(wl)
+    cos_h, sin_h = rope_tables(16384, D)
+    kc, vc, q = wl.k_cache0.to(dev), wl.v_cache0.to(dev), wl.q.to(dev)
+    kn, vn, smd = wl.k_new.to(dev), wl.v_new.to(dev), torch.from_numpy(sm).to(dev)
+    posd = torch.from_numpy(pos_h).to(dev)
+    cos, sin = cos_h.to(dev), sin_h.to(dev)
+    q_out = torch.empty_like(q)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    scrub = torch.zeros(128 << 20, dtype=torch.float32, device=dev)
+    cs = torch.cuda.Stream(dev)
+    stream = torch.cuda.current_stream(dev)
+    step = lambda st: pa.rope_write_kv(q, kn, vn, posd, cos, sin, smd, kc, vc, q_out=q_out, stream=st)
+    for _ in range(max(3, args.warmup)):
+        step(stream)
+    torch.cuda.synchronize(dev)
+    assert pa.device_error() == 0
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cs):
+            fn()
+        return g
+
+    g_step = capture(lambda: step(cs))
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    with ClockSampler(0) as clk:
+        for i in range(K):
+            flush.fill_(i & 0xFF)          # evict q/k/v and the cache rows from L2 (not timed) ...
+            scrub.sum()                    # ... and write the flush's dirty lines back before the launch
+            ev[i][0].record(stream)
+            g_step.replay()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    assert pa.device_error() == 0
+    times = sorted(a.elapsed_time(b) for a, b in ev)
+    ms = float(np.mean(times))
+    nbytes = rope_bytes(T, Hq, Hkv, D, len(np.unique(pos_h)))
+    gbs = nbytes / (ms * 1e-3) / 1e9
+
+    # ---- end to end through the public API: pinned host q/k/v/positions/slots -> device, step, q_out -> host
+    pin = lambda t: t.pin_memory()
+    h_q, h_kn, h_vn, h_sm, h_pos = pin(wl.q), pin(wl.k_new), pin(wl.v_new), pin(torch.from_numpy(sm)), \
+        pin(torch.from_numpy(pos_h))
+    h_out = torch.empty(q_out.shape, dtype=q_out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_kn, h_vn, h_sm, h_pos))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step(st):
+        for dst, src in ((q, h_q), (kn, h_kn), (vn, h_vn), (smd, h_sm), (posd, h_pos)):
+            dst.copy_(src, non_blocking=True)
+        step(st)
+        h_out.copy_(q_out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step(stream)
+    torch.cuda.synchronize(dev)
+    g_e2e = capture(lambda: e2e_step(cs))
+    g_e2e.replay()
+    torch.cuda.synchronize(dev)
+    e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e4.record(stream)
+    for _ in range(K):
+        g_e2e.replay()
+    e5.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e4.elapsed_time(e5) / K
+    assert pa.device_error() == 0
+    del g_step, g_e2e
+
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        from oracle import rope as orope
+        try:
+            from threadpoolctl import threadpool_info
+            threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        except Exception:
+            threads = 1
+        _, _, _, oslots, _ = oracle.replay(wl.ops, wl.num_blocks, c["block_size"], wl.free_order, wl.batch)
+        vcb = wl.v_cache0.view(torch.int16).numpy().view(np.uint16).copy()
+        vb = wl.v_new.view(torch.int16).numpy().view(np.uint16)
+        qd, kd = wl.q.double().numpy(), wl.k_new.double().numpy()
+        reps, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < 10.0:
+            orope.rope_write_kv(qd, kd, vb, pos_h, cos_h.numpy(), sin_h.numpy(), oslots, vcb)
+            reps += 1
+        el = time.perf_counter() - t0
+        cpu = {"value": nbytes * reps / el / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"oracle (numpy fp64 rotation + byte write of V) on the whole {T}-token step, {reps} "
+                         f"repetitions in {el:.1f} s; GB/s counts the same algorithmic bytes"}
+    tr = NCU_TRAFFIC.get("rope_write")
+    traffic = tr["bytes"] if tr and tr["src"] == kernel_source_hash(tr["files"]) else None
+    peak, kind = measured_hbm_peak()
+    line = {
+        "metric": "rotary embedding + KV cache write GB/s (% of HBM peak)", "value": gbs, "unit": "GB/s",
+        "n_gpus": 1, "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": str(c["dtype"]), "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT["rope_write"], "bytes_per_step": nbytes, "l2": "flushed"},
+        "roofline": {"bound": "hbm", "kernel": "pa_rope_write_kv", "achieved": gbs, "peak": peak,
+                     "peak_kind": kind, "unit": "GB/s", "frac": gbs / peak, "traffic": traffic,
+                     "avg_launch_ms": ms, "median_launch_ms": times[len(times) // 2]},
+        "e2e": {"value": nbytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "cpu_baseline": cpu,
+        "gpu_launches": K,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -583,6 +722,8 @@ def main():
         return run_reference(args)
     if args.workload == "prefill":
         return run_prefill(args)
+    if args.workload == "rope_write":
+        return run_rope(args)
     return run_ours(args)
 
 
