@@ -36,6 +36,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "paged decode KV GB/s (% of HBM peak) and decode tokens/s at batch 128"
 UNIT = "GB/s"
+PREFILL_METRIC = "chunked prefill TFLOP/s (bf16, causal, paged context)"
+ROPE_METRIC = "rotary embedding + KV cache write GB/s (% of HBM peak)"
 FALLBACK_HBM_GBS = 6650.0
 
 WORKLOAD_TEXT = {
@@ -236,29 +238,108 @@ def time_oracle(wl, budget_s: float, n_seqs: int):
     return gbs, desc, threads, el / reps
 
 
+def _oracle_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return 1
+
+
+def time_oracle_prefill(wl, budget_s: float):
+    """Oracle chunked prefill (pool replay, byte write of the chunk, fp64 causal attention) over
+    (sequence, head) pairs in order until budget_s; returns (TFLOP/s, desc, threads, seconds of the sample)."""
+    import oracle
+    from oracle import attention as oatt
+    import torch
+    t0 = time.perf_counter()
+    _, rows, lens, slots, _ = oracle.replay(wl.ops, wl.num_blocks, wl.cfg["block_size"], wl.free_order, wl.batch)
+    kc = wl.k_cache0.view(torch.int16).numpy().view(np.uint16).copy()
+    vc = wl.v_cache0.view(torch.int16).numpy().view(np.uint16).copy()
+    oracle.write_kv(wl.k_new.view(torch.int16).numpy().view(np.uint16),
+                    wl.v_new.view(torch.int16).numpy().view(np.uint16), slots, kc, vc)
+    dt = wl.k_cache0.dtype
+    kt, vt = torch.from_numpy(kc.view(np.int16)).view(dt), torch.from_numpy(vc.view(np.int16)).view(dt)
+    D, Hq = wl.cfg["head_dim"], wl.cfg["num_q_heads"]
+    flops, pairs = 0.0, 0
+    for b in range(wl.batch):
+        C = int(wl.query_start_loc[b + 1] - wl.query_start_loc[b])
+        L = int(wl.context_lens[b])
+        for h in range(Hq):
+            oatt.prefill_attention(wl.q, wl.query_start_loc, kt, vt, rows, lens, wl.scale, seqs=[b], heads=[h])
+            flops += (C * (L - C) + C * (C + 1) // 2) * 4.0 * D
+            pairs += 1
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    el = time.perf_counter() - t0
+    desc = (f"oracle (numpy fp64: pool replay, byte write of the chunk, causal attention) on the first {pairs} of "
+            f"{wl.batch * Hq} (sequence, head) pairs of {wl.name} in {el:.1f} s; TFLOP/s counts those pairs' flops")
+    return flops / el / 1e12, desc, _oracle_threads(), el
+
+
+def time_oracle_rope(wl, budget_s: float):
+    """Oracle rotary + cache write of the prefill step's new tokens, repeated until budget_s; returns
+    (GB/s of the same algorithmic bytes as the GPU line, desc, threads, seconds per step)."""
+    import oracle
+    from oracle import rope as orope
+    from workloads import new_token_positions, rope_tables
+    import torch
+    c = wl.cfg
+    pos = new_token_positions(wl)
+    cos, sin = rope_tables(16384, c["head_dim"])
+    _, _, _, slots, _ = oracle.replay(wl.ops, wl.num_blocks, c["block_size"], wl.free_order, wl.batch)
+    vcb = wl.v_cache0.view(torch.int16).numpy().view(np.uint16).copy()
+    vb = wl.v_new.view(torch.int16).numpy().view(np.uint16)
+    qd, kd = wl.q.double().numpy(), wl.k_new.double().numpy()
+    nbytes = rope_bytes(int(pos.shape[0]), c["num_q_heads"], c["num_kv_heads"], c["head_dim"], len(np.unique(pos)))
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        orope.rope_write_kv(qd, kd, vb, pos, cos.numpy(), sin.numpy(), slots, vcb)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    el = time.perf_counter() - t0
+    desc = (f"oracle (numpy fp64 rotation + byte write of V) on the whole {pos.shape[0]}-token step, {reps} "
+            f"repetitions in {el:.1f} s; GB/s counts the same algorithmic bytes")
+    return nbytes * reps / el / 1e9, desc, _oracle_threads(), el / reps
+
+
 def run_reference(args):
     ws, rank, _ = dist_setup()
     if rank != 0:
         return 0
     from workloads import make_workload
-    wl = make_workload(args.workload)
-    n = min(wl.batch, args.ref_seqs)
+    wname = "prefill" if args.workload == "rope_write" else args.workload
+    wl = make_workload(wname)
+    metric, unit, sample = METRIC, UNIT, {}
+    if args.workload == "prefill":
+        metric, unit = PREFILL_METRIC, "TFLOP/s"
+        sample_fn = lambda: time_oracle_prefill(wl, args.ref_budget)
+    elif args.workload == "rope_write":
+        metric = ROPE_METRIC
+        sample_fn = lambda: time_oracle_rope(wl, args.ref_budget)
+    else:
+        n = min(wl.batch, args.ref_seqs)
+        sample = {"sample_seqs": n}
+        sample_fn = lambda: time_oracle(wl, args.ref_budget, n)
     step_times = []
-    gbs_all = []
+    vals = []
     desc = threads = None
     for i in range(args.warmup + args.steps):
-        gbs, desc, threads, per = time_oracle(wl, args.ref_budget, n)
+        v, desc, threads, per = sample_fn()
         if i >= args.warmup:
             step_times.append(per)
-            gbs_all.append(gbs)
-    value = float(np.mean(gbs_all))
+            vals.append(v)
+    value = float(np.mean(vals))
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * float(np.mean(step_times)), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD_TEXT.get(args.workload, args.workload), "sample_seqs": n},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
-        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "config": {"workload": WORKLOAD_TEXT.get(args.workload, args.workload), **sample},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -548,11 +629,15 @@ def run_prefill(args):
     assert pa.device_error() == 0
     del g_step, g_pf, g_e2e
     fl = prefill_flops(wl)
+    cpu = None
+    if not args.no_cpu_baseline:
+        v, desc, threads, _ = time_oracle_prefill(wl, 10.0)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
     tr = NCU_TRAFFIC["prefill"]
     pf_traffic = tr["bytes"] if tr["src"] == kernel_source_hash(tr["files"]) else None
     burst, sustained, kind = measured_bf16_peak()
     line = {
-        "metric": "chunked prefill TFLOP/s (bf16, causal, paged context)", "value": fl / (ms_step * 1e-3) / 1e12,
+        "metric": PREFILL_METRIC, "value": fl / (ms_step * 1e-3) / 1e12,
         "unit": "TFLOP/s", "n_gpus": 1, "steps": K, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": str(c["dtype"]),
         "data": "synthetic", "config": {"workload": WORKLOAD_TEXT["prefill"], "flops_per_step": fl},
@@ -563,6 +648,7 @@ def run_prefill(args):
                      "avg_launch_ms": ms_pf},
         "e2e": {"value": fl / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "cpu_baseline": cpu,
         "gpu_launches": 2 * K,
         "clocks": clk.summary(),
     }
@@ -663,30 +749,13 @@ def run_rope(args):
 
     cpu = None
     if not args.no_cpu_baseline:
-        import oracle
-        from oracle import rope as orope
-        try:
-            from threadpoolctl import threadpool_info
-            threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-        except Exception:
-            threads = 1
-        _, _, _, oslots, _ = oracle.replay(wl.ops, wl.num_blocks, c["block_size"], wl.free_order, wl.batch)
-        vcb = wl.v_cache0.view(torch.int16).numpy().view(np.uint16).copy()
-        vb = wl.v_new.view(torch.int16).numpy().view(np.uint16)
-        qd, kd = wl.q.double().numpy(), wl.k_new.double().numpy()
-        reps, t0 = 0, time.perf_counter()
-        while time.perf_counter() - t0 < 10.0:
-            orope.rope_write_kv(qd, kd, vb, pos_h, cos_h.numpy(), sin_h.numpy(), oslots, vcb)
-            reps += 1
-        el = time.perf_counter() - t0
-        cpu = {"value": nbytes * reps / el / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-               "sample": f"oracle (numpy fp64 rotation + byte write of V) on the whole {T}-token step, {reps} "
-                         f"repetitions in {el:.1f} s; GB/s counts the same algorithmic bytes"}
+        v, desc, threads, _ = time_oracle_rope(wl, 10.0)
+        cpu = {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc}
     tr = NCU_TRAFFIC.get("rope_write")
     traffic = tr["bytes"] if tr and tr["src"] == kernel_source_hash(tr["files"]) else None
     peak, kind = measured_hbm_peak()
     line = {
-        "metric": "rotary embedding + KV cache write GB/s (% of HBM peak)", "value": gbs, "unit": "GB/s",
+        "metric": ROPE_METRIC, "value": gbs, "unit": "GB/s",
         "n_gpus": 1, "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": str(c["dtype"]), "data": "synthetic",
         "config": {"workload": WORKLOAD_TEXT["rope_write"], "bytes_per_step": nbytes, "l2": "flushed"},

@@ -87,3 +87,27 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
 
     assert bench.run_reference(Args()) == 0
     assert capsys.readouterr().out == ""
+
+
+@pytest.mark.parametrize("workload,metric_attr,unit", [("tiny", "METRIC", "GB/s"), ("prefill", "PREFILL_METRIC", "TFLOP/s"),
+                                                        ("rope_write", "ROPE_METRIC", "GB/s")])
+def test_reference_arm_times_the_matching_oracle(monkeypatch, capsys, workload, metric_attr, unit):
+    """`--impl reference` times the oracle of the same workload, on the metric and unit of our arm's line."""
+    import json
+    bench = _load_bench()
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+
+    class Args:
+        ref_seqs = 4
+        ref_budget = 0.2
+        steps = 1
+        warmup = 0
+        gpus = 1
+
+    Args.workload = workload
+    assert bench.run_reference(Args()) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == getattr(bench, metric_attr) and line["unit"] == unit
+    assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["unit"] == unit
+    assert line["e2e"] == {"value": line["value"], "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
