@@ -20,20 +20,26 @@ source pages, in float64 with numpy:
   vLLM-Ascend page, section 3.1, moves softmax out of fp16 for accuracy); causal
   chunked prefill over the paged context (vllm-ascend page, section 1.1, PCP).
 * ``brute``       - a scalar pure-Python twin of ``attention`` for tiny cases.
+* ``kv_quant``    - INT8 KV cache (Nano-vLLM-Ascend page, section 4.3; vLLM-Ascend
+  page, section 5): per-(token, KV head) symmetric absmax codes with an fp32
+  scale, written on append and dequantised for attention.
 * ``rope``        - rotary position embedding of new tokens' queries and keys
   fused with the KV write (Nano-vLLM-Ascend page, sections 3.1 and 5.1: the
   rotary multiply by per-position cos/sin tables, inverted by negating sin).
 
-Parity pins (tests/test_oracle_pins.py, tests/test_oracle_rope.py): the pages' worked block arithmetic
+Parity pins (tests/test_oracle_pins.py, tests/test_oracle_rope.py,
+tests/test_oracle_kv_quant.py): the pages' worked block arithmetic
 (tests/golden/), closed forms, torch's float64 scaled_dot_product_attention on
 dense inputs, the scalar twin, and invariants (block permutation, prefix
 sharing, prefill row i == decode of the first prefix+i+1 tokens); for the
 rotary step, rotation closed forms, the page's inverse rule, angle addition,
-the relative-position property and torch complex multiplication.  No function
+the relative-position property and torch complex multiplication; for the
+INT8 cache, the absmax code, the half-step error bound, exact grid rows and
+torch's int8 quantiser.  No function
 here is "parity unpinned".
 """
 
-from . import attention, block_pool, brute, kv_write, rope  # noqa: F401
+from . import attention, block_pool, brute, kv_quant, kv_write, rope  # noqa: F401
 from .attention import decode_attention, gather_kv, prefill_attention, split_partials  # noqa: F401
 from .block_pool import OraclePool, replay  # noqa: F401
 from .kv_write import write_kv  # noqa: F401
