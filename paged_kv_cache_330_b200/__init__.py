@@ -129,18 +129,69 @@ def _stream_handle(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _want(name, t, dtype=None, shape=None, ndim=None):
+    """Host-side check of one tensor argument's dtype / shape (None: not checked)."""
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got shape {tuple(t.shape)}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _caches(k_cache, v_cache):
+    """Both caches [num_blocks, block_size, Hkv, D], same shape and 16-bit dtype; returns the shape."""
+    _want("k_cache", k_cache, ndim=4)
+    _want("v_cache", v_cache, dtype=k_cache.dtype, shape=k_cache.shape)
+    _dtype_code(k_cache)
+    return tuple(int(x) for x in k_cache.shape)
+
+
+def _device(stream, *tensors):
+    """Every tensor argument must live on the current CUDA device (a host pointer, or another device's memory,
+    must never reach a kernel), and a given stream must belong to that device.  Checked after the dtype and
+    shape checks, before anything is launched."""
+    torch = _torch()
+    dev = None
+    for t in tensors:
+        if t is None:
+            continue
+        if t.device.type != "cuda":
+            raise ValueError(f"device calls take CUDA tensors; got a tensor on {t.device}")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"tensor arguments on {dev} and {t.device}")
+    if dev is not None:
+        if dev.index != torch.cuda.current_device():
+            raise ValueError(f"tensors are on {dev} but the current device is cuda:{torch.cuda.current_device()}")
+        if stream is not None and stream.device != dev:
+            raise ValueError(f"stream belongs to {stream.device}, tensors to {dev}")
+    return dev
+
+
 def write_kv(k, v, slot_mapping, k_cache, v_cache, stream=None) -> None:
     """k, v [T, Hkv, D]; slot_mapping int64 [T] (-1 = skip); caches [NB, bs, Hkv, D]."""
+    torch = _torch()
     _contig(k, v, slot_mapping, k_cache, v_cache)
-    NB, bs, Hkv, D = k_cache.shape
+    NB, bs, Hkv, D = _caches(k_cache, v_cache)
+    T = int(k.shape[0]) if k.dim() > 0 else -1
+    _want("k", k, dtype=k_cache.dtype, shape=(T, Hkv, D))
+    _want("v", v, dtype=k_cache.dtype, shape=(T, Hkv, D))
+    _want("slot_mapping", slot_mapping, dtype=torch.int64, shape=(T,))
+    _device(stream, k, v, slot_mapping, k_cache, v_cache)
     _check(lib.pa_write_kv(_ptr(k), _ptr(v), _ptr(slot_mapping), int(k.shape[0]), _ptr(k_cache), _ptr(v_cache),
                            NB, bs, Hkv, D, _dtype_code(k_cache), _stream_handle(stream)), "pa_write_kv")
 
 
 def copy_blocks(pairs, k_cache, v_cache, stream=None) -> None:
     """pairs int32 [n, 2] (src, dst) on the device."""
+    torch = _torch()
     _contig(pairs, k_cache, v_cache)
-    NB, bs, Hkv, D = k_cache.shape
+    NB, bs, Hkv, D = _caches(k_cache, v_cache)
+    _want("pairs", pairs, dtype=torch.int32, ndim=2)
+    _want("pairs", pairs, shape=(pairs.shape[0], 2))
+    _device(stream, pairs, k_cache, v_cache)
     _check(lib.pa_copy_blocks(_ptr(pairs), int(pairs.shape[0]), _ptr(k_cache), _ptr(v_cache), NB, bs, Hkv, D,
                               _dtype_code(k_cache), _stream_handle(stream)), "pa_copy_blocks")
 
@@ -159,12 +210,18 @@ def rope_write_kv(q, k, v, positions, cos_table, sin_table, slot_mapping, k_cach
         raise ValueError("cos/sin tables must be float32")
     if q_out.shape != q.shape or q_out.dtype != q.dtype:
         raise ValueError("q_out must match q")
-    NB, bs, Hkv, D = k_cache.shape
+    NB, bs, Hkv, D = _caches(k_cache, v_cache)
+    _want("q", q, dtype=k_cache.dtype, ndim=3)
     T, Hq = int(q.shape[0]), int(q.shape[1])
     if tuple(k.shape) != (T, Hkv, D) or tuple(v.shape) != (T, Hkv, D) or q.shape[2] != D:
         raise ValueError("q/k/v shapes do not match the cache")
-    if tuple(cos_table.shape) != tuple(sin_table.shape) or cos_table.shape[1] != D // 2:
+    _want("k", k, dtype=k_cache.dtype)
+    _want("v", v, dtype=k_cache.dtype)
+    _want("positions", positions, dtype=torch.int64, shape=(T,))
+    _want("slot_mapping", slot_mapping, dtype=torch.int64, shape=(T,))
+    if cos_table.dim() != 2 or tuple(cos_table.shape) != tuple(sin_table.shape) or cos_table.shape[1] != D // 2:
         raise ValueError("cos/sin tables must be [max_position, head_dim/2]")
+    _device(stream, q, q_out, k, v, positions, cos_table, sin_table, slot_mapping, k_cache, v_cache)
     _check(lib.pa_rope_write_kv(_ptr(q), _ptr(q_out), _ptr(k), _ptr(v), _ptr(positions), _ptr(cos_table),
                                 _ptr(sin_table), int(cos_table.shape[0]), _ptr(slot_mapping), T, Hq,
                                 _ptr(k_cache), _ptr(v_cache), NB, bs, Hkv, D, _dtype_code(k_cache),
@@ -180,13 +237,30 @@ def decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num
     return gr.value, mp.value, ws.value
 
 
+def _decode_args(q, k_cache, v_cache, block_tables, context_lens, out):
+    """Shapes and dtypes of a decode call: q [B, Hq, D] in the caches' dtype, block_tables int32 [B, n],
+    context_lens int32 [B], out (if given) like q.  Returns (B, Hq, D)."""
+    torch = _torch()
+    _, _, _, D = _caches(k_cache, v_cache)
+    _want("q", q, dtype=k_cache.dtype, ndim=3)
+    B, Hq = int(q.shape[0]), int(q.shape[1])
+    _want("q", q, shape=(B, Hq, D))
+    _want("block_tables", block_tables, dtype=torch.int32, ndim=2)
+    _want("block_tables", block_tables, shape=(B, block_tables.shape[1]))
+    _want("context_lens", context_lens, dtype=torch.int32, shape=(B,))
+    if out is not None:
+        _want("out", out, dtype=q.dtype, shape=q.shape)
+    return B, Hq, D
+
+
 def decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float, out=None,
            workspace=None, num_partitions: int = 0, stream=None):
     """q [B, Hq, D]; block_tables int32 [B, max_blocks]; context_lens int32 [B]. Returns out [B, Hq, D]."""
     torch = _torch()
     _contig(q, k_cache, v_cache, block_tables, context_lens, out, workspace)
-    B, Hq, D = q.shape
+    B, Hq, D = _decode_args(q, k_cache, v_cache, block_tables, context_lens, out)
     NB, bs, Hkv, _ = k_cache.shape
+    _device(stream, q, k_cache, v_cache, block_tables, context_lens, out, workspace)
     if out is None:
         out = torch.empty_like(q)
     _, _, need = decode_plan(B, Hq, Hkv, D, max_context_len, num_partitions)
@@ -206,8 +280,9 @@ def decode_static_scratch(q, k_cache, v_cache, block_tables, context_lens, max_c
     that must not allocate where they run decode).  Calls overlapping on the GPU race on that scratch."""
     torch = _torch()
     _contig(q, k_cache, v_cache, block_tables, context_lens, out)
-    B, Hq, D = q.shape
+    B, Hq, D = _decode_args(q, k_cache, v_cache, block_tables, context_lens, out)
     NB, bs, Hkv, _ = k_cache.shape
+    _device(stream, q, k_cache, v_cache, block_tables, context_lens, out)
     if out is None:
         out = torch.empty_like(q)
     _check(lib.pa_decode_static_scratch(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
@@ -222,9 +297,18 @@ def prefill_chunk(q, query_start_loc, k_cache, v_cache, block_tables, context_le
     """q [sum C, Hq, D]; query_start_loc int32 [B+1]; returns out [sum C, Hq, D]."""
     torch = _torch()
     _contig(q, query_start_loc, k_cache, v_cache, block_tables, context_lens, out)
-    T, Hq, D = q.shape
-    NB, bs, Hkv, _ = k_cache.shape
+    NB, bs, Hkv, D = _caches(k_cache, v_cache)
+    _want("q", q, dtype=k_cache.dtype, ndim=3)
+    T, Hq = int(q.shape[0]), int(q.shape[1])
+    _want("q", q, shape=(T, Hq, D))
+    _want("context_lens", context_lens, dtype=torch.int32, ndim=1)
     B = int(context_lens.shape[0])
+    _want("query_start_loc", query_start_loc, dtype=torch.int32, shape=(B + 1,))
+    _want("block_tables", block_tables, dtype=torch.int32, ndim=2)
+    _want("block_tables", block_tables, shape=(B, block_tables.shape[1]))
+    if out is not None:
+        _want("out", out, dtype=q.dtype, shape=q.shape)
+    _device(stream, q, query_start_loc, k_cache, v_cache, block_tables, context_lens, out)
     if out is None:
         out = torch.empty_like(q)
     _check(lib.pa_prefill_chunk(_ptr(q), _ptr(query_start_loc), T, int(max_chunk_len), _ptr(k_cache), _ptr(v_cache),
