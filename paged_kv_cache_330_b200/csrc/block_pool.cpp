@@ -10,18 +10,34 @@
 // caller's device tensors.  Every operation checks first and mutates second,
 // so a failed call leaves the pool unchanged.
 
-#include <algorithm>
 #include <cstdint>
-#include <deque>
 #include <unordered_map>
 #include <vector>
 
 #include "paged_attn.h"
 
+// The free list is a ring of num_blocks entries allocated once at creation: a block is in it at most once,
+// so handing blocks out and taking them back never allocates, and an operation cannot fail half-way.
+struct FreeRing {
+  std::vector<int32_t> slot;
+  size_t head = 0, count = 0;
+  size_t size() const { return count; }
+  int32_t pop_front() {
+    const int32_t b = slot[head];
+    head = (head + 1) % slot.size();
+    --count;
+    return b;
+  }
+  void push_back(int32_t b) {
+    slot[(head + count) % slot.size()] = b;
+    ++count;
+  }
+};
+
 struct pa_pool {
   int num_blocks = 0;
   int block_size = 0;
-  std::deque<int32_t> free_list;        // head = next block handed out
+  FreeRing free_list;                   // head = next block handed out
   std::vector<int32_t> ref;             // reference count per physical block
   struct Seq {
     std::vector<int32_t> blocks;        // logical block j -> physical block
@@ -30,8 +46,7 @@ struct pa_pool {
   std::unordered_map<int64_t, Seq> seqs;
 
   int32_t take() {
-    int32_t b = free_list.front();
-    free_list.pop_front();
+    const int32_t b = free_list.pop_front();
     ref[b] = 1;
     return b;
   }
@@ -39,87 +54,110 @@ struct pa_pool {
 
 static inline int64_t blocks_for(int64_t n, int bs) { return (n + bs - 1) / bs; }
 
+// Every call below does all of its allocation before it changes the pool, and no exception leaves the C
+// ABI: an allocation failure is reported as PA_ERR_OOM (NULL from pa_pool_create) with the pool unchanged.
+
 extern "C" pa_pool* pa_pool_create(int num_blocks, int block_size, const int32_t* free_order) {
   if (num_blocks < 0 || block_size <= 0) return nullptr;
-  pa_pool* p = new pa_pool;
-  p->num_blocks = num_blocks;
-  p->block_size = block_size;
-  p->ref.assign(num_blocks, 0);
-  if (free_order) {
-    std::vector<char> seen(num_blocks, 0);
-    for (int i = 0; i < num_blocks; ++i) {
-      int32_t b = free_order[i];
-      if (b < 0 || b >= num_blocks || seen[b]) {
-        delete p;
-        return nullptr;
+  pa_pool* p = nullptr;
+  try {
+    p = new pa_pool;
+    p->num_blocks = num_blocks;
+    p->block_size = block_size;
+    p->ref.assign(num_blocks, 0);
+    p->free_list.slot.assign(num_blocks, 0);
+    if (free_order) {
+      std::vector<char> seen(num_blocks, 0);
+      for (int i = 0; i < num_blocks; ++i) {
+        const int32_t b = free_order[i];
+        if (b < 0 || b >= num_blocks || seen[b]) {
+          delete p;
+          return nullptr;
+        }
+        seen[b] = 1;
+        p->free_list.push_back(b);
       }
-      seen[b] = 1;
-      p->free_list.push_back(b);
+    } else {
+      for (int i = 0; i < num_blocks; ++i) p->free_list.push_back(i);
     }
-  } else {
-    for (int i = 0; i < num_blocks; ++i) p->free_list.push_back(i);
+    return p;
+  } catch (...) {
+    delete p;
+    return nullptr;
   }
-  return p;
 }
 
 extern "C" void pa_pool_destroy(pa_pool* pool) { delete pool; }
 
 extern "C" int pa_seq_alloc(pa_pool* pool, int64_t seq_id, int num_tokens) {
   if (!pool || num_tokens < 0) return PA_ERR_INVALID;
-  if (pool->seqs.count(seq_id)) return PA_ERR_NOT_FOUND;
-  int64_t need = blocks_for(num_tokens, pool->block_size);
-  if (need > (int64_t)pool->free_list.size()) return PA_ERR_OOM;
-  pa_pool::Seq s;
-  s.blocks.reserve(need);
-  for (int64_t i = 0; i < need; ++i) s.blocks.push_back(pool->take());
-  s.len = num_tokens;
-  pool->seqs.emplace(seq_id, std::move(s));
-  return PA_OK;
+  try {
+    if (pool->seqs.count(seq_id)) return PA_ERR_NOT_FOUND;
+    const int64_t need = blocks_for(num_tokens, pool->block_size);
+    if (need > (int64_t)pool->free_list.size()) return PA_ERR_OOM;
+    pa_pool::Seq s;
+    s.blocks.reserve(need);
+    s.len = num_tokens;
+    pa_pool::Seq& in = pool->seqs.emplace(seq_id, std::move(s)).first->second;
+    for (int64_t i = 0; i < need; ++i) in.blocks.push_back(pool->take());  // within capacity: no allocation
+    return PA_OK;
+  } catch (...) {
+    return PA_ERR_OOM;
+  }
 }
 
 extern "C" int pa_seq_fork(pa_pool* pool, int64_t parent_id, int64_t child_id, int n_prefix) {
   if (!pool || n_prefix < 0) return PA_ERR_INVALID;
-  auto it = pool->seqs.find(parent_id);
-  if (it == pool->seqs.end() || pool->seqs.count(child_id)) return PA_ERR_NOT_FOUND;
-  if (n_prefix > it->second.len) return PA_ERR_INVALID;
-  pa_pool::Seq c;
-  int64_t nb = blocks_for(n_prefix, pool->block_size);
-  c.blocks.assign(it->second.blocks.begin(), it->second.blocks.begin() + nb);
-  for (int32_t b : c.blocks) pool->ref[b] += 1;
-  c.len = n_prefix;
-  pool->seqs.emplace(child_id, std::move(c));
-  return PA_OK;
+  try {
+    auto it = pool->seqs.find(parent_id);
+    if (it == pool->seqs.end() || pool->seqs.count(child_id)) return PA_ERR_NOT_FOUND;
+    if (n_prefix > it->second.len) return PA_ERR_INVALID;
+    pa_pool::Seq c;
+    const int64_t nb = blocks_for(n_prefix, pool->block_size);
+    c.blocks.assign(it->second.blocks.begin(), it->second.blocks.begin() + nb);
+    c.len = n_prefix;
+    const pa_pool::Seq& in = pool->seqs.emplace(child_id, std::move(c)).first->second;
+    for (int32_t b : in.blocks) pool->ref[b] += 1;
+    return PA_OK;
+  } catch (...) {
+    return PA_ERR_OOM;
+  }
 }
 
 extern "C" int pa_seq_append(pa_pool* pool, int64_t seq_id, int n, int64_t* slot_mapping_out,
                              int32_t* cow_pairs_out, int* num_cow_out) {
   if (!pool || n < 0) return PA_ERR_INVALID;
-  auto it = pool->seqs.find(seq_id);
-  if (it == pool->seqs.end()) return PA_ERR_NOT_FOUND;
-  pa_pool::Seq& s = it->second;
-  const int bs = pool->block_size;
-  const int64_t n0 = s.len;
-  const bool cow = n > 0 && (n0 % bs) != 0 && pool->ref[s.blocks.back()] > 1;
-  int64_t need = blocks_for(n0 + n, bs) - (int64_t)s.blocks.size() + (cow ? 1 : 0);
-  if (need > (int64_t)pool->free_list.size()) return PA_ERR_OOM;
-  if (num_cow_out) *num_cow_out = 0;
-  if (cow) {
-    int32_t old_b = s.blocks.back();
-    int32_t new_b = pool->take();
-    pool->ref[old_b] -= 1;
-    s.blocks.back() = new_b;
-    if (cow_pairs_out) {
-      cow_pairs_out[0] = old_b;
-      cow_pairs_out[1] = new_b;
+  try {
+    auto it = pool->seqs.find(seq_id);
+    if (it == pool->seqs.end()) return PA_ERR_NOT_FOUND;
+    pa_pool::Seq& s = it->second;
+    const int bs = pool->block_size;
+    const int64_t n0 = s.len;
+    const bool cow = n > 0 && (n0 % bs) != 0 && pool->ref[s.blocks.back()] > 1;
+    const int64_t need = blocks_for(n0 + n, bs) - (int64_t)s.blocks.size() + (cow ? 1 : 0);
+    if (need > (int64_t)pool->free_list.size()) return PA_ERR_OOM;
+    s.blocks.reserve(blocks_for(n0 + n, bs));
+    if (num_cow_out) *num_cow_out = 0;
+    if (cow) {
+      const int32_t old_b = s.blocks.back();
+      const int32_t new_b = pool->take();
+      pool->ref[old_b] -= 1;
+      s.blocks.back() = new_b;
+      if (cow_pairs_out) {
+        cow_pairs_out[0] = old_b;
+        cow_pairs_out[1] = new_b;
+      }
+      if (num_cow_out) *num_cow_out = 1;
     }
-    if (num_cow_out) *num_cow_out = 1;
+    for (int64_t p = n0; p < n0 + n; ++p) {
+      if (p % bs == 0) s.blocks.push_back(pool->take());  // within capacity: no allocation
+      if (slot_mapping_out) slot_mapping_out[p - n0] = (int64_t)s.blocks[p / bs] * bs + p % bs;
+    }
+    s.len = n0 + n;
+    return PA_OK;
+  } catch (...) {
+    return PA_ERR_OOM;
   }
-  for (int64_t p = n0; p < n0 + n; ++p) {
-    if (p % bs == 0) s.blocks.push_back(pool->take());
-    if (slot_mapping_out) slot_mapping_out[p - n0] = (int64_t)s.blocks[p / bs] * bs + p % bs;
-  }
-  s.len = n0 + n;
-  return PA_OK;
 }
 
 extern "C" int pa_seq_free(pa_pool* pool, int64_t seq_id) {
@@ -128,7 +166,7 @@ extern "C" int pa_seq_free(pa_pool* pool, int64_t seq_id) {
   if (it == pool->seqs.end()) return PA_ERR_NOT_FOUND;
   for (int32_t b : it->second.blocks) {
     pool->ref[b] -= 1;
-    if (pool->ref[b] == 0) pool->free_list.push_back(b);
+    if (pool->ref[b] == 0) pool->free_list.push_back(b);  // the ring has room for every block
   }
   pool->seqs.erase(it);
   return PA_OK;
