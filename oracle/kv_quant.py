@@ -58,8 +58,10 @@ def write_kv_int8(k_new, v_new, slot_mapping, k_codes: np.ndarray, v_codes: np.n
                   k_scales: np.ndarray, v_scales: np.ndarray) -> None:
     """In place: quantise each new token's K and V rows (per KV head) into the INT8 caches.
 
-    k_new/v_new [T, Hkv, D] (16-bit values as float32); code caches int8 [NB, bs, Hkv, D]; scale caches
-    float32 [NB, bs, Hkv].  Slot s is block s // bs, row s % bs; a slot of -1 writes nothing."""
+    k_new/v_new [T, Hkv, D] (16-bit values as float32); code caches int8 [NB, bs, Hkv, D], laid out like
+    the 16-bit caches; scale caches float32 [NB, Hkv, bs], so that the scales of consecutive tokens of one
+    head are contiguous (a 16-token chunk's scales are one 64-byte run).  Slot s is block s // bs, row
+    s % bs; a slot of -1 writes nothing."""
     bs = k_codes.shape[1]
     kq, ks = quantize_rows(k_new)
     vq, vs = quantize_rows(v_new)
@@ -70,10 +72,10 @@ def write_kv_int8(k_new, v_new, slot_mapping, k_codes: np.ndarray, v_codes: np.n
         blk, row = slot // bs, slot % bs
         k_codes[blk, row] = kq[t]
         v_codes[blk, row] = vq[t]
-        k_scales[blk, row] = ks[t]
-        v_scales[blk, row] = vs[t]
+        k_scales[blk, :, row] = ks[t]
+        v_scales[blk, :, row] = vs[t]
 
 
 def dequantized_cache(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
-    """The float64 cache [NB, bs, Hkv, D] that attention over the INT8 cache reads."""
-    return dequantize_rows(codes, scales)
+    """The float64 cache [NB, bs, Hkv, D] that attention over the INT8 cache reads (scales [NB, Hkv, bs])."""
+    return dequantize_rows(codes, np.transpose(scales, (0, 2, 1)))

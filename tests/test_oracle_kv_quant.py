@@ -89,15 +89,17 @@ def check_write_places_rows(m):
     v = _rows(11, n=T * Hkv, D=D).reshape(T, Hkv, D)
     kc = rng.integers(-127, 128, size=(NB, bs, Hkv, D)).astype(np.int8)
     vc = rng.integers(-127, 128, size=(NB, bs, Hkv, D)).astype(np.int8)
-    ks = rng.random((NB, bs, Hkv)).astype(np.float32)
-    vs = rng.random((NB, bs, Hkv)).astype(np.float32)
+    ks = rng.random((NB, Hkv, bs)).astype(np.float32)
+    vs = rng.random((NB, Hkv, bs)).astype(np.float32)
     old = [a.copy() for a in (kc, vc, ks, vs)]
     slots = np.array([3, -1, 14, 0, 9, 15])
     m.write_kv_int8(k, v, slots, kc, vc, ks, vs)
     kq, kss = m.quantize_rows(k)
     vq, vss = m.quantize_rows(v)
-    flat = [a.reshape(NB * bs, *a.shape[2:]) for a in (kc, vc, ks, vs)]
-    flat_old = [a.reshape(NB * bs, *a.shape[2:]) for a in old]
+    # every array viewed as [NB * bs rows, ...]: codes directly, scales after moving the token axis forward
+    rows = lambda a: a.reshape(NB * bs, *a.shape[2:]) if a.ndim == 4 else a.transpose(0, 2, 1).reshape(NB * bs, Hkv)
+    flat = [rows(a) for a in (kc, vc, ks, vs)]
+    flat_old = [rows(a) for a in old]
     for t, s in enumerate(slots):
         if s >= 0:
             assert np.array_equal(flat[0][s], kq[t]) and np.array_equal(flat[1][s], vq[t])
@@ -107,8 +109,19 @@ def check_write_places_rows(m):
         assert np.array_equal(a[untouched], b[untouched])
 
 
+def check_dequantized_cache(m):
+    """The cache attention reads: element [b, r, h, d] = code[b, r, h, d] * scale[b, h, r]."""
+    rng = np.random.default_rng(12)
+    codes = rng.integers(-127, 128, size=(3, 4, 2, 8)).astype(np.int8)
+    scales = rng.random((3, 2, 4)).astype(np.float32)
+    deq = m.dequantized_cache(codes, scales)
+    for b, r, h, d in [(0, 0, 0, 0), (2, 3, 1, 7), (1, 2, 0, 5), (2, 1, 1, 0)]:
+        assert deq[b, r, h, d] == float(codes[b, r, h, d]) * float(scales[b, h, r])
+
+
 ALL_CHECKS = [check_amax_maps_to_127, check_half_step_bound, check_zero_and_single_element_rows,
-              check_grid_rows_exact, check_torch_quantizer_agrees, check_write_places_rows]
+              check_grid_rows_exact, check_torch_quantizer_agrees, check_write_places_rows,
+              check_dequantized_cache]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda f: f.__name__)
@@ -122,7 +135,9 @@ MUTATIONS = {
     "scale_from_mean": ("amax = np.max(np.abs(xf), axis=-1)", "amax = np.mean(np.abs(xf), axis=-1)"),
     "scale_not_divided": ("scales[nz] = amax[nz] / np.float32(QMAX)", "scales[nz] = amax[nz]"),
     "row_uses_block_index": ("blk, row = slot // bs, slot % bs", "blk, row = slot // bs, (slot // bs) % bs"),
-    "v_scale_from_k": ("v_scales[blk, row] = vs[t]", "v_scales[blk, row] = ks[t]"),
+    "v_scale_from_k": ("v_scales[blk, :, row] = vs[t]", "v_scales[blk, :, row] = ks[t]"),
+    "scales_not_transposed": ("np.transpose(scales, (0, 2, 1))", "scales.reshape(scales.shape[0], scales.shape[2], "
+                              "scales.shape[1])"),
 }
 
 
