@@ -62,8 +62,8 @@ DECODE_SRC = ("decode.cu", "common.cuh")
 PREFILL_SRC = ("prefill.cu", "common.cuh")
 ROPE_SRC = ("rope_write_kv.cu", "common.cuh")
 NCU_TRAFFIC = {
-    "qwen_decode": {"bytes": 313_465_088, "src": "25100343f6ccb086", "files": DECODE_SRC},
-    "llama70b_long": {"bytes": 1_584_901_888, "src": "25100343f6ccb086", "files": DECODE_SRC},
+    "qwen_decode": {"bytes": 313_465_088, "src": "84d9feaada7e0320", "files": DECODE_SRC},
+    "llama70b_long": {"bytes": 1_584_901_888, "src": "84d9feaada7e0320", "files": DECODE_SRC},
     "prefill": {"bytes": 348_481_024, "src": "0a0c45baf16bf168", "files": PREFILL_SRC},
     "rope_write": {"bytes": 55_164_160, "src": "9b1a5d7fb8331db7", "files": ROPE_SRC},
 }

@@ -15,8 +15,8 @@
 // [C*c/grid, C*(c+1)/grid): every CTA reads the same number of KV bytes,
 // whatever the length mix.  The part of a segment that falls in one CTA is a
 // piece; a piece that is a whole segment writes `out` directly, otherwise it
-// writes fp32 (max, sum, acc) to the workspace and the reduce kernel merges a
-// segment's pieces by the log-sum-exp rule.  This is the single-device reading
+// writes fp32 (max, sum, acc) to the workspace; the CTA that writes a segment's
+// last piece merges them (log-sum-exp rule).  This is the single-device reading
 // of the context split on "In-depth analysis of vllm-ascend", section 3.1.
 //
 // Data movement.  One producer warp walks the CTA's chunk range, looks up each
