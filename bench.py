@@ -50,6 +50,8 @@ WORKLOAD_TEXT = {
     "tiny": "tiny decode: 4 seqs, 4/4 heads, head_dim 64, fp16, block_size 16",
     "prefill": "chunked prefill: 8 seqs, each a 512-token causal chunk appended to an 8192-token paged context, "
                "32 q / 8 kv heads, head_dim 128, bf16, block_size 16",
+    "pool_host": "host block pool of the Qwen3-0.6B-shaped decode batch (128 sequences, block_size 16): per step, one "
+                 "batched append of a token to every sequence and the block-table export (CPU only)",
     "rope_write": "rotary embedding + KV cache write of the chunked-prefill step's 4096 new tokens (8 seqs x 512 at "
                   "positions 8192..8703), 32 q / 8 kv heads, head_dim 128, bf16, block_size 16, fp32 cos/sin "
                   "tables of 16384 positions; before every timed launch L2 is flushed by a 512 MB write followed by a 512 MB "
@@ -772,6 +774,69 @@ def run_rope(args):
     return 0
 
 
+def run_pool_host(args):
+    """Host block pool cost per decode step (the block-allocation row, on the CPU): append one token to each of
+    the batch's sequences with one native call, then export the block table; against one call per sequence
+    and against the oracle's pool doing the same step."""
+    import paged_kv_cache_330_b200 as pa
+    from oracle.block_pool import replay as oreplay
+    from workloads import make_workload
+
+    wl = make_workload("qwen_decode")
+    B, bs = wl.batch, wl.cfg["block_size"]
+    steps, warm = max(1, args.steps), max(3, args.warmup)
+    grow = -(-(steps + warm) // bs) + 1
+    NB = wl.num_blocks + B * 2 * grow
+    order = np.arange(NB, dtype=np.int32)
+    ids = np.arange(B, dtype=np.int64)
+
+    def timed(step_fn, n):
+        t0 = time.perf_counter()
+        for _ in range(n):
+            step_fn()
+        return (time.perf_counter() - t0) / n * 1e6
+
+    pool, bt, _, _, _ = pa.replay_ops(wl.ops, NB, bs, order, B)
+    mb = bt.shape[1] + 2 * grow
+
+    def batched():
+        pool.append_batch(ids, 1)
+        pool.block_table(ids, mb)
+
+    for _ in range(warm):
+        batched()
+    us_batched = timed(batched, steps)
+    pool2, _, _, _, _ = pa.replay_ops(wl.ops, NB, bs, order, B)
+
+    def per_seq():
+        for b in range(B):
+            pool2.append(b, 1)
+        pool2.block_table(ids, mb)
+
+    n_seq = min(steps, 200)
+    us_per_seq = timed(per_seq, n_seq)
+    opool, _, _, _, _ = oreplay(wl.ops, NB, bs, order, B)
+
+    def oracle_step():
+        for b in range(B):
+            opool.append(b, 1)
+        opool.block_table(list(range(B)), mb)
+
+    n_or = min(steps, 200)
+    us_oracle = timed(oracle_step, n_or)
+    line = {
+        "metric": "host block-pool us per decode step (batch 128)", "value": us_batched, "unit": "us",
+        "n_gpus": 0, "steps": steps, "warmup": warm, "ms_per_step": us_batched / 1e3, "higher_is_better": False,
+        "scaling": "none", "vs_baseline": None, "dtype": "int64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT["pool_host"], "one_call_per_sequence_us": us_per_seq},
+        "cpu_baseline": {"value": us_oracle, "unit": "us", "cores": 1, "kind": "oracle",
+                         "sample": f"the oracle's Python pool doing the same step {n_or} times"},
+        "host": os.cpu_count(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -793,6 +858,8 @@ def main():
         return run_prefill(args)
     if args.workload == "rope_write":
         return run_rope(args)
+    if args.workload == "pool_host":
+        return run_pool_host(args)
     return run_ours(args)
 
 

@@ -283,6 +283,16 @@ int pa_seq_fork(pa_pool* pool, int64_t parent_id, int64_t child_id, int n_prefix
 int pa_seq_append(pa_pool* pool, int64_t seq_id, int n, int64_t* slot_mapping_out, int32_t* cow_pairs_out,
                   int* num_cow_out);
 
+/* Extend n sequences in one call: seq_ids[i] by counts[i] tokens, in order i = 0..n-1, with exactly the
+   result of n pa_seq_append calls in that order (the per-step append of a decode batch without a call per
+   sequence: P2 s3.2 checks the host-side allocation hot path).  All or nothing: an unknown id (PA_ERR_NOT_FOUND), a repeated id or a negative count
+   (PA_ERR_INVALID), or a batch needing more blocks than are free (PA_ERR_OOM) leaves the pool unchanged.
+   slot_mapping_out (host int64 [sum counts], may be NULL) receives the new tokens' slots in batch order;
+   cow_pairs_out (host int32 [n][2], may be NULL) receives the copy-on-write (src, dst) pairs, packed in
+   batch order, and *num_cow_out (may be NULL) their number (at most one per sequence). */
+int pa_pool_append_batch(pa_pool* pool, const int64_t* seq_ids, const int32_t* counts, int n,
+                         int64_t* slot_mapping_out, int32_t* cow_pairs_out, int* num_cow_out);
+
 /* Drop a sequence: ref_count -= 1 on each of its blocks; blocks reaching 0 return to the free list. */
 int pa_seq_free(pa_pool* pool, int64_t seq_id);
 

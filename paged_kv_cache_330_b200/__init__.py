@@ -64,6 +64,7 @@ _SIGS = {
     "pa_seq_alloc": (_i, [_vp, _i64, _i]),
     "pa_seq_fork": (_i, [_vp, _i64, _i64, _i]),
     "pa_seq_append": (_i, [_vp, _i64, _i, _i64p, _i32p, _ip]),
+    "pa_pool_append_batch": (_i, [_vp, _i64p, _i32p, _i, _i64p, _i32p, _ip]),
     "pa_seq_free": (_i, [_vp, _i64]),
     "pa_seq_info": (_i, [_vp, _i64, _ip, _ip]),
     "pa_pool_block_table": (_i, [_vp, _i64p, _i, _i32p, _i, _i32p]),
@@ -370,6 +371,21 @@ class BlockPool:
         self._pool_check(lib.pa_seq_append(self._h, seq_id, n, slots.ctypes.data_as(_i64p), pair.ctypes.data_as(_i32p),
                                            ctypes.byref(ncow)), "append")
         return slots[:n], ([(int(pair[0]), int(pair[1]))] if ncow.value else [])
+
+    def append_batch(self, seq_ids, counts):
+        """Extend every sequence of seq_ids by its count (an int applies to all) in one native call; the
+        same result as append() per sequence in order, all or nothing.  Returns (slots int64[sum counts] in
+        batch order, copy-on-write pairs [(src, dst)])."""
+        ids = np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int64))
+        cnt = np.ascontiguousarray(np.broadcast_to(np.asarray(counts, dtype=np.int32), ids.shape))
+        total = int(cnt.sum()) if len(cnt) else 0
+        slots = np.empty(max(total, 1), dtype=np.int64)
+        pairs = np.empty((max(len(ids), 1), 2), dtype=np.int32)
+        ncow = ctypes.c_int(0)
+        self._pool_check(lib.pa_pool_append_batch(self._h, ids.ctypes.data_as(_i64p), cnt.ctypes.data_as(_i32p),
+                                                  len(ids), slots.ctypes.data_as(_i64p), pairs.ctypes.data_as(_i32p),
+                                                  ctypes.byref(ncow)), "append_batch")
+        return slots[:total], [(int(a), int(b)) for a, b in pairs[:ncow.value]]
 
     def free(self, seq_id: int) -> None:
         self._pool_check(lib.pa_seq_free(self._h, seq_id), "free")

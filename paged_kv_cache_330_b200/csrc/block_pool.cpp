@@ -42,8 +42,12 @@ struct pa_pool {
   struct Seq {
     std::vector<int32_t> blocks;        // logical block j -> physical block
     int64_t len = 0;                    // tokens
+    uint64_t mark = 0;                  // last batch that named this sequence (repeat detection)
   };
   std::unordered_map<int64_t, Seq> seqs;
+  uint64_t batch_epoch = 0;
+  std::vector<pa_pool::Seq*> batch_seqs;                      // scratch of pa_pool_append_batch
+  std::vector<std::pair<int32_t, int32_t>> batch_released;    // (block, references dropped by copies)
 
   int32_t take() {
     const int32_t b = free_list.pop_front();
@@ -124,6 +128,40 @@ extern "C" int pa_seq_fork(pa_pool* pool, int64_t parent_id, int64_t child_id, i
   }
 }
 
+// Does appending n tokens to s first copy its last block?  (A shared, partly filled last block.)
+static bool needs_copy(const pa_pool* pool, const pa_pool::Seq& s, int64_t n) {
+  return n > 0 && (s.len % pool->block_size) != 0 && pool->ref[s.blocks.back()] > 1;
+}
+
+// Blocks the pool must hand out to append n tokens to s (including the copy, if any).
+static int64_t blocks_needed(const pa_pool* pool, const pa_pool::Seq& s, int64_t n, bool copy) {
+  return blocks_for(s.len + n, pool->block_size) - (int64_t)s.blocks.size() + (copy ? 1 : 0);
+}
+
+// The state change of one append, once it is known to fit and s.blocks has the capacity: no allocation,
+// cannot fail.  Writes the slots of the new tokens and returns whether the last block was copied.
+static bool append_tokens(pa_pool* pool, pa_pool::Seq& s, int64_t n, int64_t* slots_out, int32_t* pair_out) {
+  const int bs = pool->block_size;
+  const int64_t n0 = s.len;
+  const bool cow = needs_copy(pool, s, n);
+  if (cow) {
+    const int32_t old_b = s.blocks.back();
+    const int32_t new_b = pool->take();
+    pool->ref[old_b] -= 1;
+    s.blocks.back() = new_b;
+    if (pair_out) {
+      pair_out[0] = old_b;
+      pair_out[1] = new_b;
+    }
+  }
+  for (int64_t p = n0; p < n0 + n; ++p) {
+    if (p % bs == 0) s.blocks.push_back(pool->take());  // within capacity: no allocation
+    if (slots_out) slots_out[p - n0] = (int64_t)s.blocks[p / bs] * bs + p % bs;
+  }
+  s.len = n0 + n;
+  return cow;
+}
+
 extern "C" int pa_seq_append(pa_pool* pool, int64_t seq_id, int n, int64_t* slot_mapping_out,
                              int32_t* cow_pairs_out, int* num_cow_out) {
   if (!pool || n < 0) return PA_ERR_INVALID;
@@ -131,29 +169,67 @@ extern "C" int pa_seq_append(pa_pool* pool, int64_t seq_id, int n, int64_t* slot
     auto it = pool->seqs.find(seq_id);
     if (it == pool->seqs.end()) return PA_ERR_NOT_FOUND;
     pa_pool::Seq& s = it->second;
-    const int bs = pool->block_size;
-    const int64_t n0 = s.len;
-    const bool cow = n > 0 && (n0 % bs) != 0 && pool->ref[s.blocks.back()] > 1;
-    const int64_t need = blocks_for(n0 + n, bs) - (int64_t)s.blocks.size() + (cow ? 1 : 0);
+    const int64_t need = blocks_needed(pool, s, n, needs_copy(pool, s, n));
     if (need > (int64_t)pool->free_list.size()) return PA_ERR_OOM;
-    s.blocks.reserve(blocks_for(n0 + n, bs));
-    if (num_cow_out) *num_cow_out = 0;
-    if (cow) {
-      const int32_t old_b = s.blocks.back();
-      const int32_t new_b = pool->take();
-      pool->ref[old_b] -= 1;
-      s.blocks.back() = new_b;
-      if (cow_pairs_out) {
-        cow_pairs_out[0] = old_b;
-        cow_pairs_out[1] = new_b;
+    s.blocks.reserve(blocks_for(s.len + n, pool->block_size));
+    const bool cow = append_tokens(pool, s, n, slot_mapping_out, cow_pairs_out);
+    if (num_cow_out) *num_cow_out = cow ? 1 : 0;
+    return PA_OK;
+  } catch (...) {
+    return PA_ERR_OOM;
+  }
+}
+
+extern "C" int pa_pool_append_batch(pa_pool* pool, const int64_t* seq_ids, const int32_t* counts, int n,
+                                    int64_t* slot_mapping_out, int32_t* cow_pairs_out, int* num_cow_out) {
+  if (!pool || n < 0 || (n > 0 && (!seq_ids || !counts))) return PA_ERR_INVALID;
+  try {
+    // Dry run: find every sequence, reject repeats, and count the blocks the batch takes.  A copy made for
+    // one sequence lowers the count of a block another sequence of the batch may share, exactly as
+    // separate calls in this order would see it (`released`, short: copies are rare).
+    std::vector<pa_pool::Seq*>& seq = pool->batch_seqs;
+    auto& released = pool->batch_released;
+    seq.resize(n);
+    released.clear();
+    const uint64_t epoch = ++pool->batch_epoch;
+    int64_t need = 0;
+    for (int i = 0; i < n; ++i) {
+      if (counts[i] < 0) return PA_ERR_INVALID;
+      auto it = pool->seqs.find(seq_ids[i]);
+      if (it == pool->seqs.end()) return PA_ERR_NOT_FOUND;
+      pa_pool::Seq& s = it->second;
+      if (s.mark == epoch) return PA_ERR_INVALID;  // named twice in this batch
+      s.mark = epoch;
+      seq[i] = &s;
+      bool copy = false;
+      if (counts[i] > 0 && (s.len % pool->block_size) != 0) {
+        const int32_t last = s.blocks.back();
+        int32_t dropped = 0;
+        size_t k = 0;
+        for (; k < released.size() && released[k].first != last; ++k) {
+        }
+        if (k < released.size()) dropped = released[k].second;
+        copy = pool->ref[last] - dropped > 1;
+        if (copy) {
+          if (k < released.size())
+            released[k].second += 1;
+          else
+            released.emplace_back(last, 1);
+        }
       }
-      if (num_cow_out) *num_cow_out = 1;
+      need += blocks_needed(pool, s, counts[i], copy);
     }
-    for (int64_t p = n0; p < n0 + n; ++p) {
-      if (p % bs == 0) s.blocks.push_back(pool->take());  // within capacity: no allocation
-      if (slot_mapping_out) slot_mapping_out[p - n0] = (int64_t)s.blocks[p / bs] * bs + p % bs;
+    if (need > (int64_t)pool->free_list.size()) return PA_ERR_OOM;
+    for (int i = 0; i < n; ++i) seq[i]->blocks.reserve(blocks_for(seq[i]->len + counts[i], pool->block_size));
+    // Apply: nothing below allocates or fails.
+    int64_t off = 0;
+    int ncow = 0;
+    for (int i = 0; i < n; ++i) {
+      int32_t* pair = cow_pairs_out ? cow_pairs_out + 2 * ncow : nullptr;
+      if (append_tokens(pool, *seq[i], counts[i], slot_mapping_out ? slot_mapping_out + off : nullptr, pair)) ++ncow;
+      off += counts[i];
     }
-    s.len = n0 + n;
+    if (num_cow_out) *num_cow_out = ncow;
     return PA_OK;
   } catch (...) {
     return PA_ERR_OOM;

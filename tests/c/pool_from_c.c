@@ -66,6 +66,19 @@ int main(void) {
   CHECK(pa_pool_ref_count(p, last_shared) == 1 && pa_pool_ref_count(p, cow[1]) == 1);
   CHECK(invariants(p));
 
+  /* one call for a whole batch: sequences 1 and 2 gain two tokens each, in order */
+  {
+    int64_t bids[2] = {1, 2}, bslots[4];
+    int32_t bcounts[2] = {2, 2}, bpairs[4];
+    int bncow = -1;
+    CHECK(pa_pool_append_batch(p, bids, bcounts, 2, bslots, bpairs, &bncow) == PA_OK && bncow == 0);
+    CHECK(pa_pool_block_table(p, ids, 2, &table[0][0], 64, lens) == PA_OK && lens[0] == 1002 && lens[1] == 995);
+    CHECK(bslots[0] == (int64_t)table[0][62] * BS + 1000 % BS && bslots[1] == bslots[0] + 1);
+    CHECK(bslots[2] == (int64_t)table[1][62] * BS + 1 && bslots[3] == bslots[2] + 1);
+    int64_t dup[2] = {1, 1};
+    CHECK(pa_pool_append_batch(p, dup, bcounts, 2, NULL, NULL, NULL) == PA_ERR_INVALID);
+  }
+
   /* too many tokens: refused, pool unchanged */
   CHECK(pa_pool_stats(p, &st) == PA_OK);
   const int64_t free_before = st.free_blocks;

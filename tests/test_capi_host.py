@@ -211,6 +211,93 @@ def test_pool_errors_leave_state_unchanged():
     assert p.stats()["used_blocks"] == 4
 
 
+def _oracle_batch(orc: OraclePool, ids, counts):
+    """The oracle's reading of a batched append: one append per sequence, in batch order."""
+    slots, pairs = [], []
+    for sid, n in zip(ids, counts):
+        s, p = orc.append(sid, n)
+        slots += s
+        pairs += p
+    return slots, pairs
+
+
+def _snapshot(pool: pa.BlockPool, ids, nb):
+    mb = max(pool.info(i)[1] for i in ids) + 1
+    return pool.stats(), pool.block_table(ids, mb), [pool.ref_count(b) for b in range(nb)]
+
+
+def test_append_batch_matches_sequential_appends():
+    """Random batches over forked sequences (shared full and partial blocks): the native batched append gives
+    the oracle's sequential result — slots, copy-on-write pairs, block tables, reference counts."""
+    rnd = random.Random(23)
+    for bs in (16, 32, 128):
+        NB = 12000                                                    # never exhausted by 120 batches
+        order = list(np.random.default_rng(bs + 1).permutation(NB))
+        cpp, orc = pa.BlockPool(NB, bs, order), OraclePool(NB, bs, order)
+        live = []
+        for sid in range(6):
+            n = rnd.randint(1, 5 * bs)
+            cpp.alloc(sid, n); orc.alloc(sid, n); live.append(sid)
+        nid = 6
+        for step in range(120):
+            if rnd.random() < 0.35:                                   # fork at any point (partial blocks too)
+                p = rnd.choice(live)
+                k = rnd.randint(0, orc.seqs[p]["len"])
+                cpp.fork(p, nid, k); orc.fork(p, nid, k); live.append(nid); nid += 1
+            if len(live) > 24:
+                s = live.pop(rnd.randrange(len(live)))
+                cpp.free(s); orc.free_seq(s)
+            batch = rnd.sample(live, rnd.randint(1, len(live)))
+            counts = [rnd.choice([0, 1, 1, 1, 2, bs - 1, bs, bs + 3]) for _ in batch]
+            o_res = _oracle_batch(orc, batch, counts)
+            c_slots, c_pairs = cpp.append_batch(batch, counts)
+            np.testing.assert_array_equal(c_slots, np.array(o_res[0], dtype=np.int64))
+            assert c_pairs == o_res[1], (step, batch, counts)
+            if step % 10 == 0:
+                _compare_pools(cpp, orc, live)
+        _compare_pools(cpp, orc, live)
+
+
+def test_append_batch_two_sharers_of_one_partial_block():
+    """Two sequences share a partly filled last block: the first append copies it, after which the second
+    holds it alone and appends in place (no second copy) — and a pool with exactly the blocks that needs
+    accepts the batch."""
+    for make in (lambda: pa.BlockPool(4, 16), lambda: OraclePool(4, 16)):
+        pool = make()
+        pool.alloc(0, 20)                       # blocks 0, 1 (the second partly filled)
+        pool.fork(0, 1, 20)                     # both hold blocks 0 and 1
+        assert len(pool.free) == 2 if isinstance(pool, OraclePool) else pool.stats()["free_blocks"] == 2
+    cpp, orc = pa.BlockPool(3, 16), OraclePool(3, 16)
+    for p in (cpp, orc):
+        p.alloc(0, 20); p.fork(0, 1, 20)
+    slots, pairs = cpp.append_batch([0, 1], [1, 1])    # one free block: enough, since only one copy is made
+    o_slots, o_pairs = _oracle_batch(orc, [0, 1], [1, 1])
+    assert pairs == o_pairs == [(1, 2)]
+    np.testing.assert_array_equal(slots, np.array(o_slots, dtype=np.int64))
+    assert slots.tolist() == [2 * 16 + 4, 1 * 16 + 4]
+    _compare_pools(cpp, orc, [0, 1])
+
+
+def test_append_batch_is_all_or_nothing():
+    cpp = pa.BlockPool(10, 16)
+    cpp.alloc(0, 30); cpp.alloc(1, 5); cpp.fork(1, 2, 5)
+    before = _snapshot(cpp, [0, 1, 2], 10)
+    with pytest.raises(pa.PoolOutOfBlocks):
+        cpp.append_batch([0, 1, 2], [16, 16, 200])          # the last one cannot fit: nothing is applied
+    with pytest.raises(pa.PagedAttnError):
+        cpp.append_batch([0, 1, 0], [1, 1, 1])              # repeated id
+    with pytest.raises(pa.PagedAttnError):
+        cpp.append_batch([0, 7], [1, 1])                    # unknown id
+    with pytest.raises(pa.PagedAttnError):
+        cpp.append_batch([0, 1], [1, -1])                   # negative count
+    after = _snapshot(cpp, [0, 1, 2], 10)
+    assert before[0] == after[0] and before[2] == after[2]
+    for x, y in zip(before[1], after[1]):
+        np.testing.assert_array_equal(x, y)
+    slots, pairs = cpp.append_batch([], [])
+    assert slots.shape == (0,) and pairs == []
+
+
 @pytest.mark.parametrize("name,bs", [("tiny", None), ("qwen_decode", None), ("llama70b_long", None),
                                      ("prefix_sweep", 16), ("prefix_sweep", 256), ("prefill", None)])
 def test_workload_replay_parity(name, bs):
