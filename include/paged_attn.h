@@ -293,6 +293,15 @@ int pa_seq_append(pa_pool* pool, int64_t seq_id, int n, int64_t* slot_mapping_ou
 int pa_pool_append_batch(pa_pool* pool, const int64_t* seq_ids, const int32_t* counts, int n,
                          int64_t* slot_mapping_out, int32_t* cow_pairs_out, int* num_cow_out);
 
+/* New sequences seq_ids[i] of num_tokens[i] tokens each, as n pa_seq_alloc calls in order would make them.
+   All or nothing: a live or repeated id (PA_ERR_NOT_FOUND / PA_ERR_INVALID), a negative count
+   (PA_ERR_INVALID) or too few free blocks for the whole batch (PA_ERR_OOM) leaves the pool unchanged. */
+int pa_pool_alloc_batch(pa_pool* pool, const int64_t* seq_ids, const int32_t* num_tokens, int n);
+
+/* Drop sequences seq_ids[0..n), as n pa_seq_free calls in order would.  All or nothing: an unknown
+   (PA_ERR_NOT_FOUND) or repeated (PA_ERR_INVALID) id leaves the pool unchanged. */
+int pa_pool_free_batch(pa_pool* pool, const int64_t* seq_ids, int n);
+
 /* Drop a sequence: ref_count -= 1 on each of its blocks; blocks reaching 0 return to the free list. */
 int pa_seq_free(pa_pool* pool, int64_t seq_id);
 

@@ -65,6 +65,8 @@ _SIGS = {
     "pa_seq_fork": (_i, [_vp, _i64, _i64, _i]),
     "pa_seq_append": (_i, [_vp, _i64, _i, _i64p, _i32p, _ip]),
     "pa_pool_append_batch": (_i, [_vp, _i64p, _i32p, _i, _i64p, _i32p, _ip]),
+    "pa_pool_alloc_batch": (_i, [_vp, _i64p, _i32p, _i]),
+    "pa_pool_free_batch": (_i, [_vp, _i64p, _i]),
     "pa_seq_free": (_i, [_vp, _i64]),
     "pa_seq_info": (_i, [_vp, _i64, _ip, _ip]),
     "pa_pool_block_table": (_i, [_vp, _i64p, _i, _i32p, _i, _i32p]),
@@ -386,6 +388,18 @@ class BlockPool:
                                                   len(ids), slots.ctypes.data_as(_i64p), pairs.ctypes.data_as(_i32p),
                                                   ctypes.byref(ncow)), "append_batch")
         return slots[:total], [(int(a), int(b)) for a, b in pairs[:ncow.value]]
+
+    def alloc_batch(self, seq_ids, num_tokens) -> None:
+        """New sequences (num_tokens per id, or one int for all) in one native call; all or nothing."""
+        ids = np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int64))
+        cnt = np.ascontiguousarray(np.broadcast_to(np.asarray(num_tokens, dtype=np.int32), ids.shape))
+        self._pool_check(lib.pa_pool_alloc_batch(self._h, ids.ctypes.data_as(_i64p), cnt.ctypes.data_as(_i32p),
+                                                 len(ids)), "alloc_batch")
+
+    def free_batch(self, seq_ids) -> None:
+        """Drop every sequence of seq_ids in one native call; all or nothing."""
+        ids = np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int64))
+        self._pool_check(lib.pa_pool_free_batch(self._h, ids.ctypes.data_as(_i64p), len(ids)), "free_batch")
 
     def free(self, seq_id: int) -> None:
         self._pool_check(lib.pa_seq_free(self._h, seq_id), "free")

@@ -10,6 +10,7 @@
 // caller's device tensors.  Every operation checks first and mutates second,
 // so a failed call leaves the pool unchanged.
 
+#include <algorithm>
 #include <cstdint>
 #include <unordered_map>
 #include <vector>
@@ -234,6 +235,65 @@ extern "C" int pa_pool_append_batch(pa_pool* pool, const int64_t* seq_ids, const
   } catch (...) {
     return PA_ERR_OOM;
   }
+}
+
+// Marks every id of a batch (a sequence named twice is an error); `must_exist` selects whether each id must
+// name a live sequence or a free one.  Returns PA_OK or the error of the first offending id; sets nothing.
+static int check_batch_ids(pa_pool* pool, const int64_t* ids, int n, bool must_exist, std::vector<int64_t>& seen) {
+  seen.assign(ids, ids + n);
+  std::sort(seen.begin(), seen.end());
+  if (std::adjacent_find(seen.begin(), seen.end()) != seen.end()) return PA_ERR_INVALID;
+  for (int i = 0; i < n; ++i) {
+    const bool live = pool->seqs.count(ids[i]) != 0;
+    if (live != must_exist) return PA_ERR_NOT_FOUND;
+  }
+  return PA_OK;
+}
+
+extern "C" int pa_pool_alloc_batch(pa_pool* pool, const int64_t* seq_ids, const int32_t* num_tokens, int n) {
+  if (!pool || n < 0 || (n > 0 && (!seq_ids || !num_tokens))) return PA_ERR_INVALID;
+  try {
+    std::vector<int64_t> scratch;
+    const int st = check_batch_ids(pool, seq_ids, n, false, scratch);
+    if (st != PA_OK) return st;
+    int64_t need = 0;
+    for (int i = 0; i < n; ++i) {
+      if (num_tokens[i] < 0) return PA_ERR_INVALID;
+      need += blocks_for(num_tokens[i], pool->block_size);
+    }
+    if (need > (int64_t)pool->free_list.size()) return PA_ERR_OOM;
+    // every node and vector is allocated before the first block is taken
+    std::vector<pa_pool::Seq*> made(n);
+    for (int i = 0; i < n; ++i) {
+      pa_pool::Seq s;
+      s.blocks.reserve(blocks_for(num_tokens[i], pool->block_size));
+      s.len = num_tokens[i];
+      auto res = pool->seqs.emplace(seq_ids[i], std::move(s));
+      made[i] = &res.first->second;
+    }
+    for (int i = 0; i < n; ++i)
+      for (int64_t j = 0, nb = blocks_for(num_tokens[i], pool->block_size); j < nb; ++j)
+        made[i]->blocks.push_back(pool->take());
+    return PA_OK;
+  } catch (...) {
+    // Only an insertion can throw, before any block is taken; every id of the batch was absent on entry, so
+    // the sequences already inserted are exactly the batch ids now present.
+    for (int i = 0; i < n; ++i) pool->seqs.erase(seq_ids[i]);
+    return PA_ERR_OOM;
+  }
+}
+
+extern "C" int pa_pool_free_batch(pa_pool* pool, const int64_t* seq_ids, int n) {
+  if (!pool || n < 0 || (n > 0 && !seq_ids)) return PA_ERR_INVALID;
+  try {
+    std::vector<int64_t> scratch;
+    const int st = check_batch_ids(pool, seq_ids, n, true, scratch);
+    if (st != PA_OK) return st;
+  } catch (...) {
+    return PA_ERR_OOM;
+  }
+  for (int i = 0; i < n; ++i) pa_seq_free(pool, seq_ids[i]);  // cannot fail now: every id is live and distinct
+  return PA_OK;
 }
 
 extern "C" int pa_seq_free(pa_pool* pool, int64_t seq_id) {

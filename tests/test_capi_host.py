@@ -298,6 +298,74 @@ def test_append_batch_is_all_or_nothing():
     assert slots.shape == (0,) and pairs == []
 
 
+def test_alloc_and_free_batches_match_sequential_calls():
+    """Admission and retirement in batches: the same block tables, counts and free list as one call per
+    sequence in order (compared with the oracle pool), interleaved with batched appends and forks."""
+    rnd = random.Random(31)
+    for bs in (16, 64):
+        NB = 3000
+        order = list(np.random.default_rng(bs + 7).permutation(NB))
+        cpp, orc = pa.BlockPool(NB, bs, order), OraclePool(NB, bs, order)
+        live, nid = [], 0
+        for step in range(60):
+            k = rnd.randint(0, 6)
+            ids = list(range(nid, nid + k))
+            lens = [rnd.randint(0, 3 * bs) for _ in ids]
+            nid += k
+            cpp.alloc_batch(ids, lens)
+            for i, n in zip(ids, lens):
+                orc.alloc(i, n)
+            live += ids
+            if live and rnd.random() < 0.4:
+                p = rnd.choice(live)
+                f = rnd.randint(0, orc.seqs[p]["len"])
+                cpp.fork(p, nid, f); orc.fork(p, nid, f); live.append(nid); nid += 1
+            if live:
+                batch = rnd.sample(live, rnd.randint(1, len(live)))
+                cpp.append_batch(batch, 1)
+                _oracle_batch(orc, batch, [1] * len(batch))
+            if len(live) > 8:
+                gone = rnd.sample(live, rnd.randint(1, len(live) // 2))
+                cpp.free_batch(gone)
+                for g in gone:
+                    orc.free_seq(g)
+                    live.remove(g)
+            _compare_pools(cpp, orc, live)
+        cpp.free_batch(live)
+        for g in live:
+            orc.free_seq(g)
+        _compare_pools(cpp, orc, [])
+        assert cpp.stats()["free_blocks"] == NB
+
+
+def test_alloc_and_free_batches_are_all_or_nothing():
+    cpp = pa.BlockPool(6, 16)
+    cpp.alloc_batch([0, 1], [20, 16])                        # 3 blocks
+    before = _snapshot(cpp, [0, 1], 6)
+    with pytest.raises(pa.PoolOutOfBlocks):
+        cpp.alloc_batch([2, 3], [16, 40])                    # needs 4 of the 3 free blocks
+    with pytest.raises(pa.PagedAttnError):
+        cpp.alloc_batch([2, 2], [1, 1])                      # repeated id
+    with pytest.raises(pa.PagedAttnError):
+        cpp.alloc_batch([2, 1], [1, 1])                      # a live id
+    with pytest.raises(pa.PagedAttnError):
+        cpp.alloc_batch([2, 3], [1, -1])                     # negative count
+    with pytest.raises(pa.PagedAttnError):
+        cpp.free_batch([0, 5])                               # unknown id: sequence 0 stays
+    with pytest.raises(pa.PagedAttnError):
+        cpp.free_batch([1, 1])                               # repeated id
+    after = _snapshot(cpp, [0, 1], 6)
+    assert before[0] == after[0] and before[2] == after[2]
+    for x, y in zip(before[1], after[1]):
+        np.testing.assert_array_equal(x, y)
+    cpp.alloc_batch([2, 3, 4], [0, 16, 1])                   # 0 + 1 + 1 blocks of the 3 free
+    assert cpp.stats()["free_blocks"] == 1
+    cpp.free_batch([0, 1, 2, 3, 4])
+    assert cpp.stats()["free_blocks"] == 6 and cpp.stats()["num_seqs"] == 0
+    cpp.alloc_batch([], [])
+    cpp.free_batch([])
+
+
 @pytest.mark.parametrize("name,bs", [("tiny", None), ("qwen_decode", None), ("llama70b_long", None),
                                      ("prefix_sweep", 16), ("prefix_sweep", 256), ("prefill", None)])
 def test_workload_replay_parity(name, bs):
