@@ -188,13 +188,17 @@ int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int
 /* is one static device array of PA_DECODE_STATIC_SCRATCH_BYTES, reserved   */
 /* on every GPU that loads the library until the process exits.  Calls that */
 /* would need more (pa_decode_workspace_size() larger than that) return     */
-/* PA_ERR_WORKSPACE.  Nothing is allocated: the call only clears the piece */
-/* counters at the head of the array (cudaMemsetAsync on `stream`) and runs */
-/* the decode kernel.  The first call on a device looks up the array's     */
-/* device address (cudaGetSymbolAddress) with that device current; make     */
-/* that first call before any stream capture.  All calls share the one      */
-/* array and it keeps the last call's contents, so calls whose work overlaps */
-/* on the GPU (other streams, other threads) race: serialise them.          */
+/* PA_ERR_WORKSPACE.  Every other argument is checked as pa_decode checks  */
+/* it, before anything is enqueued; a rejected call enqueues nothing.       */
+/* Nothing is allocated: an accepted call clears the piece counters at the  */
+/* head of the array (cudaMemsetAsync on `stream`) and runs the decode      */
+/* kernel.  Because of that clear, decode on this entry point does not      */
+/* start early under a preceding pa_write_kv / pa_rope_write_kv (pa_decode  */
+/* does).  The first call on a device looks up the array's device address  */
+/* (cudaGetSymbolAddress) with that device current; make that first call    */
+/* before any stream capture.  All calls share the one array and it keeps   */
+/* the last call's contents, so calls whose work overlaps on the GPU (other */
+/* streams, other threads) race: serialise them.                            */
 /* ------------------------------------------------------------------------ */
 #define PA_DECODE_STATIC_SCRATCH_BYTES (8u << 20)
 int pa_decode_static_scratch(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,

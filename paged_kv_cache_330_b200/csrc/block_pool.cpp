@@ -252,6 +252,7 @@ static int check_batch_ids(pa_pool* pool, const int64_t* ids, int n, bool must_e
 
 extern "C" int pa_pool_alloc_batch(pa_pool* pool, const int64_t* seq_ids, const int32_t* num_tokens, int n) {
   if (!pool || n < 0 || (n > 0 && (!seq_ids || !num_tokens))) return PA_ERR_INVALID;
+  int inserted = 0;  // batch ids this call has put into the pool (ids 0..inserted-1, each absent on entry)
   try {
     std::vector<int64_t> scratch;
     const int st = check_batch_ids(pool, seq_ids, n, false, scratch);
@@ -270,15 +271,16 @@ extern "C" int pa_pool_alloc_batch(pa_pool* pool, const int64_t* seq_ids, const 
       s.len = num_tokens[i];
       auto res = pool->seqs.emplace(seq_ids[i], std::move(s));
       made[i] = &res.first->second;
+      inserted = i + 1;
     }
     for (int i = 0; i < n; ++i)
       for (int64_t j = 0, nb = blocks_for(num_tokens[i], pool->block_size); j < nb; ++j)
         made[i]->blocks.push_back(pool->take());
     return PA_OK;
   } catch (...) {
-    // Only an insertion can throw, before any block is taken; every id of the batch was absent on entry, so
-    // the sequences already inserted are exactly the batch ids now present.
-    for (int i = 0; i < n; ++i) pool->seqs.erase(seq_ids[i]);
+    // Only the id check or an insertion can throw, before any block is taken.  Remove exactly the sequences
+    // inserted here (they hold no blocks yet); a sequence that was live on entry is never touched.
+    for (int i = 0; i < inserted; ++i) pool->seqs.erase(seq_ids[i]);
     return PA_ERR_OOM;
   }
 }

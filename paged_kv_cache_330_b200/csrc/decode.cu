@@ -39,6 +39,7 @@
 //     keeps it exact to about 2^-17 instead of the 2^-9 of one bf16 rounding.
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <type_traits>
 
@@ -1043,13 +1044,14 @@ int launch(const CUtensorMap& km, const CUtensorMap& vm, const DecodeParams& p, 
   constexpr bool MMA = G >= 8;
   using LY = Layout<D, G, kNW, kStages, MMA>;
   auto kern = decode_kernel<DT, D, G, kNW, kStages, MMA>;
-  static bool attr_set[64] = {};  // per instantiation and device
+  // per instantiation and device; host threads may race to set it, which only repeats an idempotent call
+  static std::atomic<bool> attr_set[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+  if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::ALLOC) != cudaSuccess)
       return PA_ERR_CUDA;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
   }
   // programmatic dependent launch: may start while the preceding pa_write_kv runs (it signals
   // its dependents at entry); the producer waits for it before the first cache load
@@ -1103,11 +1105,23 @@ extern "C" size_t pa_decode_workspace_size(int batch, int num_q_heads, int num_k
   return ws;
 }
 
-extern "C" int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
-                         int max_blocks_per_seq, const int32_t* context_lens, int batch, int num_q_heads,
-                         int num_kv_heads, int head_dim, int block_size, int num_blocks, int max_context_len,
-                         float scale, int dtype, void* workspace, size_t workspace_bytes, int num_partitions_or_0,
-                         void* out, void* stream) {
+namespace {
+
+// Everything pa_decode does before it enqueues work: argument checks, the plan, the kernel parameters and
+// the two tensor maps.  Enqueues nothing; returns PA_OK with *launchable = false when there is nothing to
+// run (batch 0).
+struct DecodeCall {
+  DecodeParams p;
+  CUtensorMap km, vm;
+  int dtype, head_dim, G;
+  bool launchable;
+};
+
+int decode_prepare(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                   int max_blocks_per_seq, const int32_t* context_lens, int batch, int num_q_heads, int num_kv_heads,
+                   int head_dim, int block_size, int num_blocks, int max_context_len, float scale, int dtype,
+                   void* workspace, size_t workspace_bytes, int num_partitions_or_0, void* out, DecodeCall* call) {
+  call->launchable = false;
   if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks < 0 ||
       max_context_len < 0 || max_blocks_per_seq < 0 || num_partitions_or_0 < 0)
     return PA_ERR_INVALID;
@@ -1129,7 +1143,7 @@ extern "C" int pa_decode(const void* q, const void* k_cache, const void* v_cache
   if (!workspace || workspace_bytes < pl.ws_bytes) return PA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PA_ERR_ALIGN;
 
-  DecodeParams p;
+  DecodeParams& p = call->p;
   p.q = q;
   p.out = out;
   p.block_tables = block_tables;
@@ -1149,16 +1163,38 @@ extern "C" int pa_decode(const void* q, const void* k_cache, const void* v_cache
   p.scale_log2 = scale * kLog2e;
 
   // One tensor map per cache over the [num_blocks*block_size][Hkv*D] row view; 16-row x 64-column boxes.
-  CUtensorMap km, vm;
   const uint64_t rows = (uint64_t)std::max(num_blocks, 1) * block_size;
   const uint64_t cols = (uint64_t)num_kv_heads * head_dim;
-  if (pa::encode_2d_sw128(&km, k_cache, cols, rows, cols * 2, 64, 16) != PA_OK) return PA_ERR_CUDA;
-  if (pa::encode_2d_sw128(&vm, v_cache, cols, rows, cols * 2, 64, 16) != PA_OK) return PA_ERR_CUDA;
+  if (pa::encode_2d_sw128(&call->km, k_cache, cols, rows, cols * 2, 64, 16) != PA_OK) return PA_ERR_CUDA;
+  if (pa::encode_2d_sw128(&call->vm, v_cache, cols, rows, cols * 2, 64, 16) != PA_OK) return PA_ERR_CUDA;
+  call->dtype = dtype;
+  call->head_dim = head_dim;
+  call->G = G;
+  call->launchable = true;
+  return PA_OK;
+}
 
-  cudaStream_t st = (cudaStream_t)stream;
-  if (dtype == PA_BF16)
-    return head_dim == 128 ? dispatch_g<PA_BF16, 128>(G, km, vm, p, st) : dispatch_g<PA_BF16, 64>(G, km, vm, p, st);
-  return head_dim == 128 ? dispatch_g<PA_F16, 128>(G, km, vm, p, st) : dispatch_g<PA_F16, 64>(G, km, vm, p, st);
+int decode_launch(const DecodeCall& c, cudaStream_t st) {
+  if (c.dtype == PA_BF16)
+    return c.head_dim == 128 ? dispatch_g<PA_BF16, 128>(c.G, c.km, c.vm, c.p, st)
+                             : dispatch_g<PA_BF16, 64>(c.G, c.km, c.vm, c.p, st);
+  return c.head_dim == 128 ? dispatch_g<PA_F16, 128>(c.G, c.km, c.vm, c.p, st)
+                           : dispatch_g<PA_F16, 64>(c.G, c.km, c.vm, c.p, st);
+}
+
+}  // namespace
+
+extern "C" int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                         int max_blocks_per_seq, const int32_t* context_lens, int batch, int num_q_heads,
+                         int num_kv_heads, int head_dim, int block_size, int num_blocks, int max_context_len,
+                         float scale, int dtype, void* workspace, size_t workspace_bytes, int num_partitions_or_0,
+                         void* out, void* stream) {
+  DecodeCall call;
+  const int s = decode_prepare(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch,
+                               num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, max_context_len, scale,
+                               dtype, workspace, workspace_bytes, num_partitions_or_0, out, &call);
+  if (s != PA_OK || !call.launchable) return s;
+  return decode_launch(call, (cudaStream_t)stream);
 }
 
 // ------------------------------------------------------------------ decode with library-owned scratch
@@ -1196,6 +1232,7 @@ extern "C" int pa_decode_static_scratch(const void* q, const void* k_cache, cons
                                         const int32_t* context_lens, int batch, int num_q_heads, int num_kv_heads,
                                         int head_dim, int block_size, int num_blocks, int max_context_len, float scale,
                                         int dtype, int num_partitions_or_0, void* out, void* stream) {
+  // A plan larger than the static scratch is refused first, whatever the other arguments.
   size_t need = 0;
   int s = pa_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_partitions_or_0, nullptr,
                          nullptr, &need);
@@ -1203,12 +1240,18 @@ extern "C" int pa_decode_static_scratch(const void* q, const void* k_cache, cons
   if (need > PA_DECODE_STATIC_SCRATCH_BYTES) return PA_ERR_WORKSPACE;  // batch too large for the static scratch
   void* scratch = nullptr;
   if ((s = static_scratch_ptr(&scratch)) != PA_OK) return s;
-  // The head of the scratch holds the per-segment piece counters, which must start at zero.  A
-  // completed call leaves them at zero, but clear them anyway so an earlier failed call cannot leak in.
-  if (batch > 0 && num_kv_heads > 0 &&
-      cudaMemsetAsync(scratch, 0, (size_t)batch * num_kv_heads * sizeof(int), (cudaStream_t)stream) != cudaSuccess)
+  // Every check pa_decode makes, before anything is enqueued: a rejected call leaves the stream and the
+  // scratch untouched.
+  DecodeCall call;
+  s = decode_prepare(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch, num_q_heads,
+                     num_kv_heads, head_dim, block_size, num_blocks, max_context_len, scale, dtype, scratch,
+                     PA_DECODE_STATIC_SCRATCH_BYTES, num_partitions_or_0, out, &call);
+  if (s != PA_OK || !call.launchable) return s;
+  // The head of the scratch holds the per-segment piece counters, which must start at zero.  A completed
+  // call leaves them at zero, but they are cleared anyway so that an earlier call that gave up (a timed-out
+  // wait) cannot leak into this one.  The clear is a stream operation between the preceding kernel and the
+  // decode kernel, so on this entry point decode does not start early under a preceding pa_write_kv.
+  if (cudaMemsetAsync(scratch, 0, (size_t)batch * num_kv_heads * sizeof(int), (cudaStream_t)stream) != cudaSuccess)
     return PA_ERR_CUDA;
-  return pa_decode(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch, num_q_heads,
-                   num_kv_heads, head_dim, block_size, num_blocks, max_context_len, scale, dtype, scratch,
-                   PA_DECODE_STATIC_SCRATCH_BYTES, num_partitions_or_0, out, stream);
+  return decode_launch(call, (cudaStream_t)stream);
 }
