@@ -314,7 +314,7 @@ def run_reference(args):
         return 0
     from workloads import make_workload
     wname = "prefill" if args.workload == "rope_write" else args.workload
-    wl = make_workload(wname)
+    wl = make_workload(wname, block_size=getattr(args, "block_size", None))
     metric, unit, sample = METRIC, UNIT, {}
     if args.workload == "prefill":
         metric, unit = PREFILL_METRIC, "TFLOP/s"
@@ -376,7 +376,7 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    wl = make_workload(args.workload, seed=None if rank == 0 else 1000 * rank + 1)
+    wl = make_workload(args.workload, seed=None if rank == 0 else 1000 * rank + 1, block_size=args.block_size)
     c = wl.cfg
     _, bt, lens, sm, _ = pa.replay_ops(wl.ops, wl.num_blocks, c["block_size"], wl.free_order, wl.batch)
     maxL = int(lens.max())
@@ -439,26 +439,29 @@ def run_ours(args):
         g_steps.replay()
     torch.cuda.synchronize(dev)
 
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    d_start, d_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # The K-step loop is timed `repeats` times (each bracketed by barrier + synchronize); the median of the
+    # repeats is reported.  Each repeat is followed by the decode kernel alone, same launch count.
+    step_ms, dec_ms = [], []
     with ClockSampler(local) as clk:
-        barrier()
-        torch.cuda.synchronize(dev)
-        t_start.record(stream)
-        for _ in range(K // S):
-            g_steps.replay()
-        t_end.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier()
-        # decode kernel alone, same launch count, straight after the timed region
-        d_start.record(stream)
-        for _ in range(K // S):
-            g_decs.replay()
-        d_end.record(stream)
-        torch.cuda.synchronize(dev)
-    ms_total = t_start.elapsed_time(t_end)
-    dec_ms = [d_start.elapsed_time(d_end) / K]
-    ms_step = ms_total / K
+        for _ in range(args.repeats):
+            t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            d_start, d_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            barrier()
+            torch.cuda.synchronize(dev)
+            t_start.record(stream)
+            for _ in range(K // S):
+                g_steps.replay()
+            t_end.record(stream)
+            torch.cuda.synchronize(dev)
+            barrier()
+            d_start.record(stream)
+            for _ in range(K // S):
+                g_decs.replay()
+            d_end.record(stream)
+            torch.cuda.synchronize(dev)
+            step_ms.append(t_start.elapsed_time(t_end) / K)
+            dec_ms.append(d_start.elapsed_time(d_end) / K)
+    ms_step = float(statistics.median(step_ms))
     assert pa.device_error() == 0
 
     # ---- end to end through the public API: pinned host inputs -> device, step, result -> host
@@ -484,6 +487,21 @@ def run_ours(args):
     for _ in range(args.warmup):
         e2e_step(stream)
     torch.cuda.synchronize(dev)
+    # (a) eager: every step is the Python calls a user makes (argument checks, ctypes, tensor maps, launches)
+    e2e_eager = []
+    for _ in range(args.repeats):
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            e2e_step(stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_eager.append(e0.elapsed_time(e1) / K)
+    barrier()
+    e2e_ms = float(statistics.median(e2e_eager))
+    # (b) the same steps captured once in a CUDA graph and replayed (host work paid once, at capture)
     g_e2e = capture(lambda: [e2e_step(cap_stream) for _ in range(S)])
     g_e2e.replay()
     torch.cuda.synchronize(dev)
@@ -495,14 +513,16 @@ def run_ours(args):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    e2e_ms = e0.elapsed_time(e1) / K
+    e2e_graph_ms = e0.elapsed_time(e1) / K
     assert pa.device_error() == 0
     del g_write, g_dec, g_steps, g_decs, g_e2e
 
-    # ---- max over ranks, totals
-    kvb = kv_bytes(wl)
-    (ms_step, e2e_ms, dec_avg), (kv_all, seqs_all) = reduce_over_ranks(
-        [ms_step, e2e_ms, float(np.mean(dec_ms))], [kvb, B], ws, dev)
+    # ---- max over ranks, totals.  With shared prefixes the metric counts distinct cache rows (each shared
+    # block once); the logical bytes (every sequence's rows, shared ones again) are reported beside it.
+    kvb = unique_kv_bytes(wl)
+    kvb_logical = kv_bytes(wl)
+    (ms_step, e2e_ms, e2e_graph_ms, dec_avg), (kv_all, kvl_all, seqs_all) = reduce_over_ranks(
+        [ms_step, e2e_ms, e2e_graph_ms, float(statistics.median(dec_ms))], [kvb, kvb_logical, B], ws, dev)
     value = kv_all / (ms_step * 1e-3) / 1e9
     e2e_value = kv_all / (e2e_ms * 1e-3) / 1e9
 
@@ -523,22 +543,32 @@ def run_ours(args):
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": str(c["dtype"]), "data": "synthetic",
             "config": {"workload": WORKLOAD_TEXT.get(args.workload, args.workload), "global_batch": int(seqs_all),
+                       "block_size": int(c["block_size"]),
                        "parallelism": f"dp{ws} (independent replicas)", "l2": "inputs larger than L2 (no flush)",
-                       "decode_grid": grid},
+                       "decode_grid": grid, "repeats": args.repeats,
+                       "ms_per_step_repeats": step_ms},
             "tokens_per_s": seqs_all / (ms_step * 1e-3),
             "pct_hbm_peak": {"of_measured": value / ws / peak if peak_kind == "measured" else None,
                              "of_nominal_8000": value / ws / 8000.0},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_ms},
+                    "ms_per_step": e2e_ms,
+                    "how": "eager: per step, pinned H2D copies of q, new K/V, slots, block tables and lengths, "
+                           "then binding.write_kv and binding.decode (argument checks, ctypes, tensor-map "
+                           "encode, launch), then D2H of out; median of repeats",
+                    "graph_replay": {"value": kv_all / (e2e_graph_ms * 1e-3) / 1e9, "ms_per_step": e2e_graph_ms}},
             "roofline": {"bound": "hbm", "kernel": "pa_decode (one kernel: gather, attention, split-K merge)",
                          "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "algorithmic_bytes": alg,
-                         "avg_launch_ms": dec_avg,
-                         "timing": "decode-only graph replays, same launch count, right after the timed region"},
+                         "avg_launch_ms": dec_avg, "avg_launch_ms_repeats": dec_ms,
+                         "timing": "decode-only graph replays, same launch count, right after each timed loop; "
+                                   "median of repeats"},
             "gpu_launches": launches_per_step * K,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
         }
+        if kvl_all != kv_all:
+            line["logical_gbs"] = kvl_all / (ms_step * 1e-3) / 1e9
+            line["config"]["kv_bytes"] = {"unique": int(kv_all), "logical": int(kvl_all)}
         print(json.dumps(line), flush=True)
     if ws > 1:
         dist.destroy_process_group()
@@ -584,20 +614,25 @@ def run_prefill(args):
     for _ in range(3):
         g_step.replay()
     torch.cuda.synchronize(dev)
-    e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    step_ms, pf_ms = [], []
     with ClockSampler(0) as clk:
-        e[0].record(stream)
-        for _ in range(K):
-            g_step.replay()
-        e[1].record(stream)
-        e[2].record(stream)
-        for _ in range(K):
-            g_pf.replay()
-        e[3].record(stream)
-        torch.cuda.synchronize(dev)
+        for _ in range(args.repeats):
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            torch.cuda.synchronize(dev)
+            e[0].record(stream)
+            for _ in range(K):
+                g_step.replay()
+            e[1].record(stream)
+            e[2].record(stream)
+            for _ in range(K):
+                g_pf.replay()
+            e[3].record(stream)
+            torch.cuda.synchronize(dev)
+            step_ms.append(e[0].elapsed_time(e[1]) / K)
+            pf_ms.append(e[2].elapsed_time(e[3]) / K)
     assert pa.device_error() == 0
-    ms_step = e[0].elapsed_time(e[1]) / K
-    ms_pf = e[2].elapsed_time(e[3]) / K
+    ms_step = float(statistics.median(step_ms))
+    ms_pf = float(statistics.median(pf_ms))
 
     # ---- end to end through the public API: pinned host inputs -> device, step, result -> host
     pin = lambda t: t.pin_memory()
@@ -618,6 +653,13 @@ def run_prefill(args):
     for _ in range(args.warmup):
         e2e_step(stream)
     torch.cuda.synchronize(dev)
+    e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e4.record(stream)
+    for _ in range(K):
+        e2e_step(stream)          # eager: the binding calls a user makes, every step
+    e5.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e4.elapsed_time(e5) / K
     g_e2e = capture(lambda: e2e_step(cs))
     g_e2e.replay()
     torch.cuda.synchronize(dev)
@@ -627,7 +669,7 @@ def run_prefill(args):
         g_e2e.replay()
     e5.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e4.elapsed_time(e5) / K
+    e2e_graph_ms = e4.elapsed_time(e5) / K
     assert pa.device_error() == 0
     del g_step, g_pf, g_e2e
     fl = prefill_flops(wl)
@@ -642,14 +684,16 @@ def run_prefill(args):
         "metric": PREFILL_METRIC, "value": fl / (ms_step * 1e-3) / 1e12,
         "unit": "TFLOP/s", "n_gpus": 1, "steps": K, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": str(c["dtype"]),
-        "data": "synthetic", "config": {"workload": WORKLOAD_TEXT["prefill"], "flops_per_step": fl},
+        "data": "synthetic", "config": {"workload": WORKLOAD_TEXT["prefill"], "flops_per_step": fl,
+                                        "repeats": args.repeats, "ms_per_step_repeats": step_ms},
         "roofline": {"bound": "tensor", "kernel": "pa_prefill_chunk (tcgen05/TMEM, TMA)",
                      "achieved": fl / (ms_pf * 1e-3) / 1e12, "peak": burst, "peak_kind": kind + " burst",
                      "unit": "TFLOP/s", "frac": fl / (ms_pf * 1e-3) / 1e12 / burst,
                      "frac_of_sustained": fl / (ms_pf * 1e-3) / 1e12 / sustained, "traffic": pf_traffic,
-                     "avg_launch_ms": ms_pf},
+                     "avg_launch_ms": ms_pf, "avg_launch_ms_repeats": pf_ms},
         "e2e": {"value": fl / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "how": "eager binding calls every step",
+                "graph_replay": {"value": fl / (e2e_graph_ms * 1e-3) / 1e12, "ms_per_step": e2e_graph_ms}},
         "cpu_baseline": cpu,
         "gpu_launches": 2 * K,
         "clocks": clk.summary(),
@@ -846,6 +890,8 @@ def main():
     ap.add_argument("--workload", default="qwen_decode", choices=sorted(WORKLOAD_TEXT))
     ap.add_argument("--num-partitions", type=int, default=0, help="decode CTAs (0 = fill the GPU)")
     ap.add_argument("--steps-per-graph", type=int, default=10, help="whole steps captured per CUDA graph")
+    ap.add_argument("--repeats", type=int, default=5, help="timed K-step loops; the median is reported")
+    ap.add_argument("--block-size", type=int, default=None, help="override the workload's block size")
     ap.add_argument("--ref-budget", type=float, default=12.0, help="seconds of oracle time per reference sample")
     ap.add_argument("--ref-seqs", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
