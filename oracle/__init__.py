@@ -23,6 +23,11 @@ source pages, in float64 with numpy:
 * ``kv_quant``    - INT8 KV cache (Nano-vLLM-Ascend page, section 4.3; vLLM-Ascend
   page, section 5): per-(token, KV head) symmetric absmax codes with an fp32
   scale, written on append and dequantised for attention.
+* ``context_split`` - decode with each sequence's context split across devices
+  (vllm-ascend page, sections 1.1 and 3.1, DCP: every device attends over the
+  part of the KV cache it holds, the intermediate results are gathered and
+  combined): the block-interleaved split, each part's output and log-sum-exp,
+  and the log-sum-exp merge.
 * ``rope``        - rotary position embedding of new tokens' queries and keys
   fused with the KV write (Nano-vLLM-Ascend page, sections 3.1 and 5.1: the
   rotary multiply by per-position cos/sin tables, inverted by negating sin).
@@ -35,11 +40,14 @@ sharing, prefill row i == decode of the first prefix+i+1 tokens); for the
 rotary step, rotation closed forms, the page's inverse rule, angle addition,
 the relative-position property and torch complex multiplication; for the
 INT8 cache, the absmax code, the half-step error bound, exact grid rows and
-torch's int8 quantiser.  No function
+torch's int8 quantiser; for the context split, the shards partition every
+sequence (the page's 1000-token example over three ranks), torch's logsumexp
+and SDPA, and the merge against full attention (tests/test_oracle_context_split.py).
+No function
 here is "parity unpinned".
 """
 
-from . import attention, block_pool, brute, kv_quant, kv_write, rope  # noqa: F401
+from . import attention, block_pool, brute, context_split, kv_quant, kv_write, rope  # noqa: F401
 from .attention import decode_attention, gather_kv, prefill_attention, split_partials  # noqa: F401
 from .block_pool import OraclePool, replay  # noqa: F401
 from .kv_write import write_kv  # noqa: F401
