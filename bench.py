@@ -378,14 +378,15 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     wl = make_workload(args.workload, seed=None if rank == 0 else 1000 * rank + 1, block_size=args.block_size)
     c = wl.cfg
+    int8 = args.kv == "int8"
     _, bt, lens, sm, _ = pa.replay_ops(wl.ops, wl.num_blocks, c["block_size"], wl.free_order, wl.batch)
     maxL = int(lens.max())
     B, Hq, Hkv, D = wl.batch, c["num_q_heads"], c["num_kv_heads"], c["head_dim"]
-    grid, maxp, wsb = pa.decode_plan(B, Hq, Hkv, D, maxL, args.num_partitions)
+    plan = pa.decode_int8_plan if int8 else pa.decode_plan
+    grid, maxp, wsb = plan(B, Hq, Hkv, D, maxL, args.num_partitions)
 
     # device-resident inputs
-    kc = wl.k_cache0.to(dev)
-    vc = wl.v_cache0.to(dev)
+    NB, bs = wl.k_cache0.shape[0], c["block_size"]
     q = wl.q.to(dev)
     kn, vn = wl.k_new.to(dev), wl.v_new.to(dev)
     smd = torch.from_numpy(sm).to(dev)
@@ -394,13 +395,30 @@ def run_ours(args):
     out = torch.empty_like(q)
     work = torch.zeros(max(wsb, 256), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    if int8:  # the pool's prior contents, quantised into a fresh INT8 cache by the library's own write
+        kq = torch.zeros((NB, bs, Hkv, D), dtype=torch.int8, device=dev)
+        vq = torch.zeros_like(kq)
+        ksc = torch.zeros((NB, Hkv, bs), dtype=torch.float32, device=dev)
+        vsc = torch.zeros_like(ksc)
+        pa.write_kv_int8(wl.k_cache0.to(dev).view(NB * bs, Hkv, D), wl.v_cache0.to(dev).view(NB * bs, Hkv, D),
+                         torch.arange(NB * bs, dtype=torch.int64, device=dev), kq, vq, ksc, vsc)
 
-    def write_step():
-        pa.write_kv(kn, vn, smd, kc, vc, stream=stream)
+        def wr(st):
+            pa.write_kv_int8(kn, vn, smd, kq, vq, ksc, vsc, stream=st)
 
-    def decode_step():
-        pa.decode(q, kc, vc, btd, lensd, maxL, wl.scale, out=out, workspace=work, num_partitions=args.num_partitions,
-                  stream=stream)
+        def dec(st):
+            pa.decode_int8(q, kq, vq, ksc, vsc, btd, lensd, maxL, wl.scale, out=out, workspace=work,
+                           num_partitions=args.num_partitions, stream=st)
+    else:
+        kc = wl.k_cache0.to(dev)
+        vc = wl.v_cache0.to(dev)
+
+        def wr(st):
+            pa.write_kv(kn, vn, smd, kc, vc, stream=st)
+
+        def dec(st):
+            pa.decode(q, kc, vc, btd, lensd, maxL, wl.scale, out=out, workspace=work,
+                      num_partitions=args.num_partitions, stream=st)
 
     def barrier():
         if ws > 1:
@@ -409,8 +427,8 @@ def run_ours(args):
     # eager warm-up (first calls set kernel attributes), then CUDA graphs of several whole steps so
     # the timed loop measures the GPU, not Python launch overhead
     for _ in range(args.warmup):
-        write_step()
-        decode_step()
+        wr(stream)
+        dec(stream)
     torch.cuda.synchronize(dev)
     assert pa.device_error() == 0
 
@@ -425,16 +443,10 @@ def run_ours(args):
     K = args.steps
     if K % S:
         S = 1
-    # one graph = S whole steps (write_kv + decode each); a second graph = S decodes alone, for the
+    # one graph = S whole steps (write + decode each); a second graph = S decodes alone, for the
     # decode kernel's own average duration (the roofline denominator's time)
-    g_steps = capture(lambda: [(pa.write_kv(kn, vn, smd, kc, vc, stream=cap_stream),
-                                pa.decode(q, kc, vc, btd, lensd, maxL, wl.scale, out=out, workspace=work,
-                                          num_partitions=args.num_partitions, stream=cap_stream)) for _ in range(S)])
-    g_decs = capture(lambda: [pa.decode(q, kc, vc, btd, lensd, maxL, wl.scale, out=out, workspace=work,
-                                        num_partitions=args.num_partitions, stream=cap_stream) for _ in range(S)])
-    g_write = capture(lambda: pa.write_kv(kn, vn, smd, kc, vc, stream=cap_stream))
-    g_dec = capture(lambda: pa.decode(q, kc, vc, btd, lensd, maxL, wl.scale, out=out, workspace=work,
-                                      num_partitions=args.num_partitions, stream=cap_stream))
+    g_steps = capture(lambda: [(wr(cap_stream), dec(cap_stream)) for _ in range(S)])
+    g_decs = capture(lambda: [dec(cap_stream) for _ in range(S)])
     for _ in range(max(1, args.warmup // S)):
         g_steps.replay()
     torch.cuda.synchronize(dev)
@@ -479,9 +491,8 @@ def run_ours(args):
         smd.copy_(h_sm, non_blocking=True)
         btd.copy_(h_bt, non_blocking=True)
         lensd.copy_(h_lens, non_blocking=True)
-        pa.write_kv(kn, vn, smd, kc, vc, stream=st)
-        pa.decode(q, kc, vc, btd, lensd, maxL, wl.scale, out=out, workspace=work, num_partitions=args.num_partitions,
-                  stream=st)
+        wr(st)
+        dec(st)
         h_out.copy_(out, non_blocking=True)
 
     for _ in range(args.warmup):
@@ -515,12 +526,15 @@ def run_ours(args):
     barrier()
     e2e_graph_ms = e0.elapsed_time(e1) / K
     assert pa.device_error() == 0
-    del g_write, g_dec, g_steps, g_decs, g_e2e
+    del g_steps, g_decs, g_e2e
 
     # ---- max over ranks, totals.  With shared prefixes the metric counts distinct cache rows (each shared
     # block once); the logical bytes (every sequence's rows, shared ones again) are reported beside it.
     kvb = unique_kv_bytes(wl)
     kvb_logical = kv_bytes(wl)
+    if int8:  # one byte per element plus one fp32 scale per (token, KV head) row, for K and for V
+        kvb = kvb // (2 * D) * (D + 4)
+        kvb_logical = kvb_logical // (2 * D) * (D + 4)
     (ms_step, e2e_ms, e2e_graph_ms, dec_avg), (kv_all, kvl_all, seqs_all) = reduce_over_ranks(
         [ms_step, e2e_ms, e2e_graph_ms, float(statistics.median(dec_ms))], [kvb, kvb_logical, B], ws, dev)
     value = kv_all / (ms_step * 1e-3) / 1e9
@@ -529,7 +543,7 @@ def run_ours(args):
     peak, peak_kind = measured_hbm_peak()
     alg = kvb + io_bytes(wl)
     achieved = alg / (dec_avg * 1e-3) / 1e9
-    tr = NCU_TRAFFIC.get(args.workload)
+    tr = NCU_TRAFFIC.get(args.workload + ("_int8" if int8 else ""))
     traffic = tr["bytes"] if tr and tr.get("src") == kernel_source_hash(tr["files"]) else None
     launches_per_step = 2  # write_kv, decode (split-K merge inside)
     if rank == 0:
@@ -541,8 +555,9 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": K, "warmup": args.warmup,
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": str(c["dtype"]), "data": "synthetic",
+            "dtype": str(c["dtype"]) + ("+int8 cache" if int8 else ""), "data": "synthetic",
             "config": {"workload": WORKLOAD_TEXT.get(args.workload, args.workload), "global_batch": int(seqs_all),
+                       "kv_cache": "int8 codes + fp32 row scales" if int8 else str(c["dtype"]),
                        "block_size": int(c["block_size"]),
                        "parallelism": f"dp{ws} (independent replicas)", "l2": "inputs larger than L2 (no flush)",
                        "decode_grid": grid, "repeats": args.repeats,
@@ -556,7 +571,8 @@ def run_ours(args):
                            "then binding.write_kv and binding.decode (argument checks, ctypes, tensor-map "
                            "encode, launch), then D2H of out; median of repeats",
                     "graph_replay": {"value": kv_all / (e2e_graph_ms * 1e-3) / 1e9, "ms_per_step": e2e_graph_ms}},
-            "roofline": {"bound": "hbm", "kernel": "pa_decode (one kernel: gather, attention, split-K merge)",
+            "roofline": {"bound": "hbm", "kernel": ("pa_decode_int8" if int8 else "pa_decode") +
+                         " (one kernel: gather, attention, split-K merge)",
                          "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "algorithmic_bytes": alg,
                          "avg_launch_ms": dec_avg, "avg_launch_ms_repeats": dec_ms,
@@ -892,6 +908,8 @@ def main():
     ap.add_argument("--steps-per-graph", type=int, default=10, help="whole steps captured per CUDA graph")
     ap.add_argument("--repeats", type=int, default=5, help="timed K-step loops; the median is reported")
     ap.add_argument("--block-size", type=int, default=None, help="override the workload's block size")
+    ap.add_argument("--kv", choices=["bf16", "int8"], default="bf16",
+                    help="decode workloads: the cache format (int8 = codes + fp32 row scales)")
     ap.add_argument("--ref-budget", type=float, default=12.0, help="seconds of oracle time per reference sample")
     ap.add_argument("--ref-seqs", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")

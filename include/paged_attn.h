@@ -180,6 +180,42 @@ int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int
               void* out, void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Cascade decode over shared prefixes (P1 s2.1: blocks carry reference     */
+/* counts and forked sequences share their prefix blocks; P2 s4: block      */
+/* sharing for long contexts).  Same result as pa_decode, but each shared   */
+/* prefix block is read once for all sequences that share it:               */
+/*   1. pa_decode's kernel over every sequence's private suffix, tokens     */
+/*      seq_prefix_len[b] .. context_lens[b]-1, leaving (out, log-sum-exp);  */
+/*   2. one pass over each group's shared prefix with the query rows of all */
+/*      its members at once (warp MMA), merged with step 1 by the            */
+/*      log-sum-exp rule into out.                                          */
+/* Groups: num_groups consecutive ranges of the batch, group g = sequences  */
+/* group_start[g] .. group_start[g+1]-1 (int32 [num_groups+1], device,      */
+/* non-decreasing); sequences outside every range, and groups whose prefix  */
+/* is 0, get plain decode.  seq_prefix_len: int32 [batch], device: the      */
+/* shared prefix length of each sequence's group (0 outside groups), a      */
+/* multiple of 16, at most its context length; every member of a group     */
+/* has the same value and maps its first seq_prefix_len/block_size block-   */
+/* table entries to the same physical blocks (the prefix is read through    */
+/* the group's first member).  max_group_size / max_prefix_len: host upper  */
+/* bounds of group sizes and prefix lengths (they size the grid).           */
+/* Workspace: pa_decode_cascade_workspace_size() bytes, 256-byte aligned,   */
+/* zero-filled before first use; every completed call leaves its counters   */
+/* at zero.  Two launches on `stream`; same argument checks and return      */
+/* codes as pa_decode.  A prefix length that is not a multiple of 16 is     */
+/* rounded down and sets PA_ERRBIT_INDEX.                                   */
+/* ------------------------------------------------------------------------ */
+size_t pa_decode_cascade_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                                        int max_context_len, int num_partitions_or_0, int num_groups,
+                                        int max_group_size, int max_prefix_len);
+int pa_decode_cascade(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                      int max_blocks_per_seq, const int32_t* context_lens, int batch, int num_q_heads,
+                      int num_kv_heads, int head_dim, int block_size, int num_blocks, int max_context_len,
+                      float scale, int dtype, int num_groups, const int32_t* group_start,
+                      const int32_t* seq_prefix_len, int max_group_size, int max_prefix_len, void* workspace,
+                      size_t workspace_bytes, int num_partitions_or_0, void* out, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* Decode with library-owned scratch (no counterpart on the source pages).   */
 /* Same computation, arguments and results as pa_decode, but without a      */
 /* workspace argument: for callers that cannot allocate device memory where */
@@ -205,6 +241,104 @@ int pa_decode_static_scratch(const void* q, const void* k_cache, const void* v_c
                              int max_blocks_per_seq, const int32_t* context_lens, int batch, int num_q_heads,
                              int num_kv_heads, int head_dim, int block_size, int num_blocks, int max_context_len,
                              float scale, int dtype, int num_partitions_or_0, void* out, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* INT8 KV cache (P1 s4.3: KV-cache compression and INT8 in the tuning      */
+/* checklist; P2 s5: INT8 as the next throughput step once the accuracy of  */
+/* the attention scores is handled).  The pages fix no format; this one:   */
+/* every (token, KV head) row of head_dim values x is stored as head_dim    */
+/* int8 codes and one fp32 scale,                                           */
+/*   amax = max |x|, inv = 127 / amax, code = rint(x * inv) in [-127, 127],  */
+/*   scale = amax / 127                                                     */
+/* (fp32 IEEE division and multiply, round half to even; amax 0 gives zero  */
+/* codes and scale 0).  A row dequantises to code * scale.  Rows whose amax */
+/* is below 127 / FLT_MAX (about 3.7e-37; only bf16 inputs can have them)   */
+/* are outside the format.                                                  */
+/* Layout: codes k_codes, v_codes int8 [num_blocks][block_size][Hkv][D]     */
+/* (the 16-bit caches' layout, one byte per element); scales k_scales,      */
+/* v_scales fp32 [num_blocks][Hkv][block_size] (the 16 scales of a 16-token */
+/* chunk of one head are one 64-byte run).  All four 16-byte aligned.       */
+/*                                                                          */
+/* pa_write_kv_int8: for every t with slot = slot_mapping[t] >= 0,           */
+/* quantise k[t][h] and v[t][h] (16-bit, [num_tokens][Hkv][D], dtype) into  */
+/* row slot of the codes and entry [slot/bs][h][slot%bs] of the scales.     */
+/* Same argument rules as pa_write_kv; a slot >= num_blocks*block_size      */
+/* writes nothing and sets PA_ERRBIT_INDEX.  Signals its dependents at      */
+/* entry (a following pa_decode_int8 may start its set-up early).           */
+/* ------------------------------------------------------------------------ */
+int pa_write_kv_int8(const void* k, const void* v, const int64_t* slot_mapping, int num_tokens, void* k_codes,
+                     void* v_codes, float* k_scales, float* v_scales, int num_blocks, int block_size,
+                     int num_kv_heads, int head_dim, int dtype, void* stream);
+
+/* Copy-on-write for the INT8 cache: for each pair i, block pairs[2i+1] of  */
+/* the codes and of the scales becomes a bitwise copy of block pairs[2i].   */
+int pa_copy_blocks_int8(const int32_t* pairs, int num_pairs, void* k_codes, void* v_codes, float* k_scales,
+                        float* v_scales, int num_blocks, int block_size, int num_kv_heads, int head_dim,
+                        void* stream);
+
+/* pa_decode_int8: pa_decode over the INT8 cache.  Computes                 */
+/*   out[b][h] = sum_t softmax_t(scale * <q[b][h], Kd_b[t]>) Vd_b[t]        */
+/* with Kd, Vd the dequantised rows (code * scale) of KV head h/G; q and    */
+/* out are 16-bit (dtype), all scores, softmax state and accumulators fp32. */
+/* Same work split, workspace rules, argument checks and return codes as    */
+/* pa_decode; the workspace size comes from pa_decode_int8_workspace_size   */
+/* (or pa_decode_int8_plan).  Internally q is rounded to fp16 after an      */
+/* exact power-of-two prescale (its largest magnitude lands in [2^14,       */
+/* 2^15)), and the softmax weights enter the V product as fp16 in [0, 1];   */
+/* q elements below 2^-28 of the group's largest lose precision.            */
+/* ------------------------------------------------------------------------ */
+int pa_decode_int8_plan(int batch, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len,
+                        int num_partitions_or_0, int* grid_out, int* max_pieces_out, size_t* workspace_bytes_out);
+size_t pa_decode_int8_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                                     int max_context_len, int num_partitions_or_0);
+int pa_decode_int8(const void* q, const void* k_codes, const void* v_codes, const float* k_scales,
+                   const float* v_scales, const int32_t* block_tables, int max_blocks_per_seq,
+                   const int32_t* context_lens, int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                   int block_size, int num_blocks, int max_context_len, float scale, int dtype, void* workspace,
+                   size_t workspace_bytes, int num_partitions_or_0, void* out, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Decode with the context split across devices (P3 s1.1 / s3.1 DCP: each  */
+/* device attends over the part of the KV cache it holds; the intermediate */
+/* results are gathered from all devices (AllGather) and combined).         */
+/* Split rule (the pages give none): logical block j of every sequence      */
+/* lives on rank j mod world; on its rank it is local block j / world, so a */
+/* rank's blocks form an ordinary paged sequence whose blocks are full but  */
+/* the last.  The caller keeps one pool and cache per rank and gathers the  */
+/* per-rank results with its collective library (e.g. NCCL all-gather).     */
+/*                                                                          */
+/* pa_dcp_owner: rank holding token `position` (PA_ERR_INVALID on bad args).*/
+/* pa_dcp_local_position: the token's index in its rank's local sequence.  */
+/* pa_dcp_local_lens: host int32 arrays; local_lens_out[b] = tokens of      */
+/* sequence b (context_lens[b] in all) held by `rank`.                      */
+/* ------------------------------------------------------------------------ */
+int pa_dcp_owner(int64_t position, int block_size, int world);
+int64_t pa_dcp_local_position(int64_t position, int block_size, int world);
+int pa_dcp_local_lens(const int32_t* context_lens, int batch, int block_size, int world, int rank,
+                      int32_t* local_lens_out);
+
+/* pa_decode_lse: pa_decode that also writes lse_out, fp32 [batch][Hq]       */
+/* (device, 4-byte aligned): lse = ln sum_t exp(scale * <q[b][h], K_b[t]>)   */
+/* over the sequence's context_lens[b] tokens, -inf when it has none (out   */
+/* is then 0).  With a rank's local cache, block tables and local lengths,  */
+/* (out, lse) is that rank's intermediate result.  Same rules and return    */
+/* codes as pa_decode; lse_out NULL with batch > 0 is PA_ERR_INVALID.       */
+int pa_decode_lse(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                  int max_blocks_per_seq, const int32_t* context_lens, int batch, int num_q_heads,
+                  int num_kv_heads, int head_dim, int block_size, int num_blocks, int max_context_len, float scale,
+                  int dtype, void* workspace, size_t workspace_bytes, int num_partitions_or_0, void* out,
+                  float* lse_out, void* stream);
+
+/* pa_merge_attn_states: combine num_parts intermediate results.            */
+/* parts: 16-bit (dtype) [num_parts][batch][num_heads][head_dim], lses:     */
+/* fp32 [num_parts][batch][num_heads], out: [batch][num_heads][head_dim],   */
+/* all device.  out = sum_r exp(lse_r - M) parts_r / sum_r exp(lse_r - M),  */
+/* M = max_r lse_r, accumulated in fp32 and rounded to nearest even; a part */
+/* with lse -inf adds nothing (its bytes are not read); a row whose parts   */
+/* are all -inf is 0.  parts and out 16-byte aligned; out must not overlap  */
+/* parts.  One kernel launch on `stream`.                                   */
+int pa_merge_attn_states(const void* parts, const float* lses, int num_parts, int batch, int num_heads, int head_dim,
+                         int dtype, void* out, void* stream);
 
 /* ------------------------------------------------------------------------ */
 /* Chunked prefill (P3 s1.1 / s3.1 PCP: prefill cut into chunks on one       */

@@ -12,6 +12,7 @@ Calls (see the header for exact semantics):
 * ``rope_write_kv``  - rotary embedding of new tokens' q and k, fused with the K/V cache write
 * ``decode``         - one-token paged attention, split-K with the merge in the same kernel
 * ``prefill_chunk``  - causal chunked-prefill attention over the paged cache
+* ``write_kv_int8``, ``decode_int8``, ``copy_blocks_int8`` - the same over an INT8 cache (codes + fp32 scales)
 * ``BlockPool``      - host block pool: blocks, block tables, reference counts
 """
 
@@ -25,7 +26,9 @@ import numpy as np
 __all__ = ["PagedAttnError", "PoolOutOfBlocks", "BlockPool", "write_kv", "copy_blocks", "rope_write_kv", "decode",
            "decode_plan",
            "decode_static_scratch",
-           "prefill_chunk", "device_error", "lib", "LIB_PATH", "replay_ops", "version"]
+           "prefill_chunk", "device_error", "lib", "LIB_PATH", "replay_ops", "version",
+           "write_kv_int8", "copy_blocks_int8", "decode_int8", "decode_int8_plan", "decode_lse", "merge_attn_states",
+           "decode_cascade", "decode_cascade_workspace_size"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpaged_attn.so")
 
@@ -59,6 +62,21 @@ _SIGS = {
     "pa_decode_static_scratch": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp, _vp]),
     "pa_prefill_chunk": (_i, [_vp, _vp, _i, _i, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _vp]),
     "pa_device_error": (_i, [_ip]),
+    "pa_decode_lse": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _sz, _i, _vp, _vp,
+                           _vp]),
+    "pa_decode_cascade_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
+    "pa_decode_cascade": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp, _vp, _i, _i,
+                               _vp, _sz, _i, _vp, _vp]),
+    "pa_merge_attn_states": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
+    "pa_dcp_owner": (_i, [_i64, _i, _i]),
+    "pa_dcp_local_position": (_i64, [_i64, _i, _i]),
+    "pa_dcp_local_lens": (_i, [_i32p, _i, _i, _i, _i, _i32p]),
+    "pa_write_kv_int8": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
+    "pa_copy_blocks_int8": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
+    "pa_decode_int8_plan": (_i, [_i, _i, _i, _i, _i, _i, _ip, _ip, ctypes.POINTER(_sz)]),
+    "pa_decode_int8_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "pa_decode_int8": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _sz, _i,
+                            _vp, _vp]),
     "pa_pool_create": (_vp, [_i, _i, _i32p]),
     "pa_pool_destroy": (None, [_vp]),
     "pa_seq_alloc": (_i, [_vp, _i64, _i]),
@@ -318,6 +336,167 @@ def prefill_chunk(q, query_start_loc, k_cache, v_cache, block_tables, context_le
                                 _ptr(block_tables), int(block_tables.shape[1]), _ptr(context_lens), B, Hq, Hkv, D,
                                 bs, NB, float(scale), _dtype_code(q), _ptr(out), _stream_handle(stream)),
            "pa_prefill_chunk")
+    return out
+
+
+def decode_lse(q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float, out=None,
+               lse=None, workspace=None, num_partitions: int = 0, stream=None):
+    """pa_decode that also returns the log-sum-exp of each (sequence, head)'s scores: (out [B, Hq, D],
+    lse float32 [B, Hq]); lse is -inf (and out 0) for a sequence with no tokens."""
+    torch = _torch()
+    _contig(q, k_cache, v_cache, block_tables, context_lens, out, lse, workspace)
+    B, Hq, D = _decode_args(q, k_cache, v_cache, block_tables, context_lens, out)
+    NB, bs, Hkv, _ = k_cache.shape
+    if lse is not None:
+        _want("lse", lse, dtype=torch.float32, shape=(B, Hq))
+    _device(stream, q, k_cache, v_cache, block_tables, context_lens, out, lse, workspace)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _, _, need = decode_plan(B, Hq, Hkv, D, max_context_len, num_partitions)
+    if workspace is None:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.pa_decode_lse(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), int(block_tables.shape[1]),
+                             _ptr(context_lens), B, Hq, Hkv, D, bs, NB, int(max_context_len), float(scale),
+                             _dtype_code(q), _ptr(workspace), ws_bytes, int(num_partitions), _ptr(out), _ptr(lse),
+                             _stream_handle(stream)), "pa_decode_lse")
+    return out, lse
+
+
+def decode_cascade_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_groups,
+                                  max_group_size, max_prefix_len, num_partitions=0) -> int:
+    n = lib.pa_decode_cascade_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                                             num_partitions, num_groups, max_group_size, max_prefix_len)
+    if n == 0:
+        raise PagedAttnError(-1, "pa_decode_cascade_workspace_size")
+    return n
+
+
+def decode_cascade(q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float, group_start,
+                   seq_prefix_len, max_group_size: int, max_prefix_len: int, out=None, workspace=None,
+                   num_partitions: int = 0, stream=None):
+    """Decode with every shared prefix read once for all its sharers.  group_start int32 [G+1] (device):
+    group g = sequences group_start[g] .. group_start[g+1]-1; seq_prefix_len int32 [B] (device): each
+    sequence's shared prefix length (a multiple of 16; 0 = none).  Returns out [B, Hq, D]."""
+    torch = _torch()
+    _contig(q, k_cache, v_cache, block_tables, context_lens, group_start, seq_prefix_len, out, workspace)
+    B, Hq, D = _decode_args(q, k_cache, v_cache, block_tables, context_lens, out)
+    NB, bs, Hkv, _ = k_cache.shape
+    _want("group_start", group_start, dtype=torch.int32, ndim=1)
+    _want("seq_prefix_len", seq_prefix_len, dtype=torch.int32, shape=(B,))
+    ngroups = max(int(group_start.shape[0]) - 1, 0)
+    _device(stream, q, k_cache, v_cache, block_tables, context_lens, group_start, seq_prefix_len, out, workspace)
+    if out is None:
+        out = torch.empty_like(q)
+    need = decode_cascade_workspace_size(B, Hq, Hkv, D, max_context_len, ngroups, max_group_size, max_prefix_len,
+                                         num_partitions)
+    if workspace is None:  # zero-filled once; every call leaves its counters zeroed again
+        workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.pa_decode_cascade(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                 int(block_tables.shape[1]), _ptr(context_lens), B, Hq, Hkv, D, bs, NB,
+                                 int(max_context_len), float(scale), _dtype_code(q), ngroups, _ptr(group_start),
+                                 _ptr(seq_prefix_len), int(max_group_size), int(max_prefix_len), _ptr(workspace),
+                                 ws_bytes, int(num_partitions), _ptr(out), _stream_handle(stream)),
+           "pa_decode_cascade")
+    return out
+
+
+def merge_attn_states(parts, lses, out=None, stream=None):
+    """parts [P, B, H, D] (bf16/fp16), lses float32 [P, B, H] -> out [B, H, D]: the softmax-weighted
+    combination of the parts by their log-sum-exps."""
+    torch = _torch()
+    _contig(parts, lses, out)
+    _want("parts", parts, ndim=4)
+    P, B, H, D = (int(x) for x in parts.shape)
+    _want("lses", lses, dtype=torch.float32, shape=(P, B, H))
+    if out is not None:
+        _want("out", out, dtype=parts.dtype, shape=(B, H, D))
+    _device(stream, parts, lses, out)
+    if out is None:
+        out = torch.empty((B, H, D), dtype=parts.dtype, device=parts.device)
+    _check(lib.pa_merge_attn_states(_ptr(parts), _ptr(lses), P, B, H, D, _dtype_code(parts), _ptr(out),
+                                    _stream_handle(stream)), "pa_merge_attn_states")
+    return out
+
+
+# ---------------------------------------------------------------------------------------------- INT8 cache
+def _int8_caches(k_codes, v_codes, k_scales, v_scales):
+    """Codes int8 [NB, bs, Hkv, D] (both alike), scales float32 [NB, Hkv, bs] (both alike); returns the shape."""
+    torch = _torch()
+    _want("k_codes", k_codes, dtype=torch.int8, ndim=4)
+    _want("v_codes", v_codes, dtype=torch.int8, shape=k_codes.shape)
+    NB, bs, Hkv, D = (int(x) for x in k_codes.shape)
+    _want("k_scales", k_scales, dtype=torch.float32, shape=(NB, Hkv, bs))
+    _want("v_scales", v_scales, dtype=torch.float32, shape=(NB, Hkv, bs))
+    return NB, bs, Hkv, D
+
+
+def write_kv_int8(k, v, slot_mapping, k_codes, v_codes, k_scales, v_scales, stream=None) -> None:
+    """Quantise k, v [T, Hkv, D] (bf16/fp16) into the INT8 cache rows of slot_mapping int64 [T] (-1 = skip)."""
+    torch = _torch()
+    _contig(k, v, slot_mapping, k_codes, v_codes, k_scales, v_scales)
+    NB, bs, Hkv, D = _int8_caches(k_codes, v_codes, k_scales, v_scales)
+    _want("k", k, ndim=3)
+    T = int(k.shape[0])
+    _dtype_code(k)
+    _want("k", k, shape=(T, Hkv, D))
+    _want("v", v, dtype=k.dtype, shape=(T, Hkv, D))
+    _want("slot_mapping", slot_mapping, dtype=torch.int64, shape=(T,))
+    _device(stream, k, v, slot_mapping, k_codes, v_codes, k_scales, v_scales)
+    _check(lib.pa_write_kv_int8(_ptr(k), _ptr(v), _ptr(slot_mapping), T, _ptr(k_codes), _ptr(v_codes),
+                                _ptr(k_scales), _ptr(v_scales), NB, bs, Hkv, D, _dtype_code(k),
+                                _stream_handle(stream)), "pa_write_kv_int8")
+
+
+def copy_blocks_int8(pairs, k_codes, v_codes, k_scales, v_scales, stream=None) -> None:
+    """pairs int32 [n, 2] (src, dst) on the device: copy whole blocks of the INT8 codes and scales."""
+    torch = _torch()
+    _contig(pairs, k_codes, v_codes, k_scales, v_scales)
+    NB, bs, Hkv, D = _int8_caches(k_codes, v_codes, k_scales, v_scales)
+    _want("pairs", pairs, dtype=torch.int32, ndim=2)
+    _want("pairs", pairs, shape=(pairs.shape[0], 2))
+    _device(stream, pairs, k_codes, v_codes, k_scales, v_scales)
+    _check(lib.pa_copy_blocks_int8(_ptr(pairs), int(pairs.shape[0]), _ptr(k_codes), _ptr(v_codes), _ptr(k_scales),
+                                   _ptr(v_scales), NB, bs, Hkv, D, _stream_handle(stream)), "pa_copy_blocks_int8")
+
+
+def decode_int8_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_partitions=0):
+    """(grid, max_pieces, workspace_bytes) of decode over the INT8 cache on the current device."""
+    gr, mp, ws = ctypes.c_int(), ctypes.c_int(), ctypes.c_size_t()
+    _check(lib.pa_decode_int8_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_partitions,
+                                   ctypes.byref(gr), ctypes.byref(mp), ctypes.byref(ws)), "pa_decode_int8_plan")
+    return gr.value, mp.value, ws.value
+
+
+def decode_int8(q, k_codes, v_codes, k_scales, v_scales, block_tables, context_lens, max_context_len: int,
+                scale: float, out=None, workspace=None, num_partitions: int = 0, stream=None):
+    """Decode over the INT8 cache: q [B, Hq, D] bf16/fp16; returns out [B, Hq, D] in q's dtype."""
+    torch = _torch()
+    _contig(q, k_codes, v_codes, k_scales, v_scales, block_tables, context_lens, out, workspace)
+    NB, bs, Hkv, D = _int8_caches(k_codes, v_codes, k_scales, v_scales)
+    _want("q", q, ndim=3)
+    _dtype_code(q)
+    B, Hq = int(q.shape[0]), int(q.shape[1])
+    _want("q", q, shape=(B, Hq, D))
+    _want("block_tables", block_tables, dtype=torch.int32, ndim=2)
+    _want("block_tables", block_tables, shape=(B, block_tables.shape[1]))
+    _want("context_lens", context_lens, dtype=torch.int32, shape=(B,))
+    if out is not None:
+        _want("out", out, dtype=q.dtype, shape=q.shape)
+    _device(stream, q, k_codes, v_codes, k_scales, v_scales, block_tables, context_lens, out, workspace)
+    if out is None:
+        out = torch.empty_like(q)
+    _, _, need = decode_int8_plan(B, Hq, Hkv, D, max_context_len, num_partitions)
+    if workspace is None:  # zero-filled once; every call leaves it zeroed again
+        workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.pa_decode_int8(_ptr(q), _ptr(k_codes), _ptr(v_codes), _ptr(k_scales), _ptr(v_scales),
+                              _ptr(block_tables), int(block_tables.shape[1]), _ptr(context_lens), B, Hq, Hkv, D, bs,
+                              NB, int(max_context_len), float(scale), _dtype_code(q), _ptr(workspace), ws_bytes,
+                              int(num_partitions), _ptr(out), _stream_handle(stream)), "pa_decode_int8")
     return out
 
 

@@ -53,6 +53,7 @@ namespace {
 using namespace pa;
 
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kChunk = 16;  // tokens per chunk = rows per TMA box
 constexpr int kPlanRing = 8;  // producer plan ring slots
 constexpr int kMaxPieces = 32;  // pieces per segment the epilogue merges with precomputed weights
@@ -62,6 +63,10 @@ static_assert(kPlanRing > kLookahead, "plan ring must hold the stages in flight 
 struct DecodeParams {
   const void* q;
   void* out;
+  const float* k_scales;  // int8 cache only: fp32 [num_blocks][Hkv][block_size]
+  const float* v_scales;
+  float* lse;             // optional fp32 [batch][Hq]: ln sum_t exp(scale <q, K_t>) (-inf for an empty context)
+  const int32_t* ctx_start;  // optional int32 [batch]: tokens skipped at the head of each context (multiple of 16)
   const int32_t* block_tables;
   const int32_t* context_lens;
   int* ws_cnt;        // [B*Hkv] pieces of each segment written so far (zero between calls)
@@ -87,16 +92,22 @@ struct StageMeta {
   int b, g, tok0, ntok, flags, nchunk, c0, npieces;
 };
 
-template <int D, int G, int NW, int NSTAGES, bool MMA>
+// Shared-memory layout of one CTA.  Q8: the cache holds int8 codes (one byte per element) and per-token
+// fp32 scales, which each stage carries next to the codes.
+template <int D, int G, int NW, int NSTAGES, bool MMA, bool Q8 = false>
 struct Layout {
   static constexpr int TOK = NW * 32;             // tokens per stage
   static constexpr int CPS = TOK / kChunk;        // chunks (16-row boxes) per stage
-  static constexpr int HALVES = D / 64;           // 128-byte column boxes per row
-  static constexpr int STAGE_BYTES = TOK * D * 2; // K (or V) bytes per stage
+  static constexpr int ROWB = Q8 ? D : 2 * D;     // bytes of one (token, KV head) cache row
+  static constexpr int BOXB = ROWB >= 128 ? 128 : ROWB;  // bytes per row of one TMA box
+  static constexpr int HALVES = ROWB / BOXB;      // column boxes per row
+  static constexpr int STAGE_BYTES = TOK * ROWB;  // K (or V) bytes per stage
   static constexpr int QSLOT = G * D * 2;         // the group's q rows
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + NSTAGES * STAGE_BYTES;
-  static constexpr int QS_OFF = V_OFF + NSTAGES * STAGE_BYTES;
+  static constexpr int SK_OFF = V_OFF + NSTAGES * STAGE_BYTES;                // fp32 K scales [NSTAGES][TOK] (Q8)
+  static constexpr int SV_OFF = SK_OFF + (Q8 ? NSTAGES * TOK * 4 : 0);        // fp32 V scales [NSTAGES][TOK] (Q8)
+  static constexpr int QS_OFF = SV_OFF + (Q8 ? NSTAGES * TOK * 4 : 0);
   static constexpr int META_OFF = QS_OFF + NSTAGES * QSLOT;
   static constexpr int PLAN_OFF = META_OFF + NSTAGES * (int)sizeof(StageMeta);  // producer plan ring
   static constexpr int PLAN_BYTES = kPlanRing * ((int)sizeof(StageMeta) + 8 * 4);
@@ -128,6 +139,17 @@ __device__ __forceinline__ uint32_t swz_addr(uint32_t base, int r, int d) {
   const int half = d >> 6;
   const int chunk = (d >> 3) & 7;
   return base + half * (TOK * 128) + r * 128 + ((chunk ^ (r & 7)) << 4) + ((d & 7) << 1);
+}
+
+// Address of byte `byte` (a multiple of 4 within its 16-byte chunk is what callers use) of row r of an
+// int8 stage buffer of ROWB-byte rows written by TMA: 128-byte rows carry the 128-byte swizzle (16-byte
+// chunk index XOR r%8), 64-byte rows the 64-byte swizzle (chunk index XOR (r/2)%4).
+template <int ROWB>
+__device__ __forceinline__ uint32_t swz8_addr(uint32_t base, int r, int byte) {
+  if constexpr (ROWB == 128)
+    return base + r * 128 + ((((byte >> 4) ^ (r & 7)) & 7) << 4) + (byte & 15);
+  else
+    return base + r * 64 + ((((byte >> 4) ^ (r >> 1)) & 3) << 4) + (byte & 15);
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
@@ -483,6 +505,273 @@ struct MmaConsumer {
   }
 };
 
+// ------------------------------------------------------------------ int8-cache consumer (every G)
+// Scores and PV on mma.m16n8k16 with fp16 operands and tokens as the M rows, so a group of G <= 8 heads
+// fills one n-tile of 8 columns instead of padding 16 rows:
+//   S^T[t][h] = sum_d code_k[t][d] q[h][d]           (A = K codes, B = q^T)
+//   O^T[d][h] += sum_t code_v[t][d] P'[h][t]          (A = V^T codes, B = P'^T)
+// The codes become fp16 exactly (|code| <= 127): biased by 128 (XOR 0x80), two bytes are placed under
+// the fp16 exponent of 1024 by one byte permute, and 1152 is subtracted (HSUB2).  The head_dim order
+// inside a k-step is permuted so that every lane's operand bytes are contiguous: the sum over d does not
+// depend on the order as long as q uses the same one, and O^T's row order is undone when it is stored.
+// q is converted to fp16 once per piece after an exact power-of-two prescale that puts its largest
+// magnitude in [2^14, 2^15); the prescale is undone in the score scale.  The dequantisation costs one
+// multiply per token and head for K, s = scale_k[t] * (q . code_k[t]), and folds scale_v into the
+// softmax weight that enters PV: with m the running score maximum, u = (s - m) + log2(scale_v[t]) (formed
+// relative to m so that fp32 keeps the scale's bits however large the logits) and P' = 2^(u - rho), rho
+// the running maximum of u, so the largest weight of a head is exactly 1 and every P' lies in [0, 1]
+// (fp16 holds it to 2^-11 relative).  O is kept relative to (m, rho): O relative to m is O * 2^rho; the
+// sum l is relative to m; both are rescaled when a maximum moves.
+template <int D, int G, int NW, int NSTAGES>
+struct Q8Consumer {
+  using LY = Layout<D, G, NW, NSTAGES, true, true>;
+  static constexpr int NT = (G + 7) / 8;  // n-tiles of 8 heads
+  static constexpr int KS = D / 16;       // k-steps of QK^T, and m-tiles (16 rows of d) of O^T
+  static constexpr int QB = D / 4;        // bytes of a K row one lane reads (its quarter of the row)
+  uint32_t qb[NT][KS][2];                 // B fragments of q^T (fp16, prescaled)
+  float o[NT][KS][4];                     // O^T relative to (m, rho): rows d (permuted), columns heads
+  float m[NT][2], l[NT][2];               // heads 8nt + 2(lane%4) + {0,1}; l is this lane's partial sum
+  float rho[NT][2];                       // running max of (s - m) + log2(scale_v) per head
+  float qs;                               // scale * log2(e) / prescale
+
+  static __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+  }
+  // fp16x2 of bytes 0,1 (lo) or 2,3 (hi) of a word of codes already XORed with 0x80808080
+  static __device__ __forceinline__ uint32_t to_h2(uint32_t xb, uint32_t sel) {
+    uint32_t h = prmt(xb, 0x64646464u, sel), d;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(h), "r"(0x64806480u));
+    return d;
+  }
+  static __device__ __forceinline__ void mma_f16(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                 uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+  static __device__ __forceinline__ uint32_t trans8x8(uint32_t a) {
+    uint32_t d;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+    return d;
+  }
+  static __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      m[nt][0] = m[nt][1] = -INFINITY;
+      rho[nt][0] = rho[nt][1] = -INFINITY;
+      l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+      for (int i = 0; i < KS; ++i) o[nt][i][0] = o[nt][i][1] = o[nt][i][2] = o[nt][i][3] = 0.f;
+    }
+  }
+
+  // The group's q rows (16-bit [G][D], element type DT) -> fp16 B fragments after the prescale.
+  template <int DT>
+  __device__ __forceinline__ void load_q(const uint8_t* qslot, float scale_log2, int lane) {
+    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qslot);
+    float amax = 0.f;
+    for (int i = lane; i < G * D / 2; i += 32) {
+      const float2 f = Elt<DT>::to_f2(q32[i]);
+      amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+    amax = warp_max(amax);
+    int e = 0;
+    if (amax > 0.f) {
+      int k;
+      frexpf(amax, &k);  // amax in [2^(k-1), 2^k)
+      e = 15 - k;
+      e = e < -60 ? -60 : (e > 60 ? 60 : e);
+    }
+    const float f = __int_as_float((127 + e) << 23), finv = __int_as_float((127 - e) << 23);
+    qs = scale_log2 * finv;
+    const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int h = nt * 8 + g;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        uint32_t b0 = 0u, b1 = 0u;
+        if (h < G) {
+          const int d0 = c * QB + 4 * ks;
+          const float2 x01 = Elt<DT>::to_f2(q32[(h * D + d0) / 2]);
+          const float2 x23 = Elt<DT>::to_f2(q32[(h * D + d0) / 2 + 1]);
+          b0 = pack_h2(x01.x * f, x01.y * f);
+          b1 = pack_h2(x23.x * f, x23.y * f);
+        }
+        qb[nt][ks][0] = b0;
+        qb[nt][ks][1] = b1;
+      }
+    }
+  }
+
+  // One 32-token tile: rows r0 .. r0+31 of the stage, nv of them valid.  skb/svb: the stage's scales.
+  __device__ __forceinline__ void tile(uint32_t kbase, uint32_t vbase, const float* skb, const float* svb, int r0,
+                                       int nv, int lane) {
+    const int g = lane >> 2, c = lane & 3;
+    // ---- S^T = K q^T: 2 m-tiles of 16 tokens x NT n-tiles of 8 heads
+    float s[2][NT][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) s[mt][nt][0] = s[mt][nt][1] = s[mt][nt][2] = s[mt][nt][3] = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      const int ta = r0 + 16 * mt + g, tb = ta + 8;
+      uint32_t ka[KS], kb[KS];
+#pragma unroll
+      for (int i = 0; i < QB / 16; ++i) {
+        const uint4 u = lds128(swz8_addr<LY::ROWB>(kbase, ta, c * QB + 16 * i));
+        const uint4 w = lds128(swz8_addr<LY::ROWB>(kbase, tb, c * QB + 16 * i));
+        ka[4 * i + 0] = u.x ^ 0x80808080u; ka[4 * i + 1] = u.y ^ 0x80808080u;
+        ka[4 * i + 2] = u.z ^ 0x80808080u; ka[4 * i + 3] = u.w ^ 0x80808080u;
+        kb[4 * i + 0] = w.x ^ 0x80808080u; kb[4 * i + 1] = w.y ^ 0x80808080u;
+        kb[4 * i + 2] = w.z ^ 0x80808080u; kb[4 * i + 3] = w.w ^ 0x80808080u;
+      }
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const uint32_t a0 = to_h2(ka[ks], 0x4140u), a2 = to_h2(ka[ks], 0x4342u);
+        const uint32_t a1 = to_h2(kb[ks], 0x4140u), a3 = to_h2(kb[ks], 0x4342u);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_f16(s[mt][nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
+      }
+    }
+    // ---- per-token K scales, mask, online softmax per head (column), fp32 in the log2 domain
+    float lsv[2][2];  // log2 of the V scale of this lane's rows (-inf for invalid tokens and zero scales)
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int t = 16 * mt + g + 8 * hh;  // token within the tile
+        const bool ok = t < nv;
+        const float sk = skb[r0 + t] * qs;
+        const float sv = svb[r0 + t];
+        lsv[mt][hh] = (ok && sv > 0.f) ? __log2f(sv) : -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          s[mt][nt][2 * hh] = ok ? s[mt][nt][2 * hh] * sk : -INFINITY;
+          s[mt][nt][2 * hh + 1] = ok ? s[mt][nt][2 * hh + 1] * sk : -INFINITY;
+        }
+      }
+    }
+    uint32_t pb[NT][2][2];  // B fragments of P'^T per n-tile and k-step (16 tokens)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float beta[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float mx = fmaxf(fmaxf(s[0][nt][e], s[0][nt][e + 2]), fmaxf(s[1][nt][e], s[1][nt][e + 2]));
+#pragma unroll
+        for (int o2 = 4; o2 < 32; o2 <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
+        const float mn = fmaxf(m[nt][e], mx);  // finite: the tile holds a valid token
+        const float alpha = fast_exp2(m[nt][e] - mn);
+        const float rho_old = rho[nt][e] + (m[nt][e] - mn);  // rho relative to the new maximum (-inf stays -inf)
+        m[nt][e] = mn;
+        float u[2][2];
+        float ux = -INFINITY, ls = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          const float d0 = s[mt][nt][e] - mn, d1 = s[mt][nt][e + 2] - mn;
+          ls += fast_exp2(d0) + fast_exp2(d1);
+          u[mt][0] = d0 + lsv[mt][0];
+          u[mt][1] = d1 + lsv[mt][1];
+          ux = fmaxf(ux, fmaxf(u[mt][0], u[mt][1]));
+        }
+#pragma unroll
+        for (int o2 = 4; o2 < 32; o2 <<= 1) ux = fmaxf(ux, __shfl_xor_sync(0xffffffffu, ux, o2));
+        const float rn = fmaxf(rho_old, ux);
+        const bool any = rn > -INFINITY;  // some token so far has a non-zero V scale
+        beta[e] = any ? fast_exp2(rho_old - rn) : 1.f;
+        rho[nt][e] = rn;
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          s[mt][nt][e] = any ? fast_exp2(u[mt][0] - rn) : 0.f;
+          s[mt][nt][e + 2] = any ? fast_exp2(u[mt][1] - rn) : 0.f;
+        }
+        l[nt][e] = l[nt][e] * alpha + ls;
+      }
+#pragma unroll
+      for (int i = 0; i < KS; ++i) {
+        o[nt][i][0] *= beta[0]; o[nt][i][2] *= beta[0];
+        o[nt][i][1] *= beta[1]; o[nt][i][3] *= beta[1];
+      }
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        pb[nt][mt][0] = trans8x8(pack_h2(s[mt][nt][0], s[mt][nt][1]));  // tokens 2c, 2c+1 of head g
+        pb[nt][mt][1] = trans8x8(pack_h2(s[mt][nt][2], s[mt][nt][3]));  // tokens 2c+8, 2c+9
+      }
+    }
+    // ---- O^T += V^T P'^T: k-steps of 16 tokens; m-tiles (j, sub) hold d = 4g + 32j + 2sub + {0 (row g), 1 (row g+8)}
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      if (ks * 16 >= nv) break;
+      const int t0 = r0 + 16 * ks + 2 * c;
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) {
+        const int byte = 4 * g + 32 * j;
+        const uint32_t wa = lds32(swz8_addr<LY::ROWB>(vbase, t0, byte));
+        const uint32_t wb = lds32(swz8_addr<LY::ROWB>(vbase, t0 + 1, byte));
+        const uint32_t wc = lds32(swz8_addr<LY::ROWB>(vbase, t0 + 8, byte));
+        const uint32_t wd = lds32(swz8_addr<LY::ROWB>(vbase, t0 + 9, byte));
+        const uint32_t xab = prmt(wa, wb, 0x5140u) ^ 0x80808080u, yab = prmt(wa, wb, 0x7362u) ^ 0x80808080u;
+        const uint32_t xcd = prmt(wc, wd, 0x5140u) ^ 0x80808080u, ycd = prmt(wc, wd, 0x7362u) ^ 0x80808080u;
+        const uint32_t a00 = to_h2(xab, 0x4140u), a01 = to_h2(xab, 0x4342u);
+        const uint32_t a02 = to_h2(xcd, 0x4140u), a03 = to_h2(xcd, 0x4342u);
+        const uint32_t a10 = to_h2(yab, 0x4140u), a11 = to_h2(yab, 0x4342u);
+        const uint32_t a12 = to_h2(ycd, 0x4140u), a13 = to_h2(ycd, 0x4342u);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          mma_f16(o[nt][2 * j], a00, a01, a02, a03, pb[nt][ks][0], pb[nt][ks][1]);
+          mma_f16(o[nt][2 * j + 1], a10, a11, a12, a13, pb[nt][ks][0], pb[nt][ks][1]);
+        }
+      }
+    }
+  }
+
+  __device__ __forceinline__ void stash(float* merge_o, float* merge_ml, int lane) {
+    const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float rel[2];  // O relative to m = O relative to (m, rho) times 2^rho
+#pragma unroll
+      for (int e = 0; e < 2; ++e) rel[e] = rho[nt][e] > -INFINITY ? exp2f(rho[nt][e]) : 0.f;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float le = l[nt][e];
+        le += __shfl_xor_sync(0xffffffffu, le, 4);
+        le += __shfl_xor_sync(0xffffffffu, le, 8);
+        le += __shfl_xor_sync(0xffffffffu, le, 16);
+        const int h = nt * 8 + 2 * c + e;
+        if (g == 0 && h < G) {
+          merge_ml[h * 2] = m[nt][e];
+          merge_ml[h * 2 + 1] = le;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < KS; ++i) {
+        const int d = 4 * g + 32 * (i >> 1) + 2 * (i & 1);
+        const int h0 = nt * 8 + 2 * c;
+        if (h0 < G) {
+          merge_o[h0 * D + d] = o[nt][i][0] * rel[0];
+          merge_o[h0 * D + d + 1] = o[nt][i][2] * rel[0];
+        }
+        if (h0 + 1 < G) {
+          merge_o[(h0 + 1) * D + d] = o[nt][i][1] * rel[1];
+          merge_o[(h0 + 1) * D + d + 1] = o[nt][i][3] * rel[1];
+        }
+      }
+    }
+  }
+};
+
 // ------------------------------------------------------------------ producer: walk of a CTA's chunk range
 // Lane-uniform state (every lane of the producer warp holds the same values).
 struct Walker {
@@ -494,6 +783,7 @@ struct Walker {
   int batch, hkv, cap, grid;
   long long total;            // chunks on the whole line
   const int32_t* lens;
+  const int32_t* starts;      // per-sequence first token (null: 0); the walk sees L - start tokens
   // sub-ranges still to walk after the current one, in order (at most two)
   int nq;
   long long q0_start, q0_end, q0_pre, q1_start, q1_end, q1_pre;
@@ -507,10 +797,21 @@ __device__ __forceinline__ long long owner_of(long long x, long long total, long
 
 __device__ __forceinline__ int clamp_len(int L, int cap) { return L < 0 ? 0 : (L > cap ? cap : L); }
 
+// First token attended of sequence i: ctx_start[i] rounded down to a multiple of the 16-token chunk
+// (callers pass multiples of 16; anything else is recorded as an index error where it is first read).
+__device__ __forceinline__ int start_of(const int32_t* starts, int i) {
+  return starts ? (max(0, __ldg(starts + i)) & ~(kChunk - 1)) : 0;
+}
+// Tokens of sequence i the walk covers: its clamped length minus its start.
+__device__ __forceinline__ int eff_len(const int32_t* lens, const int32_t* starts, int i, int cap) {
+  const int L = clamp_len(__ldg(lens + i), cap), s0 = start_of(starts, i);
+  return L > s0 ? L - s0 : 0;
+}
+
 __device__ __forceinline__ void load_window(Walker& w, int base, int lane) {
   w.win_base = base;
   const int i = base + lane;
-  w.win_len = i < w.batch ? clamp_len(__ldg(w.lens + i), w.cap) : 0;
+  w.win_len = i < w.batch ? eff_len(w.lens, w.starts, i, w.cap) : 0;
 }
 
 // Sequence b holding chunk x of the line (x < total) and pre = chunks of all sequences before it.
@@ -525,7 +826,7 @@ __device__ __forceinline__ void find_seq(const Walker& w, long long x, int lane,
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int i = base + lane * 8 + j;
-      v[j] = i < w.batch ? (clamp_len(__ldg(w.lens + i), w.cap) + kChunk - 1) / kChunk : 0;
+      v[j] = i < w.batch ? (eff_len(w.lens, w.starts, i, w.cap) + kChunk - 1) / kChunk : 0;
       s += v[j];
     }
     const long long incl = warp_incl_scan_ll(s, lane);
@@ -635,11 +936,11 @@ __device__ __forceinline__ StageMeta walker_next(Walker& w, int cta, int lane) {
 }
 
 // ------------------------------------------------------------------ decode kernel
-template <int DT, int D, int G, int NW, int NSTAGES, bool MMA>
+template <int DT, int D, int G, int NW, int NSTAGES, bool MMA, bool Q8>
 __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_constant__ CUtensorMap kmap,
                                                                const __grid_constant__ CUtensorMap vmap,
                                                                const DecodeParams p) {
-  using LY = Layout<D, G, NW, NSTAGES, MMA>;
+  using LY = Layout<D, G, NW, NSTAGES, MMA, Q8>;
   using T = typename Elt<DT>::T;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -680,10 +981,17 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
         if (i < B) {
           const int L = __ldg(p.context_lens + i);
           clamped |= (L < 0 || L > cap);
-          s += (clamp_len(L, cap) + kChunk - 1) / kChunk;
-          if (cta == 0 && clamp_len(L, cap) == 0) {
+          if (p.ctx_start) {
+            const int s0 = __ldg(p.ctx_start + i);
+            clamped |= (s0 < 0 || (s0 & (kChunk - 1)) != 0);
+          }
+          const int Le = eff_len(p.context_lens, p.ctx_start, i, cap);
+          s += (Le + kChunk - 1) / kChunk;
+          if (cta == 0 && Le == 0) {
             uint4* o4 = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.out) + (size_t)i * p.num_q_heads * D);
             for (int e = 0; e < p.num_q_heads * D * 2 / 16; ++e) o4[e] = make_uint4(0, 0, 0, 0);
+            if (p.lse)
+              for (int h = 0; h < p.num_q_heads; ++h) p.lse[(size_t)i * p.num_q_heads + h] = -INFINITY;
           }
         }
       }
@@ -704,6 +1012,7 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
     w.grid = p.grid;
     w.total = C;
     w.lens = p.context_lens;
+    w.starts = p.ctx_start;
     w.win_base = -64;
     w.nq = 0;
     if (x0 < x1) {
@@ -713,7 +1022,7 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
       find_seq(w, x1 - 1, lane, bl, pl);
       walker_seek(w, x0, x1, b0, p0, lane);
       const long long s0 = w.seg_start, e0 = s0 + w.nch;
-      const int Ll = clamp_len(__ldg(p.context_lens + bl), cap), nl = (Ll + kChunk - 1) / kChunk;
+      const int Ll = eff_len(p.context_lens, p.ctx_start, bl, cap), nl = (Ll + kChunk - 1) / kChunk;
       const long long sl = pl * Hkv + ((x1 - 1 - pl * Hkv) / nl) * nl, el = sl + nl;
       const bool last_sep = sl > s0 && x1 < el;
       const long long first_end = e0 < x1 ? e0 : x1, mid_end = last_sep ? sl : x1;
@@ -738,7 +1047,8 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
       const int slot = j % kPlanRing;
       if (lane == 0) plan[slot] = dn;
       if (!(dn.flags & F_END) && lane < dn.nchunk)
-        cp_async4(plan_phys + slot * 8 + lane, bt_all + (size_t)dn.b * mb + (dn.tok0 + lane * kChunk) / bs);
+        cp_async4(plan_phys + slot * 8 + lane,
+                  bt_all + (size_t)dn.b * mb + (start_of(p.ctx_start, dn.b) + dn.tok0 + lane * kChunk) / bs);
       cp_async_commit();
     };
     for (int j = 0; j < kLookahead; ++j) plan_push(j);
@@ -764,19 +1074,29 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
         break;
       }
       const bool first = d.flags & F_FIRST;
+      constexpr uint32_t kChunkBytes = kChunk * LY::ROWB * 2 + (Q8 ? 2 * kChunk * 4 : 0);  // K + V (+ scales)
       if (lane == 0)
-        mbar_arrive_expect_tx(&full[st], (uint32_t)(d.nchunk * kChunk * D * 2 * 2 + (first ? LY::QSLOT : 0)));
+        mbar_arrive_expect_tx(&full[st], (uint32_t)d.nchunk * kChunkBytes + (first ? LY::QSLOT : 0));
       __syncwarp();
       if (lane < d.nchunk) {
-        if (phys < 0 || phys >= p.num_blocks) PA_RECORD_ERROR(PA_ERRBIT_INDEX);  // TMA zero-fills out of range
-        const int tok = d.tok0 + lane * kChunk;
+        const bool in_range = phys >= 0 && phys < p.num_blocks;
+        if (!in_range) PA_RECORD_ERROR(PA_ERRBIT_INDEX);  // TMA zero-fills out of range
+        const int tok = start_of(p.ctx_start, d.b) + d.tok0 + lane * kChunk;  // token of the sequence
         const int y = phys * bs + (tok % bs);
-        uint8_t* kd = smem + LY::K_OFF + st * LY::STAGE_BYTES + lane * kChunk * 128;
-        uint8_t* vd = smem + LY::V_OFF + st * LY::STAGE_BYTES + lane * kChunk * 128;
+        uint8_t* kd = smem + LY::K_OFF + st * LY::STAGE_BYTES + lane * kChunk * LY::BOXB;
+        uint8_t* vd = smem + LY::V_OFF + st * LY::STAGE_BYTES + lane * kChunk * LY::BOXB;
+        // tensor-map columns are 16-bit units: a row of one KV head starts at column g * ROWB / 2
 #pragma unroll
         for (int h = 0; h < LY::HALVES; ++h) {
-          tma_load_2d(kd + h * LY::TOK * 128, &kmap, d.g * D + h * 64, y, &full[st]);
-          tma_load_2d(vd + h * LY::TOK * 128, &vmap, d.g * D + h * 64, y, &full[st]);
+          tma_load_2d(kd + h * LY::TOK * LY::BOXB, &kmap, d.g * (LY::ROWB / 2) + h * 64, y, &full[st]);
+          tma_load_2d(vd + h * LY::TOK * LY::BOXB, &vmap, d.g * (LY::ROWB / 2) + h * 64, y, &full[st]);
+        }
+        if constexpr (Q8) {
+          // the chunk's 16 scales of KV head g: one 64-byte run of [num_blocks][Hkv][block_size] (a block id
+          // out of range reads block 0 instead; the error bit is set above)
+          const size_t so = ((size_t)(in_range ? phys : 0) * p.num_kv_heads + d.g) * bs + (tok % bs);
+          bulk_load(smem + LY::SK_OFF + (st * LY::TOK + lane * kChunk) * 4, p.k_scales + so, kChunk * 4, &full[st]);
+          bulk_load(smem + LY::SV_OFF + (st * LY::TOK + lane * kChunk) * 4, p.v_scales + so, kChunk * 4, &full[st]);
         }
       }
       if (first && lane == 31) {
@@ -834,6 +1154,8 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
         }
         if (direct) {
           outp[i] = Elt<DT>::from_f(num / den);
+          if (p.lse && dd == 0)
+            p.lse[(size_t)d.b * p.num_q_heads + (size_t)d.g * G + h] = (M + __log2f(den)) * kLn2;
         } else {
           const size_t srow = slot * G + h;
           p.ws_o[srow * D + dd] = num;
@@ -881,6 +1203,7 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
               den = fmaf(w, __ldcg(p.ws_l + srow), den);
             }
             const float inv = 1.f / den;
+            if (p.lse) p.lse[(size_t)d.b * p.num_q_heads + (size_t)d.g * G + h] = (Mh + __log2f(den)) * kLn2;
             for (int n = 0; n < np; ++n) wts[h * np + n] *= inv;
           }
           __syncwarp();
@@ -915,6 +1238,8 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
               den = fmaf(w, __ldcg(p.ws_l + srow), den);
             }
             outp[i] = Elt<DT>::from_f(num / den);
+            if (p.lse && dd == 0)
+              p.lse[(size_t)d.b * p.num_q_heads + (size_t)d.g * G + h] = (M + __log2f(den)) * kLn2;
           }
         }
       }
@@ -924,7 +1249,10 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
   }
 
   // =================================================== consumer warps
-  using C = typename std::conditional<MMA, MmaConsumer<DT, D, G, NW, NSTAGES>, CoreConsumer<DT, D, G, NW, NSTAGES>>::type;
+  using C = typename std::conditional<
+      Q8, Q8Consumer<D, G, NW, NSTAGES>,
+      typename std::conditional<MMA, MmaConsumer<DT, D, G, NW, NSTAGES>,
+                                CoreConsumer<DT, D, G, NW, NSTAGES>>::type>::type;
   C c;
   c.init();
   float* qf = reinterpret_cast<float*>(smem + LY::QF_OFF) + warp * G * D;
@@ -961,13 +1289,19 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
     }
     if (d.flags & F_FIRST) {
       c.init();
-      c.load_q(smem + LY::QS_OFF + st * LY::QSLOT, qf, p.scale_log2, lane);
+      if constexpr (Q8)
+        c.template load_q<DT>(smem + LY::QS_OFF + st * LY::QSLOT, p.scale_log2, lane);
+      else
+        c.load_q(smem + LY::QS_OFF + st * LY::QSLOT, qf, p.scale_log2, lane);
     }
     const int nv = min(32, max(0, d.ntok - warp * 32));
     if (nv > 0) {
       const uint32_t kb = sbase + LY::K_OFF + st * LY::STAGE_BYTES;
       const uint32_t vb = sbase + LY::V_OFF + st * LY::STAGE_BYTES;
-      if constexpr (MMA)
+      if constexpr (Q8)
+        c.tile(kb, vb, reinterpret_cast<const float*>(smem + LY::SK_OFF) + st * LY::TOK,
+               reinterpret_cast<const float*>(smem + LY::SV_OFF) + st * LY::TOK, warp * 32, nv, lane);
+      else if constexpr (MMA)
         c.tile(kb, vb, p.scale_log2, warp * 32, nv, lane);
       else
         c.tile(kb, vb, qbase, pbase, warp * 32, nv, lane);
@@ -982,30 +1316,281 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
   if (!ok && lane == 0) PA_RECORD_ERROR(PA_ERRBIT_TIMEOUT);
 }
 
-// ------------------------------------------------------------------ host side
-constexpr int kNW = 2;       // consumer warps per CTA (64-token stages)
-constexpr int kStages = 2;   // ring depth (three CTAs per SM)
+// ------------------------------------------------------------------ cascade decode: the shared-prefix pass
+// Sequences forked from one parent share the blocks of their common prefix (page "Nano-vLLM-Ascend:
+// lightweight LLM inference framework for Ascend NPU", section 2.1: reference-counted blocks; page "Ascend
+// NPU LLM inference optimisation: the vLLM-Ascend approach", section 4: block sharing for long contexts).
+// Plain decode reads every shared block once per sharer.  The cascade reads it once for all of them: the
+// decode kernel first attends over each sequence's private suffix (ctx_start = prefix length) and leaves
+// (out, lse) per (sequence, head); then this kernel attends over the shared prefix of every group with
+// the query rows of all its members at once, and merges the two parts by the log-sum-exp rule.
+//
+// Work: CTA (group, KV head, row tile, split) holds up to 64 query rows (member, head of the KV head's
+// group) and the split's share of the prefix's 16-token chunks.  One producer warp bulk-copies the q rows
+// and gathers K/V boxes through the first member's block table with TMA into a 2-stage ring; four
+// consumer warps own 16 rows each and run every 64-token stage through the warp-MMA consumer (QK^T and PV
+// on mma.m16n8k16, P as hi + lo 16-bit terms, fp32 online softmax).  Each CTA writes fp32 (m, l, o) per
+// row; the CTA that completes a row tile's last split (atomic count, no waiting) merges the splits with
+// the suffix part and writes out.
 
-template <int D, int G>
-constexpr int alloc_bytes() {
-  return Layout<D, G, kNW, kStages, (G >= 8)>::ALLOC;
+constexpr int kCasRows = 64;  // query rows per CTA (4 consumer warps x 16)
+
+struct CascadeParams {
+  const void* q;
+  void* out;                   // on entry the suffix result, on exit the final result
+  const float* lse_s;          // [batch][Hq] suffix log-sum-exp (natural log)
+  const int32_t* block_tables;
+  const int32_t* group_start;  // [num_groups + 1]
+  const int32_t* seq_prefix;   // [batch] shared prefix tokens of each sequence (the group's value)
+  int* cnt;                    // [num_groups * Hkv * tiles] splits done per row tile (zero between calls)
+  float* pm;                   // [units * splits][kCasRows]
+  float* pl;
+  float* po;                   // [units * splits][kCasRows][D]
+  int max_blocks_per_seq, batch, num_q_heads, num_kv_heads, block_size, num_blocks, num_groups, tiles, splits;
+  float scale_log2;
+};
+
+template <int D, int NSTAGES>
+struct CasLayout {
+  static constexpr int TOK = 64;
+  static constexpr int HALVES = D / 64;
+  static constexpr int STAGE_BYTES = TOK * D * 2;
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = NSTAGES * STAGE_BYTES;
+  static constexpr int Q_OFF = 2 * NSTAGES * STAGE_BYTES;
+  static constexpr int MISC_OFF = Q_OFF + kCasRows * D * 2;
+  static constexpr int BAR_OFF = MISC_OFF + 16;  // full[NSTAGES], empty[NSTAGES], qbar
+  static constexpr int BYTES = BAR_OFF + (2 * NSTAGES + 1) * 8;
+  static constexpr int ALLOC = BYTES + 1024;
+};
+
+template <int DT, int D, int G, int NSTAGES>
+__global__ void __launch_bounds__(160) cascade_prefix_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                             const __grid_constant__ CUtensorMap vmap,
+                                                             const CascadeParams p) {
+  using LY = CasLayout<D, NSTAGES>;
+  using T = typename Elt<DT>::T;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + LY::BAR_OFF);
+  uint64_t* empty = full + NSTAGES;
+  uint64_t* qbar = empty + NSTAGES;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = p.splits;
+  const int sp = blockIdx.x % S;
+  const int unit = blockIdx.x / S;  // (group, KV head, row tile)
+  const int rt = unit % p.tiles;
+  const int kvh = (unit / p.tiles) % p.num_kv_heads;
+  const int gi = unit / (p.tiles * p.num_kv_heads);
+  const int gs = __ldg(p.group_start + gi), ge = __ldg(p.group_start + gi + 1);
+  const int nrows = max(0, ge - gs) * G;
+  const int r0 = rt * kCasRows;
+  if (ge <= gs || r0 >= nrows) return;  // the same decision in every thread of the CTA
+  const int P0 = __ldg(p.seq_prefix + gs);
+  const int cap = p.max_blocks_per_seq * p.block_size;
+  const int P = min(max(0, P0), cap) & ~(kChunk - 1);
+  if (P == 0) return;  // no shared prefix: the suffix result already is the answer
+  const int C = P / kChunk;
+  const int c_begin = (int)((long long)C * sp / S), c_end = (int)((long long)C * (sp + 1) / S);
+  const int my_tok = (c_end - c_begin) * kChunk;
+  const int nstages = (my_tok + LY::TOK - 1) / LY::TOK;
+
+  if (threadIdx.x == 0) {
+    if (P0 != P || ((P0 & (kChunk - 1)) != 0)) PA_RECORD_ERROR(PA_ERRBIT_INDEX);
+    for (int i = 0; i < NSTAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 4);
+    }
+    mbar_init(qbar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == 4) {
+    // ================================================= producer warp
+    // q rows of the tile: row i = member gs + (r0+i)/G, query head kvh*G + (r0+i)%G; rows past the group
+    // are zero.
+    int valid = 0;
+    for (int i = lane; i < kCasRows; i += 32) {
+      const int rr = r0 + i;
+      uint8_t* dst = smem + LY::Q_OFF + i * D * 2;
+      if (rr < nrows) {
+        ++valid;
+      } else {
+        for (int e = 0; e < D * 2 / 16; ++e) reinterpret_cast<uint4*>(dst)[e] = make_uint4(0, 0, 0, 0);
+      }
+    }
+    for (int o = 16; o > 0; o >>= 1) valid += __shfl_xor_sync(0xffffffffu, valid, o);
+    __syncwarp();
+    if (lane == 0) mbar_arrive_expect_tx(qbar, (uint32_t)valid * D * 2);
+    __syncwarp();
+    for (int i = lane; i < kCasRows; i += 32) {
+      const int rr = r0 + i;
+      if (rr < nrows) {
+        const int b = gs + rr / G, h = kvh * G + rr % G;
+        bulk_load(smem + LY::Q_OFF + i * D * 2,
+                  reinterpret_cast<const uint8_t*>(p.q) + ((size_t)b * p.num_q_heads + h) * D * 2, D * 2, qbar);
+      }
+    }
+    const int32_t* bt = p.block_tables + (size_t)gs * p.max_blocks_per_seq;
+    const int bs = p.block_size;
+    bool ok = true;
+    // block of this lane's chunk of stage k (lanes 0..3), fetched one stage ahead
+    auto lookup = [&](int k) -> int {
+      const int c = c_begin + k * 4 + lane;
+      return (lane < 4 && c < c_end) ? __ldg(bt + (c * kChunk) / bs) : 0;
+    };
+    int phys = lookup(0);
+    int k = 0;
+    for (; k < nstages; ++k) {
+      const int st = k % NSTAGES;
+      const int next = lookup(k + 1);
+      if (k >= NSTAGES && !mbar_wait(&empty[st], ((k / NSTAGES) - 1) & 1)) {
+        ok = false;
+        break;
+      }
+      const int nch = min(4, c_end - (c_begin + k * 4));
+      if (lane == 0) mbar_arrive_expect_tx(&full[st], (uint32_t)(nch * kChunk * D * 2 * 2));
+      __syncwarp();
+      if (lane < nch) {
+        if (phys < 0 || phys >= p.num_blocks) PA_RECORD_ERROR(PA_ERRBIT_INDEX);  // TMA zero-fills out of range
+        const int tok = (c_begin + k * 4 + lane) * kChunk;
+        const int y = phys * bs + (tok % bs);
+        uint8_t* kd = smem + LY::K_OFF + st * LY::STAGE_BYTES + lane * kChunk * 128;
+        uint8_t* vd = smem + LY::V_OFF + st * LY::STAGE_BYTES + lane * kChunk * 128;
+#pragma unroll
+        for (int h = 0; h < LY::HALVES; ++h) {
+          tma_load_2d(kd + h * LY::TOK * 128, &kmap, kvh * D + h * 64, y, &full[st]);
+          tma_load_2d(vd + h * LY::TOK * 128, &vmap, kvh * D + h * 64, y, &full[st]);
+        }
+      }
+      phys = next;
+    }
+    if (!ok && lane == 0) PA_RECORD_ERROR(PA_ERRBIT_TIMEOUT);
+    // drain: every copy this CTA issued has landed before the warp leaves
+    if (lane == 0) {
+      if (!mbar_wait(qbar, 0)) PA_RECORD_ERROR(PA_ERRBIT_TIMEOUT);
+      for (int j = max(0, k - NSTAGES); j < k; ++j)
+        if (!mbar_wait(&full[j % NSTAGES], (j / NSTAGES) & 1)) PA_RECORD_ERROR(PA_ERRBIT_TIMEOUT);
+    }
+    return;
+  }
+
+  // =================================================== consumer warps (16 rows each)
+  MmaConsumer<DT, D, 16, 2, NSTAGES> c;
+  c.init();
+  bool ok = mbar_wait(qbar, 0);
+  if (ok) c.load_q(smem + LY::Q_OFF + warp * 16 * D * 2, nullptr, 0.f, lane);
+  for (int k = 0; ok && k < nstages; ++k) {
+    const int st = k % NSTAGES;
+    if (!mbar_wait(&full[st], (k / NSTAGES) & 1)) {
+      ok = false;
+      break;
+    }
+    const int ntok = min(LY::TOK, my_tok - k * LY::TOK);
+    const uint32_t kb = sbase + LY::K_OFF + st * LY::STAGE_BYTES;
+    const uint32_t vb = sbase + LY::V_OFF + st * LY::STAGE_BYTES;
+    c.tile(kb, vb, p.scale_log2, 0, min(32, ntok), lane);
+    if (ntok > 32) c.tile(kb, vb, p.scale_log2, 32, ntok - 32, lane);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+  }
+  if (!ok && lane == 0) PA_RECORD_ERROR(PA_ERRBIT_TIMEOUT);
+  // ---- this split's partial (m, l, o) of the warp's 16 rows
+  {
+    float l0 = c.l[0], l1 = c.l[1];
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    const size_t slot = (size_t)unit * S + sp;
+    const int ra = warp * 16 + (lane >> 2), rb = ra + 8;
+    float* po = p.po + slot * kCasRows * D;
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      const int col = n * 8 + (lane & 3) * 2;
+      *reinterpret_cast<float2*>(po + (size_t)ra * D + col) = make_float2(c.o[n][0], c.o[n][1]);
+      *reinterpret_cast<float2*>(po + (size_t)rb * D + col) = make_float2(c.o[n][2], c.o[n][3]);
+    }
+    if ((lane & 3) == 0) {
+      p.pm[slot * kCasRows + ra] = c.m[0];
+      p.pl[slot * kCasRows + ra] = l0;
+      p.pm[slot * kCasRows + rb] = c.m[1];
+      p.pl[slot * kCasRows + rb] = l1;
+    }
+  }
+  __threadfence();                // this split's partial is visible device-wide before it is counted
+  named_barrier_sync(1, 128);     // all four consumer warps
+  int* last_flag = reinterpret_cast<int*>(smem + LY::MISC_OFF);
+  if (threadIdx.x == 0) {
+    const int prev = atomicAdd(p.cnt + unit, 1);
+    const int last = prev == S - 1;
+    if (last) atomicExch(p.cnt + unit, 0);  // leave the counter at zero for the next call
+    *last_flag = last;
+  }
+  named_barrier_sync(1, 128);
+  if (!*last_flag) return;
+  __threadfence();
+  // ---- merge the S splits with the suffix part: row i of the tile = (b, h)
+  const float* pm = p.pm + (size_t)unit * S * kCasRows;
+  const float* pl = p.pl + (size_t)unit * S * kCasRows;
+  const float* po = p.po + (size_t)unit * S * kCasRows * D;
+  for (int i = warp; i < kCasRows; i += 4) {
+    const int rr = r0 + i;
+    if (rr >= nrows) break;
+    const int b = gs + rr / G, h = kvh * G + rr % G;
+    const float ms = __ldg(p.lse_s + (size_t)b * p.num_q_heads + h) * kLog2e;  // suffix, log2 domain, l = 1
+    float M = ms;
+    for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, __ldcg(pm + (size_t)s2 * kCasRows + i));
+    const float ws = fast_exp2(ms - M);  // 0 when the suffix is empty (ms = -inf)
+    float den = ws;
+    for (int s2 = 0; s2 < S; ++s2)
+      den = fmaf(fast_exp2(__ldcg(pm + (size_t)s2 * kCasRows + i) - M), __ldcg(pl + (size_t)s2 * kCasRows + i), den);
+    const float inv = 1.f / den;
+    T* orow = reinterpret_cast<T*>(p.out) + ((size_t)b * p.num_q_heads + h) * D;
+    for (int d0 = lane * 2; d0 < D; d0 += 64) {
+      const float2 so = Elt<DT>::to_f2(*reinterpret_cast<const uint32_t*>(orow + d0));
+      float a0 = ws * so.x, a1 = ws * so.y;
+      for (int s2 = 0; s2 < S; ++s2) {
+        const float w = fast_exp2(__ldcg(pm + (size_t)s2 * kCasRows + i) - M);
+        const float2 o2 = __ldcg(reinterpret_cast<const float2*>(po + ((size_t)s2 * kCasRows + i) * D + d0));
+        a0 = fmaf(w, o2.x, a0);
+        a1 = fmaf(w, o2.y, a1);
+      }
+      *reinterpret_cast<uint32_t*>(orow + d0) = Elt<DT>::from_f2(a0 * inv, a1 * inv);
+    }
+  }
 }
 
-int smem_per_cta(int D, int G) {
+// ------------------------------------------------------------------ host side
+constexpr int kNW = 2;        // consumer warps per CTA (64-token stages)
+constexpr int kStages = 2;    // ring depth, 16-bit cache (three CTAs per SM)
+constexpr int kStagesQ8 = 4;  // ring depth, int8 cache: the same bytes in flight per SM as the 16-bit ring
+
+template <int D, int G, bool Q8>
+constexpr int alloc_bytes() {
+  return Layout<D, G, kNW, Q8 ? kStagesQ8 : kStages, Q8 || (G >= 8), Q8>::ALLOC;
+}
+
+template <bool Q8>
+int smem_per_cta_t(int D, int G) {
   switch (D * 100 + G) {
-    case 6401: return alloc_bytes<64, 1>();
-    case 6402: return alloc_bytes<64, 2>();
-    case 6404: return alloc_bytes<64, 4>();
-    case 6408: return alloc_bytes<64, 8>();
-    case 6416: return alloc_bytes<64, 16>();
-    case 12801: return alloc_bytes<128, 1>();
-    case 12802: return alloc_bytes<128, 2>();
-    case 12804: return alloc_bytes<128, 4>();
-    case 12808: return alloc_bytes<128, 8>();
-    case 12816: return alloc_bytes<128, 16>();
+    case 6401: return alloc_bytes<64, 1, Q8>();
+    case 6402: return alloc_bytes<64, 2, Q8>();
+    case 6404: return alloc_bytes<64, 4, Q8>();
+    case 6408: return alloc_bytes<64, 8, Q8>();
+    case 6416: return alloc_bytes<64, 16, Q8>();
+    case 12801: return alloc_bytes<128, 1, Q8>();
+    case 12802: return alloc_bytes<128, 2, Q8>();
+    case 12804: return alloc_bytes<128, 4, Q8>();
+    case 12808: return alloc_bytes<128, 8, Q8>();
+    case 12816: return alloc_bytes<128, 16, Q8>();
   }
   return 0;
 }
+
+int smem_per_cta(int D, int G, bool q8) { return q8 ? smem_per_cta_t<true>(D, G) : smem_per_cta_t<false>(D, G); }
 
 struct Plan {
   int grid;
@@ -1015,10 +1600,10 @@ struct Plan {
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-bool make_plan(int batch, int Hq, int Hkv, int D, int num_partitions, Plan* pl) {
+bool make_plan(int batch, int Hq, int Hkv, int D, int num_partitions, bool q8, Plan* pl) {
   if (batch < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || num_partitions < 0 || Hq % Hkv) return false;
   const int G = Hq / Hkv;
-  const int smem = smem_per_cta(D, G);
+  const int smem = smem_per_cta(D, G, q8);
   if (smem == 0) return false;
   int grid = num_partitions;
   if (grid == 0) {
@@ -1039,11 +1624,12 @@ bool make_plan(int batch, int Hq, int Hkv, int D, int num_partitions, Plan* pl) 
   return true;
 }
 
-template <int DT, int D, int G>
+template <int DT, int D, int G, bool Q8>
 int launch(const CUtensorMap& km, const CUtensorMap& vm, const DecodeParams& p, cudaStream_t st) {
-  constexpr bool MMA = G >= 8;
-  using LY = Layout<D, G, kNW, kStages, MMA>;
-  auto kern = decode_kernel<DT, D, G, kNW, kStages, MMA>;
+  constexpr bool MMA = Q8 || G >= 8;
+  constexpr int NS = Q8 ? kStagesQ8 : kStages;
+  using LY = Layout<D, G, kNW, NS, MMA, Q8>;
+  auto kern = decode_kernel<DT, D, G, kNW, NS, MMA, Q8>;
   // per instantiation and device; host threads may race to set it, which only repeats an idempotent call
   static std::atomic<bool> attr_set[64] = {};
   int dev = 0;
@@ -1053,7 +1639,7 @@ int launch(const CUtensorMap& km, const CUtensorMap& vm, const DecodeParams& p, 
       return PA_ERR_CUDA;
     if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
   }
-  // programmatic dependent launch: may start while the preceding pa_write_kv runs (it signals
+  // programmatic dependent launch: may start while the preceding cache write runs (it signals
   // its dependents at entry); the producer waits for it before the first cache load
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.grid);
@@ -1070,16 +1656,28 @@ int launch(const CUtensorMap& km, const CUtensorMap& vm, const DecodeParams& p, 
   return PA_OK;
 }
 
-template <int DT, int D>
+template <int DT, int D, bool Q8>
 int dispatch_g(int G, const CUtensorMap& km, const CUtensorMap& vm, const DecodeParams& p, cudaStream_t st) {
   switch (G) {
-    case 1: return launch<DT, D, 1>(km, vm, p, st);
-    case 2: return launch<DT, D, 2>(km, vm, p, st);
-    case 4: return launch<DT, D, 4>(km, vm, p, st);
-    case 8: return launch<DT, D, 8>(km, vm, p, st);
-    case 16: return launch<DT, D, 16>(km, vm, p, st);
+    case 1: return launch<DT, D, 1, Q8>(km, vm, p, st);
+    case 2: return launch<DT, D, 2, Q8>(km, vm, p, st);
+    case 4: return launch<DT, D, 4, Q8>(km, vm, p, st);
+    case 8: return launch<DT, D, 8, Q8>(km, vm, p, st);
+    case 16: return launch<DT, D, 16, Q8>(km, vm, p, st);
   }
   return PA_ERR_UNSUPPORTED;
+}
+
+int decode_plan_impl(int batch, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len,
+                     int num_partitions_or_0, bool q8, int* grid_out, int* max_pieces_out,
+                     size_t* workspace_bytes_out) {
+  if (max_context_len < 0 || !pa::valid_head_dim(head_dim)) return PA_ERR_INVALID;
+  Plan pl;
+  if (!make_plan(batch, num_q_heads, num_kv_heads, head_dim, num_partitions_or_0, q8, &pl)) return PA_ERR_INVALID;
+  if (grid_out) *grid_out = pl.grid;
+  if (max_pieces_out) *max_pieces_out = batch * num_kv_heads + pl.grid;
+  if (workspace_bytes_out) *workspace_bytes_out = pl.ws_bytes;
+  return PA_OK;
 }
 
 }  // namespace
@@ -1087,40 +1685,52 @@ int dispatch_g(int G, const CUtensorMap& km, const CUtensorMap& vm, const Decode
 extern "C" int pa_decode_plan(int batch, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len,
                               int num_partitions_or_0, int* grid_out, int* max_pieces_out,
                               size_t* workspace_bytes_out) {
-  if (max_context_len < 0 || !pa::valid_head_dim(head_dim)) return PA_ERR_INVALID;
-  Plan pl;
-  if (!make_plan(batch, num_q_heads, num_kv_heads, head_dim, num_partitions_or_0, &pl)) return PA_ERR_INVALID;
-  if (grid_out) *grid_out = pl.grid;
-  if (max_pieces_out) *max_pieces_out = batch * num_kv_heads + pl.grid;
-  if (workspace_bytes_out) *workspace_bytes_out = pl.ws_bytes;
-  return PA_OK;
+  return decode_plan_impl(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_partitions_or_0, false,
+                          grid_out, max_pieces_out, workspace_bytes_out);
 }
 
 extern "C" size_t pa_decode_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
                                            int max_context_len, int num_partitions_or_0) {
   size_t ws = 0;
-  if (pa_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_partitions_or_0, nullptr,
-                     nullptr, &ws) != PA_OK)
+  if (decode_plan_impl(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_partitions_or_0, false,
+                       nullptr, nullptr, &ws) != PA_OK)
+    return 0;
+  return ws;
+}
+
+extern "C" int pa_decode_int8_plan(int batch, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len,
+                                   int num_partitions_or_0, int* grid_out, int* max_pieces_out,
+                                   size_t* workspace_bytes_out) {
+  return decode_plan_impl(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_partitions_or_0, true,
+                          grid_out, max_pieces_out, workspace_bytes_out);
+}
+
+extern "C" size_t pa_decode_int8_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                                                int max_context_len, int num_partitions_or_0) {
+  size_t ws = 0;
+  if (decode_plan_impl(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, num_partitions_or_0, true,
+                       nullptr, nullptr, &ws) != PA_OK)
     return 0;
   return ws;
 }
 
 namespace {
 
-// Everything pa_decode does before it enqueues work: argument checks, the plan, the kernel parameters and
-// the two tensor maps.  Enqueues nothing; returns PA_OK with *launchable = false when there is nothing to
-// run (batch 0).
+// Everything a decode call does before it enqueues work: argument checks, the plan, the kernel parameters
+// and the two tensor maps.  Enqueues nothing; returns PA_OK with *launchable = false when there is nothing
+// to run (batch 0).  q8: the caches are int8 codes with fp32 scales (k_scales, v_scales).
 struct DecodeCall {
   DecodeParams p;
   CUtensorMap km, vm;
   int dtype, head_dim, G;
-  bool launchable;
+  bool q8, launchable;
 };
 
-int decode_prepare(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
-                   int max_blocks_per_seq, const int32_t* context_lens, int batch, int num_q_heads, int num_kv_heads,
-                   int head_dim, int block_size, int num_blocks, int max_context_len, float scale, int dtype,
-                   void* workspace, size_t workspace_bytes, int num_partitions_or_0, void* out, DecodeCall* call) {
+int decode_prepare(const void* q, const void* k_cache, const void* v_cache, const float* k_scales,
+                   const float* v_scales, bool q8, const int32_t* block_tables, int max_blocks_per_seq,
+                   const int32_t* context_lens, int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                   int block_size, int num_blocks, int max_context_len, float scale, int dtype, void* workspace,
+                   size_t workspace_bytes, int num_partitions_or_0, void* out, float* lse, DecodeCall* call) {
   call->launchable = false;
   if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks < 0 ||
       max_context_len < 0 || max_blocks_per_seq < 0 || num_partitions_or_0 < 0)
@@ -1132,20 +1742,27 @@ int decode_prepare(const void* q, const void* k_cache, const void* v_cache, cons
   if (!pa::valid_group(G)) return PA_ERR_UNSUPPORTED;
   if (batch == 0) return PA_OK;
   if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out) return PA_ERR_INVALID;
+  if (q8 && (!k_scales || !v_scales)) return PA_ERR_INVALID;
   if (!pa::aligned16(q) || !pa::aligned16(k_cache) || !pa::aligned16(v_cache) || !pa::aligned16(out) ||
       (reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u))
     return PA_ERR_ALIGN;
+  if (q8 && (!pa::aligned16(k_scales) || !pa::aligned16(v_scales))) return PA_ERR_ALIGN;
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return PA_ERR_ALIGN;
   if ((long)max_blocks_per_seq * block_size < max_context_len) return PA_ERR_INVALID;
   if (num_blocks == 0 && max_context_len > 0) return PA_ERR_INVALID;
   if ((long)num_blocks * block_size >= (1L << 31)) return PA_ERR_UNSUPPORTED;
   Plan pl;
-  if (!make_plan(batch, num_q_heads, num_kv_heads, head_dim, num_partitions_or_0, &pl)) return PA_ERR_INVALID;
+  if (!make_plan(batch, num_q_heads, num_kv_heads, head_dim, num_partitions_or_0, q8, &pl)) return PA_ERR_INVALID;
   if (!workspace || workspace_bytes < pl.ws_bytes) return PA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PA_ERR_ALIGN;
 
   DecodeParams& p = call->p;
   p.q = q;
   p.out = out;
+  p.k_scales = k_scales;
+  p.v_scales = v_scales;
+  p.lse = lse;
+  p.ctx_start = nullptr;
   p.block_tables = block_tables;
   p.context_lens = context_lens;
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
@@ -1162,24 +1779,35 @@ int decode_prepare(const void* q, const void* k_cache, const void* v_cache, cons
   p.grid = pl.grid;
   p.scale_log2 = scale * kLog2e;
 
-  // One tensor map per cache over the [num_blocks*block_size][Hkv*D] row view; 16-row x 64-column boxes.
+  // One tensor map per cache over the [num_blocks*block_size][Hkv*D] row view, in 16-bit units (an int8
+  // row of D codes is D/2 units); boxes of 16 rows x 128 bytes (128-byte swizzle), or 16 rows x 64 bytes
+  // (64-byte swizzle) for the int8 rows of head_dim 64.
   const uint64_t rows = (uint64_t)std::max(num_blocks, 1) * block_size;
-  const uint64_t cols = (uint64_t)num_kv_heads * head_dim;
-  if (pa::encode_2d_sw128(&call->km, k_cache, cols, rows, cols * 2, 64, 16) != PA_OK) return PA_ERR_CUDA;
-  if (pa::encode_2d_sw128(&call->vm, v_cache, cols, rows, cols * 2, 64, 16) != PA_OK) return PA_ERR_CUDA;
+  const uint64_t row_bytes = (uint64_t)num_kv_heads * head_dim * (q8 ? 1 : 2);
+  const uint32_t box_bytes = (q8 && head_dim == 64) ? 64u : 128u;
+  if (pa::encode_2d_u16(&call->km, k_cache, row_bytes / 2, rows, row_bytes, box_bytes / 2, 16, box_bytes) != PA_OK)
+    return PA_ERR_CUDA;
+  if (pa::encode_2d_u16(&call->vm, v_cache, row_bytes / 2, rows, row_bytes, box_bytes / 2, 16, box_bytes) != PA_OK)
+    return PA_ERR_CUDA;
   call->dtype = dtype;
   call->head_dim = head_dim;
   call->G = G;
+  call->q8 = q8;
   call->launchable = true;
   return PA_OK;
 }
 
-int decode_launch(const DecodeCall& c, cudaStream_t st) {
+template <bool Q8>
+int decode_launch_t(const DecodeCall& c, cudaStream_t st) {
   if (c.dtype == PA_BF16)
-    return c.head_dim == 128 ? dispatch_g<PA_BF16, 128>(c.G, c.km, c.vm, c.p, st)
-                             : dispatch_g<PA_BF16, 64>(c.G, c.km, c.vm, c.p, st);
-  return c.head_dim == 128 ? dispatch_g<PA_F16, 128>(c.G, c.km, c.vm, c.p, st)
-                           : dispatch_g<PA_F16, 64>(c.G, c.km, c.vm, c.p, st);
+    return c.head_dim == 128 ? dispatch_g<PA_BF16, 128, Q8>(c.G, c.km, c.vm, c.p, st)
+                             : dispatch_g<PA_BF16, 64, Q8>(c.G, c.km, c.vm, c.p, st);
+  return c.head_dim == 128 ? dispatch_g<PA_F16, 128, Q8>(c.G, c.km, c.vm, c.p, st)
+                           : dispatch_g<PA_F16, 64, Q8>(c.G, c.km, c.vm, c.p, st);
+}
+
+int decode_launch(const DecodeCall& c, cudaStream_t st) {
+  return c.q8 ? decode_launch_t<true>(c, st) : decode_launch_t<false>(c, st);
 }
 
 }  // namespace
@@ -1190,11 +1818,176 @@ extern "C" int pa_decode(const void* q, const void* k_cache, const void* v_cache
                          float scale, int dtype, void* workspace, size_t workspace_bytes, int num_partitions_or_0,
                          void* out, void* stream) {
   DecodeCall call;
-  const int s = decode_prepare(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch,
-                               num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, max_context_len, scale,
-                               dtype, workspace, workspace_bytes, num_partitions_or_0, out, &call);
+  const int s = decode_prepare(q, k_cache, v_cache, nullptr, nullptr, false, block_tables, max_blocks_per_seq,
+                               context_lens, batch, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                               max_context_len, scale, dtype, workspace, workspace_bytes, num_partitions_or_0, out,
+                               nullptr, &call);
   if (s != PA_OK || !call.launchable) return s;
   return decode_launch(call, (cudaStream_t)stream);
+}
+
+extern "C" int pa_decode_lse(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                             int max_blocks_per_seq, const int32_t* context_lens, int batch, int num_q_heads,
+                             int num_kv_heads, int head_dim, int block_size, int num_blocks, int max_context_len,
+                             float scale, int dtype, void* workspace, size_t workspace_bytes, int num_partitions_or_0,
+                             void* out, float* lse_out, void* stream) {
+  if (!lse_out && batch > 0) return PA_ERR_INVALID;
+  DecodeCall call;
+  const int s = decode_prepare(q, k_cache, v_cache, nullptr, nullptr, false, block_tables, max_blocks_per_seq,
+                               context_lens, batch, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                               max_context_len, scale, dtype, workspace, workspace_bytes, num_partitions_or_0, out,
+                               lse_out, &call);
+  if (s != PA_OK || !call.launchable) return s;
+  return decode_launch(call, (cudaStream_t)stream);
+}
+
+extern "C" int pa_decode_int8(const void* q, const void* k_codes, const void* v_codes, const float* k_scales,
+                              const float* v_scales, const int32_t* block_tables, int max_blocks_per_seq,
+                              const int32_t* context_lens, int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                              int block_size, int num_blocks, int max_context_len, float scale, int dtype,
+                              void* workspace, size_t workspace_bytes, int num_partitions_or_0, void* out,
+                              void* stream) {
+  DecodeCall call;
+  const int s = decode_prepare(q, k_codes, v_codes, k_scales, v_scales, true, block_tables, max_blocks_per_seq,
+                               context_lens, batch, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                               max_context_len, scale, dtype, workspace, workspace_bytes, num_partitions_or_0, out,
+                               nullptr, &call);
+  if (s != PA_OK || !call.launchable) return s;
+  return decode_launch(call, (cudaStream_t)stream);
+}
+
+// ------------------------------------------------------------------ cascade decode (shared prefixes)
+namespace {
+
+constexpr int kCasStages = 2;
+
+struct CascadePlan {
+  Plan dec;
+  size_t off_lse, off_cnt, off_pm, off_pl, off_po, total;
+  int tiles, splits, units;
+};
+
+bool make_cascade_plan(int batch, int Hq, int Hkv, int D, int num_partitions, int num_groups, int max_group_size,
+                       int max_prefix_len, CascadePlan* cp) {
+  if (num_groups < 0 || max_group_size < 0 || max_prefix_len < 0) return false;
+  if (!make_plan(batch, Hq, Hkv, D, num_partitions, false, &cp->dec)) return false;
+  const int G = Hq / Hkv;
+  cp->tiles = std::max(1, (max_group_size * G + kCasRows - 1) / kCasRows);
+  cp->units = num_groups * Hkv * cp->tiles;
+  const int target = pa::sm_count() * 2;  // two CTAs per SM
+  const int by_work = std::max(1, max_prefix_len / 64);
+  cp->splits = cp->units > 0 ? std::max(1, std::min(by_work, (target + cp->units - 1) / cp->units)) : 1;
+  const size_t slots = (size_t)cp->units * cp->splits;
+  cp->off_lse = align256(cp->dec.ws_bytes);
+  cp->off_cnt = cp->off_lse + align256((size_t)batch * Hq * 4);
+  cp->off_pm = cp->off_cnt + align256((size_t)cp->units * 4);
+  cp->off_pl = cp->off_pm + align256(slots * kCasRows * 4);
+  cp->off_po = cp->off_pl + align256(slots * kCasRows * 4);
+  cp->total = cp->off_po + align256(slots * kCasRows * D * 4);
+  return true;
+}
+
+template <int DT, int D, int G>
+int launch_cascade(const CUtensorMap& km, const CUtensorMap& vm, const CascadeParams& cp, int grid, cudaStream_t st) {
+  using LY = CasLayout<D, kCasStages>;
+  auto kern = cascade_prefix_kernel<DT, D, G, kCasStages>;
+  static std::atomic<bool> attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_acquire)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::ALLOC) != cudaSuccess)
+      return PA_ERR_CUDA;
+    if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
+  }
+  kern<<<grid, 160, LY::ALLOC, st>>>(km, vm, cp);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <int DT, int D>
+int dispatch_cascade(int G, const CUtensorMap& km, const CUtensorMap& vm, const CascadeParams& cp, int grid,
+                     cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_cascade<DT, D, 1>(km, vm, cp, grid, st);
+    case 2: return launch_cascade<DT, D, 2>(km, vm, cp, grid, st);
+    case 4: return launch_cascade<DT, D, 4>(km, vm, cp, grid, st);
+    case 8: return launch_cascade<DT, D, 8>(km, vm, cp, grid, st);
+    case 16: return launch_cascade<DT, D, 16>(km, vm, cp, grid, st);
+  }
+  return PA_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+extern "C" size_t pa_decode_cascade_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                                                   int max_context_len, int num_partitions_or_0, int num_groups,
+                                                   int max_group_size, int max_prefix_len) {
+  if (max_context_len < 0 || !pa::valid_head_dim(head_dim)) return 0;
+  CascadePlan cp;
+  if (!make_cascade_plan(batch, num_q_heads, num_kv_heads, head_dim, num_partitions_or_0, num_groups, max_group_size,
+                         max_prefix_len, &cp))
+    return 0;
+  return cp.total;
+}
+
+extern "C" int pa_decode_cascade(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                                 int max_blocks_per_seq, const int32_t* context_lens, int batch, int num_q_heads,
+                                 int num_kv_heads, int head_dim, int block_size, int num_blocks, int max_context_len,
+                                 float scale, int dtype, int num_groups, const int32_t* group_start,
+                                 const int32_t* seq_prefix_len, int max_group_size, int max_prefix_len,
+                                 void* workspace, size_t workspace_bytes, int num_partitions_or_0, void* out,
+                                 void* stream) {
+  if (num_groups < 0 || max_group_size < 0 || max_prefix_len < 0 || max_prefix_len > max_context_len)
+    return PA_ERR_INVALID;
+  if (batch > 0 && (!seq_prefix_len || (num_groups > 0 && !group_start))) return PA_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(seq_prefix_len) & 3u) || (reinterpret_cast<uintptr_t>(group_start) & 3u))
+    return PA_ERR_ALIGN;
+  if (num_groups > batch || (num_groups > 0 && max_group_size < 1)) return PA_ERR_INVALID;
+  if (num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads) return PA_ERR_INVALID;
+  CascadePlan cp;
+  if (!make_cascade_plan(batch, num_q_heads, num_kv_heads, head_dim, num_partitions_or_0, num_groups, max_group_size,
+                         max_prefix_len, &cp))
+    return PA_ERR_INVALID;
+  if (workspace && workspace_bytes < cp.total) return PA_ERR_WORKSPACE;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  DecodeCall call;
+  int s = decode_prepare(q, k_cache, v_cache, nullptr, nullptr, false, block_tables, max_blocks_per_seq, context_lens,
+                         batch, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, max_context_len, scale,
+                         dtype, workspace, workspace ? cp.dec.ws_bytes : 0, num_partitions_or_0, out,
+                         ws ? reinterpret_cast<float*>(ws + cp.off_lse) : nullptr, &call);
+  if (s != PA_OK || !call.launchable) return s;
+  // pass 1: every sequence's private suffix (tokens from its prefix length on), with its log-sum-exp
+  call.p.ctx_start = seq_prefix_len;
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((s = decode_launch(call, st)) != PA_OK) return s;
+  if (num_groups == 0 || max_prefix_len < kChunk) return PA_OK;
+  // pass 2: the shared prefix of every group, once for all of its members, merged with pass 1
+  CascadeParams c;
+  c.q = q;
+  c.out = out;
+  c.lse_s = reinterpret_cast<const float*>(ws + cp.off_lse);
+  c.block_tables = block_tables;
+  c.group_start = group_start;
+  c.seq_prefix = seq_prefix_len;
+  c.cnt = reinterpret_cast<int*>(ws + cp.off_cnt);
+  c.pm = reinterpret_cast<float*>(ws + cp.off_pm);
+  c.pl = reinterpret_cast<float*>(ws + cp.off_pl);
+  c.po = reinterpret_cast<float*>(ws + cp.off_po);
+  c.max_blocks_per_seq = max_blocks_per_seq;
+  c.batch = batch;
+  c.num_q_heads = num_q_heads;
+  c.num_kv_heads = num_kv_heads;
+  c.block_size = block_size;
+  c.num_blocks = num_blocks;
+  c.num_groups = num_groups;
+  c.tiles = cp.tiles;
+  c.splits = cp.splits;
+  c.scale_log2 = scale * kLog2e;
+  const int grid = cp.units * cp.splits;
+  if (dtype == PA_BF16)
+    return head_dim == 128 ? dispatch_cascade<PA_BF16, 128>(call.G, call.km, call.vm, c, grid, st)
+                           : dispatch_cascade<PA_BF16, 64>(call.G, call.km, call.vm, c, grid, st);
+  return head_dim == 128 ? dispatch_cascade<PA_F16, 128>(call.G, call.km, call.vm, c, grid, st)
+                         : dispatch_cascade<PA_F16, 64>(call.G, call.km, call.vm, c, grid, st);
 }
 
 // ------------------------------------------------------------------ decode with library-owned scratch
@@ -1243,9 +2036,9 @@ extern "C" int pa_decode_static_scratch(const void* q, const void* k_cache, cons
   // Every check pa_decode makes, before anything is enqueued: a rejected call leaves the stream and the
   // scratch untouched.
   DecodeCall call;
-  s = decode_prepare(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch, num_q_heads,
-                     num_kv_heads, head_dim, block_size, num_blocks, max_context_len, scale, dtype, scratch,
-                     PA_DECODE_STATIC_SCRATCH_BYTES, num_partitions_or_0, out, &call);
+  s = decode_prepare(q, k_cache, v_cache, nullptr, nullptr, false, block_tables, max_blocks_per_seq, context_lens,
+                     batch, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, max_context_len, scale, dtype,
+                     scratch, PA_DECODE_STATIC_SCRATCH_BYTES, num_partitions_or_0, out, nullptr, &call);
   if (s != PA_OK || !call.launchable) return s;
   // The head of the scratch holds the per-segment piece counters, which must start at zero.  A completed
   // call leaves them at zero, but they are cleared anyway so that an earlier call that gave up (a timed-out

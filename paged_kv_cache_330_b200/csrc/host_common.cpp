@@ -11,6 +11,7 @@ extern "C" int pa__err_write_kv(unsigned int* out);
 extern "C" int pa__err_decode(unsigned int* out);
 extern "C" int pa__err_prefill(unsigned int* out);
 extern "C" int pa__err_rope(unsigned int* out);
+extern "C" int pa__err_int8(unsigned int* out);
 
 extern "C" const char* pa_strerror(int status) {
   switch (status) {
@@ -32,13 +33,14 @@ extern "C" const char* pa_version(void) { return "0.1.0"; }
 extern "C" int pa_device_error(int* out) {
   if (!out) return PA_ERR_INVALID;
   if (cudaDeviceSynchronize() != cudaSuccess) return PA_ERR_CUDA;
-  unsigned int a = 0, b = 0, c = 0, d = 0;
+  unsigned int a = 0, b = 0, c = 0, d = 0, e = 0;
   int s;
   if ((s = pa__err_write_kv(&a)) != PA_OK) return s;
   if ((s = pa__err_decode(&b)) != PA_OK) return s;
   if ((s = pa__err_prefill(&c)) != PA_OK) return s;
   if ((s = pa__err_rope(&d)) != PA_OK) return s;
-  *out = (int)(a | b | c | d);
+  if ((s = pa__err_int8(&e)) != PA_OK) return s;
+  *out = (int)(a | b | c | d | e);
   return PA_OK;
 }
 
@@ -67,6 +69,12 @@ static EncodeTiledFn get_encode() {
 
 int encode_2d_sw128(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t row_stride_bytes,
                     uint32_t box_cols, uint32_t box_rows) {
+  return encode_2d_u16(map, base, cols, rows, row_stride_bytes, box_cols, box_rows, 128);
+}
+
+int encode_2d_u16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t row_stride_bytes,
+                  uint32_t box_cols, uint32_t box_rows, uint32_t swizzle_bytes) {
+  if (swizzle_bytes != 128 && swizzle_bytes != 64) return PA_ERR_CUDA;
   EncodeTiledFn fn = get_encode();
   if (!fn) return PA_ERR_CUDA;
   cuuint64_t dims[2] = {cols, rows};
@@ -74,7 +82,9 @@ int encode_2d_sw128(CUtensorMap* map, const void* base, uint64_t cols, uint64_t 
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
 }

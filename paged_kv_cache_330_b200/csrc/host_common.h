@@ -22,6 +22,10 @@ inline bool valid_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || 
 int encode_2d_sw128(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t row_stride_bytes,
                     uint32_t box_cols, uint32_t box_rows);
 
+// The same with the swizzle chosen by its span in bytes (128 or 64); box_cols * 2 must equal it.
+int encode_2d_u16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t row_stride_bytes,
+                  uint32_t box_cols, uint32_t box_rows, uint32_t swizzle_bytes);
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 

@@ -8,8 +8,8 @@ CPU oracle and the CUDA path start from what it returns and derive everything
 else on their own.
 """
 
-from .synth import (CONFIGS, RopeCase, Workload, fill_cache_blocks, make_custom, make_rope_case, make_workload,
-                    new_token_positions, ops_for, rope_tables)
+from .synth import (CONFIGS, RopeCase, Workload, fill_cache_blocks, make_custom, make_prefix_groups, make_rope_case,
+                    make_workload, new_token_positions, ops_for, rope_tables)
 
 __all__ = ["CONFIGS", "Workload", "make_workload", "make_custom", "fill_cache_blocks", "ops_for", "RopeCase",
-           "make_rope_case", "new_token_positions", "rope_tables"]
+           "make_rope_case", "new_token_positions", "rope_tables", "make_prefix_groups"]

@@ -218,6 +218,49 @@ def make_custom(*, seed: int, lens, num_q_heads: int, num_kv_heads: int, head_di
                     scale=scale)
 
 
+def make_prefix_groups(*, seed: int, group_sizes, prefix_lens, suffix_lo: int, suffix_hi: int, num_q_heads: int,
+                       num_kv_heads: int, head_dim: int, block_size: int, dtype: str = "bf16",
+                       free_frac: float = 0.2) -> Workload:
+    """Groups of sequences forked from one parent each (the parent is the group's first sequence): group i has
+    group_sizes[i] members sharing its first prefix_lens[i] tokens, then every member appends a private
+    suffix of uniform[suffix_lo, suffix_hi] tokens and one new token.  Members of a group are consecutive
+    in the batch.  ``cfg`` carries "group_sizes" and "prefix_lens" for the caller."""
+    g = torch.Generator().manual_seed(int(seed))
+    sizes = [int(x) for x in group_sizes]
+    plens = [int(x) for x in prefix_lens]
+    B = sum(sizes)
+    suffix = torch.randint(suffix_lo, suffix_hi + 1, (B,), generator=g).numpy().astype(np.int32)
+    ops, first = [], 0
+    prefix_of = np.zeros(B, dtype=np.int32)
+    for n, P in zip(sizes, plens):
+        ops.append(("alloc", first, P))
+        for m in range(first + 1, first + n):
+            ops.append(("fork", first, m, P))
+        prefix_of[first:first + n] = P
+        first += n
+    for b in range(B):
+        if suffix[b] > 0:
+            ops.append(("append", b, int(suffix[b])))
+    for b in range(B):
+        ops.append(("append_new", b, 1))
+    L = (prefix_of + suffix + 1).astype(np.int32)
+    unique = sum(plens) + int((suffix + 1).sum())
+    NB = int(math.ceil((unique / block_size + 2 * B) * (1.0 + free_frac)))
+    free_order = torch.randperm(NB, generator=g).numpy().astype(np.int32)
+    dt = TORCH_DTYPES[dtype]
+    q = _randn(g, (B, num_q_heads, head_dim), dt)
+    k_new = _randn(g, (B, num_kv_heads, head_dim), dt)
+    v_new = _randn(g, (B, num_kv_heads, head_dim), dt)
+    k_cache0 = _randn(g, (NB, block_size, num_kv_heads, head_dim), dt)
+    v_cache0 = _randn(g, (NB, block_size, num_kv_heads, head_dim), dt)
+    cfg = dict(kind="prefix_groups", batch=B, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads, head_dim=head_dim,
+               block_size=block_size, dtype=dtype, seed=seed, group_sizes=sizes, prefix_lens=plens)
+    scale = float(np.float32(1.0) / np.sqrt(np.float32(head_dim)))
+    return Workload(name="prefix_groups", cfg=cfg, ops=ops, free_order=free_order, num_blocks=NB, context_lens=L,
+                    q=q, k_new=k_new, v_new=v_new, k_cache0=k_cache0, v_cache0=v_cache0, query_start_loc=None,
+                    scale=scale)
+
+
 def new_token_positions(wl: Workload) -> np.ndarray:
     """int64 [T]: the index within its sequence of every token written this step, in the order of the
     ``append_new`` entries (the row order of k_new/v_new).  Pool-script bookkeeping only."""
