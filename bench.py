@@ -409,6 +409,23 @@ def run_ours(args):
         def dec(st):
             pa.decode_int8(q, kq, vq, ksc, vsc, btd, lensd, maxL, wl.scale, out=out, workspace=work,
                            num_partitions=args.num_partitions, stream=st)
+    elif args.cascade:  # shared prefixes read once for all sharers (groups of consecutive sequences)
+        if c["kind"] != "prefix":
+            raise SystemExit("--cascade needs the prefix-shared workload")
+        kc = wl.k_cache0.to(dev)
+        vc = wl.v_cache0.to(dev)
+        per = B // c["groups"]
+        gsd = torch.arange(0, B + 1, per, dtype=torch.int32, device=dev)
+        spd = torch.full((B,), c["prefix_len"], dtype=torch.int32, device=dev)
+        work = torch.zeros(pa.decode_cascade_workspace_size(B, Hq, Hkv, D, maxL, c["groups"], per, c["prefix_len"],
+                                                            args.num_partitions), dtype=torch.uint8, device=dev)
+
+        def wr(st):
+            pa.write_kv(kn, vn, smd, kc, vc, stream=st)
+
+        def dec(st):
+            pa.decode_cascade(q, kc, vc, btd, lensd, maxL, wl.scale, gsd, spd, per, c["prefix_len"], out=out,
+                              workspace=work, num_partitions=args.num_partitions, stream=st)
     else:
         kc = wl.k_cache0.to(dev)
         vc = wl.v_cache0.to(dev)
@@ -545,7 +562,7 @@ def run_ours(args):
     achieved = alg / (dec_avg * 1e-3) / 1e9
     tr = NCU_TRAFFIC.get(args.workload + ("_int8" if int8 else ""))
     traffic = tr["bytes"] if tr and tr.get("src") == kernel_source_hash(tr["files"]) else None
-    launches_per_step = 2  # write_kv, decode (split-K merge inside)
+    launches_per_step = 3 if args.cascade else 2  # write_kv, decode (split-K merge inside)[, shared-prefix pass]
     if rank == 0:
         cpu = None
         if ws == 1 and not args.no_cpu_baseline:
@@ -558,6 +575,7 @@ def run_ours(args):
             "dtype": str(c["dtype"]) + ("+int8 cache" if int8 else ""), "data": "synthetic",
             "config": {"workload": WORKLOAD_TEXT.get(args.workload, args.workload), "global_batch": int(seqs_all),
                        "kv_cache": "int8 codes + fp32 row scales" if int8 else str(c["dtype"]),
+                       "decode": "cascade over shared prefixes" if args.cascade else "per-sequence",
                        "block_size": int(c["block_size"]),
                        "parallelism": f"dp{ws} (independent replicas)", "l2": "inputs larger than L2 (no flush)",
                        "decode_grid": grid, "repeats": args.repeats,
@@ -571,8 +589,10 @@ def run_ours(args):
                            "then binding.write_kv and binding.decode (argument checks, ctypes, tensor-map "
                            "encode, launch), then D2H of out; median of repeats",
                     "graph_replay": {"value": kv_all / (e2e_graph_ms * 1e-3) / 1e9, "ms_per_step": e2e_graph_ms}},
-            "roofline": {"bound": "hbm", "kernel": ("pa_decode_int8" if int8 else "pa_decode") +
-                         " (one kernel: gather, attention, split-K merge)",
+            "roofline": {"bound": "hbm", "kernel": ("pa_decode_int8" if int8 else
+                                                    "pa_decode_cascade (suffix decode + shared-prefix pass)"
+                                                    if args.cascade else "pa_decode") +
+                         ("" if args.cascade else " (one kernel: gather, attention, split-K merge)"),
                          "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "algorithmic_bytes": alg,
                          "avg_launch_ms": dec_avg, "avg_launch_ms_repeats": dec_ms,
@@ -908,6 +928,8 @@ def main():
     ap.add_argument("--steps-per-graph", type=int, default=10, help="whole steps captured per CUDA graph")
     ap.add_argument("--repeats", type=int, default=5, help="timed K-step loops; the median is reported")
     ap.add_argument("--block-size", type=int, default=None, help="override the workload's block size")
+    ap.add_argument("--cascade", action="store_true",
+                    help="prefix-shared workload: read each shared prefix once for all sharers (pa_decode_cascade)")
     ap.add_argument("--kv", choices=["bf16", "int8"], default="bf16",
                     help="decode workloads: the cache format (int8 = codes + fp32 row scales)")
     ap.add_argument("--ref-budget", type=float, default=12.0, help="seconds of oracle time per reference sample")

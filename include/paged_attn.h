@@ -155,6 +155,7 @@ int pa_rope_write_kv(const void* q, void* q_out, const void* k, const void* v, c
 /* pa_decode_plan: the grid and workspace the call will use on the current   */
 /* device.  num_partitions_or_0 > 0 fixes the number of CTAs (the number of  */
 /* parts the chunk line is cut into); 0 fills the GPU (SMs x CTAs per SM).   */
+/* max_pieces_out: partial slots of the workspace, batch*Hkv + grid.        */
 /* max_context_len is only checked here (>= 0).  Output pointers may be NULL.*/
 /* ------------------------------------------------------------------------ */
 int pa_decode_plan(int batch, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len,

@@ -85,12 +85,14 @@ struct DecodeParams {
 
 enum : int { F_FIRST = 1, F_LAST = 2, F_DIRECT = 4, F_END = 8 };
 
-// One stage as the producer planned it.  c0/npieces (set on a piece's last
-// stage) name the first CTA holding a piece of this segment and how many
-// pieces the segment has, for the merge.
+// One stage as the producer planned it.  vid: the CTA that walks it; its piece's partial goes to workspace
+// slot segment + vid.  c0/npieces (set on a piece's last stage) name the first CTA holding a piece of this
+// segment and how many pieces the segment has, for the merge.
 struct StageMeta {
-  int b, g, tok0, ntok, flags, nchunk, c0, npieces;
+  int b, g, tok0, ntok, flags, vid, c0, npieces;
 };
+
+__device__ __forceinline__ int stage_chunks(const StageMeta& d) { return (d.ntok + 15) / 16; }
 
 // Shared-memory layout of one CTA.  Q8: the cache holds int8 codes (one byte per element) and per-token
 // fp32 scales, which each stage carries next to the codes.
@@ -123,7 +125,8 @@ struct Layout {
   static constexpr int MB_BYTES = (MB_DESC + (int)sizeof(StageMeta) + 15) / 16 * 16;
   static constexpr int M_OFF = P_OFF + P_BYTES;
   static constexpr int WTS_OFF = M_OFF + 2 * MB_BYTES;                        // merge weights fp32 [G][kMaxPieces]
-  static constexpr int MISC_OFF = WTS_OFF + G * kMaxPieces * 4;               // int64 total chunks on the line
+  static constexpr int VIDS_OFF = WTS_OFF + G * kMaxPieces * 4;               // merge: slot of each piece, int32
+  static constexpr int MISC_OFF = VIDS_OFF + kMaxPieces * 4;                  // int64 total chunks on the line
   static constexpr int BAR_OFF = MISC_OFF + 16;  // full[NSTAGES], empty[NSTAGES], mfull[2], mempty[2]
   static constexpr int BYTES = BAR_OFF + (2 * NSTAGES + 4) * 8;
   static constexpr int ALLOC = BYTES + 1024;                                  // slack for 1024-byte alignment
@@ -366,7 +369,11 @@ struct CoreConsumer {
 };
 
 // ------------------------------------------------------------------ tensor-core consumer (G >= 8)
-template <int DT, int D, int G, int NW, int NSTAGES>
+// LO_ALL: P always enters PV as hi + lo (exact to ~2^-17).  Otherwise the lo term's products are issued
+// only for a tile in which some row's share of its running softmax mass is at least 1/16 (the first tile,
+// and tiles holding dominant keys); elsewhere the hi term alone moves an output by at most 2^-9 of that
+// tile's share of |v|, which is under 1/16 of the row's mass.
+template <int DT, int D, int G, int NW, int NSTAGES, bool LO_ALL = true>
 struct MmaConsumer {
   using LY = Layout<D, G, NW, NSTAGES, true>;
   static constexpr int KS = D / 16;   // k-steps of QK^T
@@ -454,6 +461,9 @@ struct MmaConsumer {
     }
     l[0] = l[0] * al0 + ls0;
     l[1] = l[1] * al1 + ls1;
+    // this lane's columns of the tile against this lane's columns of the running sum (both partial sums
+    // over the same column subset)
+    const bool lo = LO_ALL || __any_sync(0xffffffffu, ls0 >= 0.0625f * l[0] || ls1 >= 0.0625f * l[1]);
 #pragma unroll
     for (int n = 0; n < ND; ++n) {
       o[n][0] *= al0; o[n][1] *= al0;
@@ -478,8 +488,10 @@ struct MmaConsumer {
         }
         mma16816<DT>(o[dp * 2], ph[j][0], ph[j][1], ph[j][2], ph[j][3], b0, b1);
         mma16816<DT>(o[dp * 2 + 1], ph[j][0], ph[j][1], ph[j][2], ph[j][3], b2, b3);
-        mma16816<DT>(o[dp * 2], pl[j][0], pl[j][1], pl[j][2], pl[j][3], b0, b1);
-        mma16816<DT>(o[dp * 2 + 1], pl[j][0], pl[j][1], pl[j][2], pl[j][3], b2, b3);
+        if (lo) {
+          mma16816<DT>(o[dp * 2], pl[j][0], pl[j][1], pl[j][2], pl[j][3], b0, b1);
+          mma16816<DT>(o[dp * 2 + 1], pl[j][0], pl[j][1], pl[j][2], pl[j][3], b2, b3);
+        }
       }
     }
   }
@@ -613,9 +625,10 @@ struct Q8Consumer {
     }
   }
 
-  // One 32-token tile: rows r0 .. r0+31 of the stage, nv of them valid.  skb/svb: the stage's scales.
-  __device__ __forceinline__ void tile(uint32_t kbase, uint32_t vbase, const float* skb, const float* svb, int r0,
-                                       int nv, int lane) {
+  // One 32-token tile: rows r0 .. r0+31 of the stage, nv of them valid.  skb/svb: shared-memory addresses of
+  // the stage's fp32 K and V scales.
+  __device__ __forceinline__ void tile(uint32_t kbase, uint32_t vbase, uint32_t skb, uint32_t svb, int r0, int nv,
+                                       int lane) {
     const int g = lane >> 2, c = lane & 3;
     // ---- S^T = K q^T: 2 m-tiles of 16 tokens x NT n-tiles of 8 heads
     float s[2][NT][4];
@@ -652,8 +665,8 @@ struct Q8Consumer {
       for (int hh = 0; hh < 2; ++hh) {
         const int t = 16 * mt + g + 8 * hh;  // token within the tile
         const bool ok = t < nv;
-        const float sk = skb[r0 + t] * qs;
-        const float sv = svb[r0 + t];
+        const float sk = __uint_as_float(lds32(skb + (r0 + t) * 4)) * qs;
+        const float sv = __uint_as_float(lds32(svb + (r0 + t) * 4));
         lsv[mt][hh] = (ok && sv > 0.f) ? __log2f(sv) : -INFINITY;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -782,6 +795,7 @@ struct Walker {
   int win_base, win_len;      // lens window: lane i holds the clamped length of sequence win_base + i
   int batch, hkv, cap, grid;
   long long total;            // chunks on the whole line
+  int vid;                    // this CTA (see StageMeta)
   const int32_t* lens;
   const int32_t* starts;      // per-sequence first token (null: 0); the walk sees L - start tokens
   // sub-ranges still to walk after the current one, in order (at most two)
@@ -896,7 +910,7 @@ __device__ __forceinline__ StageMeta walker_next(Walker& w, int cta, int lane) {
   }
   if (w.pos >= w.end) {
     d.flags = F_END;
-    d.b = d.g = d.tok0 = d.ntok = d.nchunk = d.c0 = d.npieces = 0;
+    d.b = d.g = d.tok0 = d.ntok = d.vid = d.c0 = d.npieces = 0;
     return d;
   }
   const long long seg_end = w.seg_start + w.nch;
@@ -908,10 +922,10 @@ __device__ __forceinline__ StageMeta walker_next(Walker& w, int cta, int lane) {
   d.tok0 = (int)(w.pos - w.seg_start) * kChunk;
   const int tok1 = min((int)(stop - w.seg_start) * kChunk, w.L);
   d.ntok = tok1 - d.tok0;
-  d.nchunk = (int)(stop - w.pos);
+  d.vid = w.vid;
   d.flags = (w.pos == w.piece_start ? F_FIRST : 0) | (stop == piece_end ? F_LAST : 0) |
             (w.piece_start == w.seg_start && piece_end == seg_end ? F_DIRECT : 0);
-  d.c0 = cta;
+  d.c0 = w.vid;
   d.npieces = 1;
   if ((d.flags & F_LAST) && !(d.flags & F_DIRECT)) {
     const long long c0 = owner_of(w.seg_start, w.total, w.grid), c1 = owner_of(seg_end - 1, w.total, w.grid);
@@ -937,7 +951,7 @@ __device__ __forceinline__ StageMeta walker_next(Walker& w, int cta, int lane) {
 
 // ------------------------------------------------------------------ decode kernel
 template <int DT, int D, int G, int NW, int NSTAGES, bool MMA, bool Q8>
-__global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_constant__ CUtensorMap kmap,
+__global__ void __launch_bounds__((NW + 2) * 32, Q8 ? 3 : 1) decode_kernel(const __grid_constant__ CUtensorMap kmap,
                                                                const __grid_constant__ CUtensorMap vmap,
                                                                const DecodeParams p) {
   using LY = Layout<D, G, NW, NSTAGES, MMA, Q8>;
@@ -1011,6 +1025,7 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
     w.cap = cap;
     w.grid = p.grid;
     w.total = C;
+    w.vid = cta;
     w.lens = p.context_lens;
     w.starts = p.ctx_start;
     w.win_base = -64;
@@ -1046,7 +1061,7 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
       const StageMeta dn = walker_next<LY::CPS>(w, cta, lane);
       const int slot = j % kPlanRing;
       if (lane == 0) plan[slot] = dn;
-      if (!(dn.flags & F_END) && lane < dn.nchunk)
+      if (!(dn.flags & F_END) && lane < stage_chunks(dn))
         cp_async4(plan_phys + slot * 8 + lane,
                   bt_all + (size_t)dn.b * mb + (start_of(p.ctx_start, dn.b) + dn.tok0 + lane * kChunk) / bs);
       cp_async_commit();
@@ -1062,7 +1077,8 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
       cp_async_wait<kLookahead - 1>();  // this lane's lookups for stage k have landed
       __syncwarp();
       const StageMeta d = plan[k % kPlanRing];
-      const int phys = lane < d.nchunk ? plan_phys[(k % kPlanRing) * 8 + lane] : 0;
+      const int nchunk = stage_chunks(d);
+      const int phys = lane < nchunk ? plan_phys[(k % kPlanRing) * 8 + lane] : 0;
       const int st = k % NSTAGES;
       if (k >= NSTAGES && !mbar_wait(&empty[st], ((k / NSTAGES) - 1) & 1)) {
         ok = false;
@@ -1076,9 +1092,9 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
       const bool first = d.flags & F_FIRST;
       constexpr uint32_t kChunkBytes = kChunk * LY::ROWB * 2 + (Q8 ? 2 * kChunk * 4 : 0);  // K + V (+ scales)
       if (lane == 0)
-        mbar_arrive_expect_tx(&full[st], (uint32_t)d.nchunk * kChunkBytes + (first ? LY::QSLOT : 0));
+        mbar_arrive_expect_tx(&full[st], (uint32_t)nchunk * kChunkBytes + (first ? LY::QSLOT : 0));
       __syncwarp();
-      if (lane < d.nchunk) {
+      if (lane < nchunk) {
         const bool in_range = phys >= 0 && phys < p.num_blocks;
         if (!in_range) PA_RECORD_ERROR(PA_ERRBIT_INDEX);  // TMA zero-fills out of range
         const int tok = start_of(p.ctx_start, d.b) + d.tok0 + lane * kChunk;  // token of the sequence
@@ -1138,7 +1154,7 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
       const StageMeta d = *reinterpret_cast<const StageMeta*>(mb + LY::MB_DESC);
       if (d.flags & F_END) break;
       const bool direct = d.flags & F_DIRECT;
-      const size_t slot = (size_t)d.b * p.num_kv_heads + d.g + cta;
+      const size_t slot = (size_t)d.b * p.num_kv_heads + d.g + d.vid;
       T* outp = reinterpret_cast<T*>(p.out) + ((size_t)d.b * p.num_q_heads + (size_t)d.g * G) * D;
       for (int i = lane; i < G * D; i += 32) {
         const int h = i / D, dd = i - h * D;
@@ -1187,37 +1203,56 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
           for (long long k2 = d.c0, m2 = 0;; ++k2)
             if (C_s * k2 / p.grid != C_s * (k2 + 1) / p.grid && m2++ == n) return k2;
         };
-        // Normalised weight of each piece per head, w[h][n] = 2^(m_n - M) / sum_n 2^(m_n - M) l_n;
-        // then out = sum_n w[h][n] o_n with every load independent, so the merge costs a few L2
-        // round trips instead of one per element.
+        // Normalised weight of each piece per head, w[h][n] = 2^(m_n - M) / sum_n 2^(m_n - M) l_n, with
+        // lane n holding piece n (its m and l loads all independent, the max and sum by warp shuffles);
+        // then out = sum_n w[h][n] o_n with the pieces' loads issued four at a time.  The merge so costs
+        // a few L2 round trips, not one per piece.
         float* wts = reinterpret_cast<float*>(smem + LY::WTS_OFF);
+        int* vids = reinterpret_cast<int*>(smem + LY::VIDS_OFF);
         const int np = d.npieces;
         if (np <= kMaxPieces) {
-          for (int h = lane; h < G; h += 32) {
-            float Mh = -INFINITY, den = 0.f;
-            for (int n = 0; n < np; ++n) Mh = fmaxf(Mh, __ldcg(p.ws_m + ((size_t)sg + piece_cta(n)) * G + h));
-            for (int n = 0; n < np; ++n) {
-              const size_t srow = ((size_t)sg + piece_cta(n)) * G + h;
-              const float w = fast_exp2(__ldcg(p.ws_m + srow) - Mh);
-              wts[h * np + n] = w;
-              den = fmaf(w, __ldcg(p.ws_l + srow), den);
+          const size_t myrow = lane < np ? ((size_t)sg + piece_cta(lane)) * G : 0;
+          if (lane < np) vids[lane] = (int)(myrow / G - sg);
+#pragma unroll 1
+          for (int h0 = 0; h0 < G; h0 += 4) {
+            float mh[4], lh[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const bool on = lane < np && h0 + e < G;
+              mh[e] = on ? __ldcg(p.ws_m + myrow + h0 + e) : -INFINITY;
+              lh[e] = on ? __ldcg(p.ws_l + myrow + h0 + e) : 0.f;
             }
-            const float inv = 1.f / den;
-            if (p.lse) p.lse[(size_t)d.b * p.num_q_heads + (size_t)d.g * G + h] = (Mh + __log2f(den)) * kLn2;
-            for (int n = 0; n < np; ++n) wts[h * np + n] *= inv;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              if (h0 + e >= G) break;
+              const float Mh = warp_max(mh[e]);
+              const float w = lane < np ? fast_exp2(mh[e] - Mh) : 0.f;
+              const float den = warp_sum(w * lh[e]);
+              if (lane < np) wts[(h0 + e) * np + lane] = w / den;
+              if (p.lse && lane == 0)
+                p.lse[(size_t)d.b * p.num_q_heads + (size_t)d.g * G + h0 + e] = (Mh + __log2f(den)) * kLn2;
+            }
           }
           __syncwarp();
           T* outp = reinterpret_cast<T*>(p.out) + ((size_t)d.b * p.num_q_heads + (size_t)d.g * G) * D;
-#pragma unroll 4
+#pragma unroll 1
           for (int i0 = lane * 4; i0 < G * D; i0 += 128) {
             const int h = i0 / D, dd = i0 - h * D;
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int n = 0; n < np; ++n) {
-              const float w = wts[h * np + n];
-              const float4 o4 = __ldcg(reinterpret_cast<const float4*>(
-                  p.ws_o + (((size_t)sg + piece_cta(n)) * G + h) * D + dd));
-              acc.x = fmaf(w, o4.x, acc.x); acc.y = fmaf(w, o4.y, acc.y);
-              acc.z = fmaf(w, o4.z, acc.z); acc.w = fmaf(w, o4.w, acc.w);
+#pragma unroll 1
+            for (int n0 = 0; n0 < np; n0 += 4) {
+              float4 o4[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                o4[e] = n0 + e < np ? __ldcg(reinterpret_cast<const float4*>(
+                                          p.ws_o + (((size_t)sg + vids[n0 + e]) * G + h) * D + dd))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float w = n0 + e < np ? wts[h * np + n0 + e] : 0.f;
+                acc.x = fmaf(w, o4[e].x, acc.x); acc.y = fmaf(w, o4[e].y, acc.y);
+                acc.z = fmaf(w, o4[e].z, acc.z); acc.w = fmaf(w, o4[e].w, acc.w);
+              }
             }
             uint2 pk;
             pk.x = Elt<DT>::from_f2(acc.x, acc.y);
@@ -1299,8 +1334,8 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
       const uint32_t kb = sbase + LY::K_OFF + st * LY::STAGE_BYTES;
       const uint32_t vb = sbase + LY::V_OFF + st * LY::STAGE_BYTES;
       if constexpr (Q8)
-        c.tile(kb, vb, reinterpret_cast<const float*>(smem + LY::SK_OFF) + st * LY::TOK,
-               reinterpret_cast<const float*>(smem + LY::SV_OFF) + st * LY::TOK, warp * 32, nv, lane);
+        c.tile(kb, vb, sbase + LY::SK_OFF + st * LY::TOK * 4, sbase + LY::SV_OFF + st * LY::TOK * 4, warp * 32, nv,
+               lane);
       else if constexpr (MMA)
         c.tile(kb, vb, p.scale_log2, warp * 32, nv, lane);
       else
@@ -1329,7 +1364,9 @@ __global__ void __launch_bounds__((NW + 2) * 32) decode_kernel(const __grid_cons
 // group) and the split's share of the prefix's 16-token chunks.  One producer warp bulk-copies the q rows
 // and gathers K/V boxes through the first member's block table with TMA into a 2-stage ring; four
 // consumer warps own 16 rows each and run every 64-token stage through the warp-MMA consumer (QK^T and PV
-// on mma.m16n8k16, P as hi + lo 16-bit terms, fp32 online softmax).  Each CTA writes fp32 (m, l, o) per
+// on mma.m16n8k16, fp32 online softmax; P as its high 16-bit term, plus the low term for tiles that carry
+// at least 1/16 of some row's running mass).  The pass is bound by the warp-MMA rate, so the low term's
+// products are spent only where they change the result measurably.  Each CTA writes fp32 (m, l, o) per
 // row; the CTA that completes a row tile's last split (atomic count, no waiting) merges the splits with
 // the suffix part and writes out.
 
@@ -1350,9 +1387,9 @@ struct CascadeParams {
   float scale_log2;
 };
 
-template <int D, int NSTAGES>
+template <int D, int NSTAGES, int CT>
 struct CasLayout {
-  static constexpr int TOK = 64;
+  static constexpr int TOK = CT * kChunk;  // tokens per stage (CT chunks)
   static constexpr int HALVES = D / 64;
   static constexpr int STAGE_BYTES = TOK * D * 2;
   static constexpr int K_OFF = 0;
@@ -1364,11 +1401,11 @@ struct CasLayout {
   static constexpr int ALLOC = BYTES + 1024;
 };
 
-template <int DT, int D, int G, int NSTAGES>
-__global__ void __launch_bounds__(160) cascade_prefix_kernel(const __grid_constant__ CUtensorMap kmap,
-                                                             const __grid_constant__ CUtensorMap vmap,
-                                                             const CascadeParams p) {
-  using LY = CasLayout<D, NSTAGES>;
+template <int DT, int D, int G, int NSTAGES, int CT, int MINB>
+__global__ void __launch_bounds__(160, MINB) cascade_prefix_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                                   const __grid_constant__ CUtensorMap vmap,
+                                                                   const CascadeParams p) {
+  using LY = CasLayout<D, NSTAGES, CT>;
   using T = typename Elt<DT>::T;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1436,10 +1473,10 @@ __global__ void __launch_bounds__(160) cascade_prefix_kernel(const __grid_consta
     const int32_t* bt = p.block_tables + (size_t)gs * p.max_blocks_per_seq;
     const int bs = p.block_size;
     bool ok = true;
-    // block of this lane's chunk of stage k (lanes 0..3), fetched one stage ahead
+    // block of this lane's chunk of stage k (lanes 0..CT-1), fetched one stage ahead
     auto lookup = [&](int k) -> int {
-      const int c = c_begin + k * 4 + lane;
-      return (lane < 4 && c < c_end) ? __ldg(bt + (c * kChunk) / bs) : 0;
+      const int c = c_begin + k * CT + lane;
+      return (lane < CT && c < c_end) ? __ldg(bt + (c * kChunk) / bs) : 0;
     };
     int phys = lookup(0);
     int k = 0;
@@ -1450,12 +1487,12 @@ __global__ void __launch_bounds__(160) cascade_prefix_kernel(const __grid_consta
         ok = false;
         break;
       }
-      const int nch = min(4, c_end - (c_begin + k * 4));
+      const int nch = min(CT, c_end - (c_begin + k * CT));
       if (lane == 0) mbar_arrive_expect_tx(&full[st], (uint32_t)(nch * kChunk * D * 2 * 2));
       __syncwarp();
       if (lane < nch) {
         if (phys < 0 || phys >= p.num_blocks) PA_RECORD_ERROR(PA_ERRBIT_INDEX);  // TMA zero-fills out of range
-        const int tok = (c_begin + k * 4 + lane) * kChunk;
+        const int tok = (c_begin + k * CT + lane) * kChunk;
         const int y = phys * bs + (tok % bs);
         uint8_t* kd = smem + LY::K_OFF + st * LY::STAGE_BYTES + lane * kChunk * 128;
         uint8_t* vd = smem + LY::V_OFF + st * LY::STAGE_BYTES + lane * kChunk * 128;
@@ -1478,7 +1515,7 @@ __global__ void __launch_bounds__(160) cascade_prefix_kernel(const __grid_consta
   }
 
   // =================================================== consumer warps (16 rows each)
-  MmaConsumer<DT, D, 16, 2, NSTAGES> c;
+  MmaConsumer<DT, D, 16, CT / 2, NSTAGES, false> c;  // its stage layout: CT/2 x 32 tokens; lo term on demand
   c.init();
   bool ok = mbar_wait(qbar, 0);
   if (ok) c.load_q(smem + LY::Q_OFF + warp * 16 * D * 2, nullptr, 0.f, lane);
@@ -1491,8 +1528,9 @@ __global__ void __launch_bounds__(160) cascade_prefix_kernel(const __grid_consta
     const int ntok = min(LY::TOK, my_tok - k * LY::TOK);
     const uint32_t kb = sbase + LY::K_OFF + st * LY::STAGE_BYTES;
     const uint32_t vb = sbase + LY::V_OFF + st * LY::STAGE_BYTES;
-    c.tile(kb, vb, p.scale_log2, 0, min(32, ntok), lane);
-    if (ntok > 32) c.tile(kb, vb, p.scale_log2, 32, ntok - 32, lane);
+#pragma unroll
+    for (int r0 = 0; r0 < LY::TOK; r0 += 32)
+      if (r0 < ntok) c.tile(kb, vb, p.scale_log2, r0, min(32, ntok - r0), lane);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
   }
@@ -1564,13 +1602,19 @@ __global__ void __launch_bounds__(160) cascade_prefix_kernel(const __grid_consta
 }
 
 // ------------------------------------------------------------------ host side
-constexpr int kNW = 2;        // consumer warps per CTA (64-token stages)
-constexpr int kStages = 2;    // ring depth, 16-bit cache (three CTAs per SM)
-constexpr int kStagesQ8 = 4;  // ring depth, int8 cache: the same bytes in flight per SM as the 16-bit ring
+// Consumer warps per CTA and ring depth.  16-bit cache: 2 warps (64-token stages), 2 stages, three CTAs per
+// SM.  int8 cache: a 64-token stage holds half the bytes and the int8 consumer is the bound, so 3 warps
+// (96-token stages), 2 stages and three CTAs per SM (nine consumer warps per SM; measured against 2 warps x 4
+// stages, 4 x 2 and 4 x 3 on the Qwen and Llama shapes).
+template <bool Q8>
+struct Shape {
+  static constexpr int NW = Q8 ? 3 : 2;
+  static constexpr int NS = 2;
+};
 
 template <int D, int G, bool Q8>
 constexpr int alloc_bytes() {
-  return Layout<D, G, kNW, Q8 ? kStagesQ8 : kStages, Q8 || (G >= 8), Q8>::ALLOC;
+  return Layout<D, G, Shape<Q8>::NW, Shape<Q8>::NS, Q8 || (G >= 8), Q8>::ALLOC;
 }
 
 template <bool Q8>
@@ -1627,9 +1671,9 @@ bool make_plan(int batch, int Hq, int Hkv, int D, int num_partitions, bool q8, P
 template <int DT, int D, int G, bool Q8>
 int launch(const CUtensorMap& km, const CUtensorMap& vm, const DecodeParams& p, cudaStream_t st) {
   constexpr bool MMA = Q8 || G >= 8;
-  constexpr int NS = Q8 ? kStagesQ8 : kStages;
-  using LY = Layout<D, G, kNW, NS, MMA, Q8>;
-  auto kern = decode_kernel<DT, D, G, kNW, NS, MMA, Q8>;
+  constexpr int NW = Shape<Q8>::NW, NS = Shape<Q8>::NS;
+  using LY = Layout<D, G, NW, NS, MMA, Q8>;
+  auto kern = decode_kernel<DT, D, G, NW, NS, MMA, Q8>;
   // per instantiation and device; host threads may race to set it, which only repeats an idempotent call
   static std::atomic<bool> attr_set[64] = {};
   int dev = 0;
@@ -1643,7 +1687,7 @@ int launch(const CUtensorMap& km, const CUtensorMap& vm, const DecodeParams& p, 
   // its dependents at entry); the producer waits for it before the first cache load
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.grid);
-  cfg.blockDim = dim3((kNW + 2) * 32);
+  cfg.blockDim = dim3((NW + 2) * 32);
   cfg.dynamicSmemBytes = LY::ALLOC;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -1785,9 +1829,13 @@ int decode_prepare(const void* q, const void* k_cache, const void* v_cache, cons
   const uint64_t rows = (uint64_t)std::max(num_blocks, 1) * block_size;
   const uint64_t row_bytes = (uint64_t)num_kv_heads * head_dim * (q8 ? 1 : 2);
   const uint32_t box_bytes = (q8 && head_dim == 64) ? 64u : 128u;
-  if (pa::encode_2d_u16(&call->km, k_cache, row_bytes / 2, rows, row_bytes, box_bytes / 2, 16, box_bytes) != PA_OK)
+  // L2 fills match one head's row: 256 bytes for a 16-bit row of head_dim 128, 128 bytes for int8 rows
+  const uint32_t fill = (uint32_t)head_dim * (q8 ? 1 : 2) >= 256 ? 256u : 128u;
+  if (pa::encode_2d_u16(&call->km, k_cache, row_bytes / 2, rows, row_bytes, box_bytes / 2, 16, box_bytes, fill) !=
+      PA_OK)
     return PA_ERR_CUDA;
-  if (pa::encode_2d_u16(&call->vm, v_cache, row_bytes / 2, rows, row_bytes, box_bytes / 2, 16, box_bytes) != PA_OK)
+  if (pa::encode_2d_u16(&call->vm, v_cache, row_bytes / 2, rows, row_bytes, box_bytes / 2, 16, box_bytes, fill) !=
+      PA_OK)
     return PA_ERR_CUDA;
   call->dtype = dtype;
   call->head_dim = head_dim;
@@ -1859,7 +1907,10 @@ extern "C" int pa_decode_int8(const void* q, const void* k_codes, const void* v_
 // ------------------------------------------------------------------ cascade decode (shared prefixes)
 namespace {
 
+// Prefix pass ring: stages of kCasChunks 16-token chunks, kCasStages deep, kCasMinBlocks CTAs per SM.
 constexpr int kCasStages = 2;
+constexpr int kCasChunks = 4;
+constexpr int kCasMinBlocks = 2;
 
 struct CascadePlan {
   Plan dec;
@@ -1874,9 +1925,11 @@ bool make_cascade_plan(int batch, int Hq, int Hkv, int D, int num_partitions, in
   const int G = Hq / Hkv;
   cp->tiles = std::max(1, (max_group_size * G + kCasRows - 1) / kCasRows);
   cp->units = num_groups * Hkv * cp->tiles;
-  const int target = pa::sm_count() * 2;  // two CTAs per SM
+  // as many splits as keep the grid within one wave of two CTAs per SM (a partial second wave would double
+  // the pass), at least one, at most one per 64-token stage of the longest prefix
+  const int wave = pa::sm_count() * kCasMinBlocks;
   const int by_work = std::max(1, max_prefix_len / 64);
-  cp->splits = cp->units > 0 ? std::max(1, std::min(by_work, (target + cp->units - 1) / cp->units)) : 1;
+  cp->splits = cp->units > 0 ? std::max(1, std::min(by_work, wave / cp->units)) : 1;
   const size_t slots = (size_t)cp->units * cp->splits;
   cp->off_lse = align256(cp->dec.ws_bytes);
   cp->off_cnt = cp->off_lse + align256((size_t)batch * Hq * 4);
@@ -1889,8 +1942,8 @@ bool make_cascade_plan(int batch, int Hq, int Hkv, int D, int num_partitions, in
 
 template <int DT, int D, int G>
 int launch_cascade(const CUtensorMap& km, const CUtensorMap& vm, const CascadeParams& cp, int grid, cudaStream_t st) {
-  using LY = CasLayout<D, kCasStages>;
-  auto kern = cascade_prefix_kernel<DT, D, G, kCasStages>;
+  using LY = CasLayout<D, kCasStages, kCasChunks>;
+  auto kern = cascade_prefix_kernel<DT, D, G, kCasStages, kCasChunks, kCasMinBlocks>;
   static std::atomic<bool> attr_set[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;

@@ -73,7 +73,7 @@ int encode_2d_sw128(CUtensorMap* map, const void* base, uint64_t cols, uint64_t 
 }
 
 int encode_2d_u16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t row_stride_bytes,
-                  uint32_t box_cols, uint32_t box_rows, uint32_t swizzle_bytes) {
+                  uint32_t box_cols, uint32_t box_rows, uint32_t swizzle_bytes, uint32_t l2_fill_bytes) {
   if (swizzle_bytes != 128 && swizzle_bytes != 64) return PA_ERR_CUDA;
   EncodeTiledFn fn = get_encode();
   if (!fn) return PA_ERR_CUDA;
@@ -84,7 +84,7 @@ int encode_2d_u16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t ro
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE,
                   swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  l2_fill_bytes == 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B : CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
 }

@@ -22,9 +22,11 @@ inline bool valid_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || 
 int encode_2d_sw128(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t row_stride_bytes,
                     uint32_t box_cols, uint32_t box_rows);
 
-// The same with the swizzle chosen by its span in bytes (128 or 64); box_cols * 2 must equal it.
+// The same with the swizzle chosen by its span in bytes (128 or 64; box_cols * 2 must equal it) and the
+// L2 fill granularity (256 or 128 bytes: a box row of 128 bytes takes 128, so that a fill does not bring
+// in the neighbouring head's row).
 int encode_2d_u16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t row_stride_bytes,
-                  uint32_t box_cols, uint32_t box_rows, uint32_t swizzle_bytes);
+                  uint32_t box_cols, uint32_t box_rows, uint32_t swizzle_bytes, uint32_t l2_fill_bytes = 256);
 
 // Number of SMs of the current device (cached per device).
 int sm_count();

@@ -44,6 +44,7 @@
 // as a polynomial on the FMA pipe to relieve the MUFU unit.
 
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 #include "host_common.h"
@@ -798,14 +799,15 @@ extern "C" int pa_prefill_chunk(const void* q, const int32_t* query_start_loc, i
   if (pa::encode_2d_sw128(&vm, v_cache, cols, rows, cols * 2, 64, 16) != PA_OK) return PA_ERR_CUDA;
 
   auto kern = dtype == PA_BF16 ? prefill_kernel<PA_BF16> : prefill_kernel<PA_F16>;
-  static bool attr_set[2][64] = {};
+  // per dtype and device; host threads may race to set it, which only repeats an idempotent call
+  static std::atomic<bool> attr_set[2][64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
   const int di = dtype == PA_BF16 ? 1 : 0;
-  if (dev < 0 || dev >= 64 || !attr_set[di][dev]) {
+  if (dev < 0 || dev >= 64 || !attr_set[di][dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC) != cudaSuccess)
       return PA_ERR_CUDA;
-    if (dev >= 0 && dev < 64) attr_set[di][dev] = true;
+    if (dev >= 0 && dev < 64) attr_set[di][dev].store(true, std::memory_order_release);
   }
   kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, (cudaStream_t)stream>>>(km, vm, p);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
