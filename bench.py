@@ -64,7 +64,11 @@ DECODE_SRC = ("decode.cu", "common.cuh")
 PREFILL_SRC = ("prefill.cu", "common.cuh")
 ROPE_SRC = ("rope_write_kv.cu", "common.cuh")
 NCU_TRAFFIC = {
-    "qwen_decode": {"bytes": 313_465_088, "src": "84d9feaada7e0320", "files": DECODE_SRC},
+    "qwen_decode": {"bytes": 313_008_640, "src": "4eb4742cfc8cb957", "files": DECODE_SRC},
+    "qwen_decode_int8": {"bytes": 165_265_408, "src": "4eb4742cfc8cb957", "files": DECODE_SRC},
+    "llama70b_long_int8": {"bytes": 843_906_048, "src": "4eb4742cfc8cb957", "files": DECODE_SRC},
+    # both kernels of one cascade call at block size 16 (suffix decode + shared-prefix pass)
+    "prefix_sweep_cascade": {"bytes": 353_382_144, "src": "4eb4742cfc8cb957", "files": DECODE_SRC},
     "llama70b_long": {"bytes": 1_584_901_888, "src": "84d9feaada7e0320", "files": DECODE_SRC},
     "prefill": {"bytes": 348_481_024, "src": "0a0c45baf16bf168", "files": PREFILL_SRC},
     "rope_write": {"bytes": 55_164_160, "src": "9b1a5d7fb8331db7", "files": ROPE_SRC},
@@ -560,7 +564,9 @@ def run_ours(args):
     peak, peak_kind = measured_hbm_peak()
     alg = kvb + io_bytes(wl)
     achieved = alg / (dec_avg * 1e-3) / 1e9
-    tr = NCU_TRAFFIC.get(args.workload + ("_int8" if int8 else ""))
+    tr = NCU_TRAFFIC.get(args.workload + ("_int8" if int8 else "") + ("_cascade" if args.cascade else ""))
+    if tr and args.cascade and c["block_size"] != 16:
+        tr = None  # captured at block size 16
     traffic = tr["bytes"] if tr and tr.get("src") == kernel_source_hash(tr["files"]) else None
     launches_per_step = 3 if args.cascade else 2  # write_kv, decode (split-K merge inside)[, shared-prefix pass]
     if rank == 0:
