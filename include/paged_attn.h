@@ -88,6 +88,11 @@ const char* pa_version(void);
 /* slot_mapping: int64 [num_tokens] device.  Duplicate slots are undefined.  */
 /* k_cache, v_cache: [num_blocks][block_size][num_kv_heads][head_dim] device.*/
 /* k and v must not overlap the caches.  num_tokens == 0 is a no-op.         */
+/* Launch: one kernel, with programmatic dependent launch.  It may start     */
+/* while the preceding kernel on the stream finishes and waits for that     */
+/* kernel to complete before it reads anything; a pa_decode after it may    */
+/* start its set-up (reading context_lens and block_tables) before the      */
+/* write completes, and waits for it before reading q or the cache.         */
 /* ------------------------------------------------------------------------ */
 int pa_write_kv(const void* k, const void* v, const int64_t* slot_mapping, int num_tokens,
                 void* k_cache, void* v_cache, int num_blocks, int block_size, int num_kv_heads,
@@ -128,9 +133,10 @@ int pa_copy_blocks(const int32_t* pairs, int num_pairs, void* k_cache, void* v_c
 /* (PA_ERR_UNSUPPORTED otherwise).  A position outside [0, max_position)    */
 /* leaves every row of that token unwritten and a slot >= num_blocks *       */
 /* block_size leaves its cache rows unwritten; both set PA_ERRBIT_INDEX in   */
-/* the device error word (pa_device_error).  One kernel launch; a          */
-/* pa_decode that follows on the stream may start its set-up early and      */
-/* waits for this kernel before it reads q_out or the cache.                 */
+/* the device error word (pa_device_error).  One kernel launch, with       */
+/* programmatic dependent launch (it waits for the preceding kernel before  */
+/* it reads anything); a pa_decode that follows on the stream may start its */
+/* set-up early and waits for this kernel before it reads q_out or the cache.*/
 /* ------------------------------------------------------------------------ */
 int pa_rope_write_kv(const void* q, void* q_out, const void* k, const void* v, const int64_t* positions,
                      const float* cos_table, const float* sin_table, int max_position,
@@ -150,7 +156,13 @@ int pa_rope_write_kv(const void* q, void* q_out, const void* k, const void* v, c
 /* that one CTA handles yields fp32 (max, sum, weighted V) in the workspace  */
 /* unless it is the whole context; the CTA that finishes a context's last    */
 /* part merges the parts by the log-sum-exp rule (atomic count, no waiting). */
-/* One kernel is launched per call.                                          */
+/* One kernel is launched per call, with programmatic dependent launch: its */
+/* set-up (reading context_lens and block_tables) may overlap the preceding */
+/* kernel, and it waits for that kernel before reading q or the cache or    */
+/* writing anything.  Once all of its loads are issued it lets the next     */
+/* programmatically launched kernel on the stream (the next step's          */
+/* pa_write_kv, or another decode) begin; that kernel waits for this one's  */
+/* completion before touching memory.                                       */
 /*                                                                           */
 /* pa_decode_plan: the grid and workspace the call will use on the current   */
 /* device.  num_partitions_or_0 > 0 fixes the number of CTAs (the number of  */
@@ -188,8 +200,9 @@ int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int
 /*   1. pa_decode's kernel over every sequence's private suffix, tokens     */
 /*      seq_prefix_len[b] .. context_lens[b]-1, leaving (out, log-sum-exp);  */
 /*   2. one pass over each group's shared prefix with the query rows of all */
-/*      its members at once (warp MMA), merged with step 1 by the            */
-/*      log-sum-exp rule into out.                                          */
+/*      its members at once (head_dim 128: the CTA-pair tensor-core kernel   */
+/*      of pa_prefill_chunk; head_dim 64: warp MMA), merged with step 1 by   */
+/*      the log-sum-exp rule into out.                                      */
 /* Groups: num_groups consecutive ranges of the batch, group g = sequences  */
 /* group_start[g] .. group_start[g+1]-1 (int32 [num_groups+1], device,      */
 /* non-decreasing); sequences outside every range, and groups whose prefix  */

@@ -284,8 +284,8 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len: int
     _device(stream, q, k_cache, v_cache, block_tables, context_lens, out, workspace)
     if out is None:
         out = torch.empty_like(q)
-    _, _, need = decode_plan(B, Hq, Hkv, D, max_context_len, num_partitions)
-    if workspace is None:  # zero-filled once; every call leaves it zeroed again
+    if workspace is None:  # zero-filled once; every call leaves it zeroed again (a given one is checked by the library)
+        _, _, need = decode_plan(B, Hq, Hkv, D, max_context_len, num_partitions)
         workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.pa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), int(block_tables.shape[1]),
@@ -354,8 +354,8 @@ def decode_lse(q, k_cache, v_cache, block_tables, context_lens, max_context_len:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
-    _, _, need = decode_plan(B, Hq, Hkv, D, max_context_len, num_partitions)
     if workspace is None:
+        _, _, need = decode_plan(B, Hq, Hkv, D, max_context_len, num_partitions)
         workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib.pa_decode_lse(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), int(block_tables.shape[1]),
@@ -390,9 +390,9 @@ def decode_cascade(q, k_cache, v_cache, block_tables, context_lens, max_context_
     _device(stream, q, k_cache, v_cache, block_tables, context_lens, group_start, seq_prefix_len, out, workspace)
     if out is None:
         out = torch.empty_like(q)
-    need = decode_cascade_workspace_size(B, Hq, Hkv, D, max_context_len, ngroups, max_group_size, max_prefix_len,
-                                         num_partitions)
     if workspace is None:  # zero-filled once; every call leaves its counters zeroed again
+        need = decode_cascade_workspace_size(B, Hq, Hkv, D, max_context_len, ngroups, max_group_size,
+                                             max_prefix_len, num_partitions)
         workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib.pa_decode_cascade(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
@@ -489,8 +489,8 @@ def decode_int8(q, k_codes, v_codes, k_scales, v_scales, block_tables, context_l
     _device(stream, q, k_codes, v_codes, k_scales, v_scales, block_tables, context_lens, out, workspace)
     if out is None:
         out = torch.empty_like(q)
-    _, _, need = decode_int8_plan(B, Hq, Hkv, D, max_context_len, num_partitions)
-    if workspace is None:  # zero-filled once; every call leaves it zeroed again
+    if workspace is None:  # zero-filled once; every call leaves it zeroed again (a given one is checked by the library)
+        _, _, need = decode_int8_plan(B, Hq, Hkv, D, max_context_len, num_partitions)
         workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib.pa_decode_int8(_ptr(q), _ptr(k_codes), _ptr(v_codes), _ptr(k_scales), _ptr(v_scales),

@@ -984,7 +984,7 @@ __global__ void __launch_bounds__((NW + 2) * 32, Q8 ? 3 : 1) decode_kernel(const
     // ================================================= producer warp
     const int B = p.batch, Hkv = p.num_kv_heads;
     const int cap = p.max_blocks_per_seq * p.block_size;
-    // pass 1: total chunks over all sequences (CTA 0 also writes out = 0 for empty sequences)
+    // pass 1: total chunks over all sequences
     long long tot = 0;
     bool clamped = false;
     for (int base = 0; base < B; base += 256) {
@@ -1001,12 +1001,6 @@ __global__ void __launch_bounds__((NW + 2) * 32, Q8 ? 3 : 1) decode_kernel(const
           }
           const int Le = eff_len(p.context_lens, p.ctx_start, i, cap);
           s += (Le + kChunk - 1) / kChunk;
-          if (cta == 0 && Le == 0) {
-            uint4* o4 = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.out) + (size_t)i * p.num_q_heads * D);
-            for (int e = 0; e < p.num_q_heads * D * 2 / 16; ++e) o4[e] = make_uint4(0, 0, 0, 0);
-            if (p.lse)
-              for (int h = 0; h < p.num_q_heads; ++h) p.lse[(size_t)i * p.num_q_heads + h] = -INFINITY;
-          }
         }
       }
       tot += warp_sum_ll(s);
@@ -1069,8 +1063,23 @@ __global__ void __launch_bounds__((NW + 2) * 32, Q8 ? 3 : 1) decode_kernel(const
     for (int j = 0; j < kLookahead; ++j) plan_push(j);
     // The cache rows read from here on may have just been written by pa_write_kv, which lets this
     // kernel launch while it runs (programmatic dependent launch; q, the block tables and the lengths
-    // are not its outputs): wait for it to complete before the first load.
+    // are not its outputs): wait for it to complete before the first load, and before any write (an
+    // earlier kernel on the stream may still be writing the same output).
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // 16-bit caches: let the next programmatically launched kernel on the stream (the next step's cache
+    // write, or the next decode) begin now.  It waits for this grid's completion before it touches memory
+    // this grid reads or writes, and meanwhile sits beside this grid's CTAs (they leave room for it), so
+    // its launch and set-up overlap this grid's tail.
+    if constexpr (!Q8) asm volatile("griddepcontrol.launch_dependents;");
+    if (cta == 0) {  // out = 0 (and log-sum-exp -inf) for sequences with no token to attend to
+      for (int i = lane; i < B; i += 32) {
+        if (eff_len(p.context_lens, p.ctx_start, i, cap) != 0) continue;
+        uint4* o4 = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.out) + (size_t)i * p.num_q_heads * D);
+        for (int e = 0; e < p.num_q_heads * D * 2 / 16; ++e) o4[e] = make_uint4(0, 0, 0, 0);
+        if (p.lse)
+          for (int h = 0; h < p.num_q_heads; ++h) p.lse[(size_t)i * p.num_q_heads + h] = -INFINITY;
+      }
+    }
     bool ok = true;
     int k = 0;
     for (;; ++k) {
@@ -1123,6 +1132,9 @@ __global__ void __launch_bounds__((NW + 2) * 32, Q8 ? 3 : 1) decode_kernel(const
       plan_push(k + kLookahead);
     }
     cp_async_wait<0>();
+    // int8 caches: the same signal once every load of this CTA is issued (three int8 CTAs per SM leave no
+    // registers for a waiting write kernel, and the early signal measured slower there)
+    if constexpr (Q8) asm volatile("griddepcontrol.launch_dependents;");
     if (!ok && lane == 0) PA_RECORD_ERROR(PA_ERRBIT_TIMEOUT);
     // drain: every copy this CTA issued has landed before the warp leaves
     if (lane == 0) {
@@ -2013,7 +2025,12 @@ extern "C" int pa_decode_cascade(const void* q, const void* k_cache, const void*
   cudaStream_t st = (cudaStream_t)stream;
   if ((s = decode_launch(call, st)) != PA_OK) return s;
   if (num_groups == 0 || max_prefix_len < kChunk) return PA_OK;
-  // pass 2: the shared prefix of every group, once for all of its members, merged with pass 1
+  // pass 2: the shared prefix of every group, once for all of its members, merged with pass 1; on the
+  // CTA-pair tensor-core kernel at head_dim 128, on warp MMA otherwise
+  if (head_dim == 128)
+    return pa::prefix_pass_pairs(q, k_cache, v_cache, block_tables, max_blocks_per_seq, num_groups, group_start,
+                                 seq_prefix_len, max_group_size, reinterpret_cast<const float*>(ws + cp.off_lse),
+                                 num_q_heads, num_kv_heads, block_size, num_blocks, scale, dtype, out, st);
   CascadeParams c;
   c.q = q;
   c.out = out;

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "paged_attn.h"
 
 namespace pa {
@@ -30,5 +32,31 @@ int encode_2d_u16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t ro
 
 // Number of SMs of the current device (cached per device).
 int sm_count();
+
+// The cascade decode's shared-prefix pass on the CTA-pair tensor-core kernel (head_dim 128; prefill.cu).
+int prefix_pass_pairs(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                      int max_blocks_per_seq, int num_groups, const int32_t* group_start, const int32_t* seq_prefix,
+                      int max_group_size, const float* lse_s, int num_q_heads, int num_kv_heads, int block_size,
+                      int num_blocks, float scale, int dtype, void* out, cudaStream_t st);
+
+// Launch with programmatic stream serialization: the kernel may start while the preceding kernel on the
+// stream is still running (once that kernel signals griddepcontrol.launch_dependents or exits), so it
+// must execute griddepcontrol.wait before it reads or writes memory the preceding kernel may touch.
+template <typename... Params, typename... Args>
+int launch_programmatic(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                        Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) return PA_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
 
 }  // namespace pa

@@ -75,6 +75,8 @@ __global__ void __launch_bounds__(256) write_kv_int8_kernel(const void* __restri
                                                             float* __restrict__ ks, float* __restrict__ vs) {
   // a decode launched after this may start its set-up now; it waits for this grid before reading the cache
   asm volatile("griddepcontrol.launch_dependents;");
+  // launched programmatically itself: wait for the preceding grid before reading inputs or writing slots
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int64_t items = (int64_t)num_tokens * hkv;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -152,22 +154,10 @@ extern "C" int pa_write_kv_int8(const void* k, const void* v, const int64_t* slo
   auto* vq = reinterpret_cast<int8_t*>(v_codes);
   cudaStream_t st = (cudaStream_t)stream;
   const unsigned g = (unsigned)blocks;
-  if (dtype == PA_BF16) {
-    if (head_dim == 128)
-      write_kv_int8_kernel<PA_BF16, 128><<<g, 256, 0, st>>>(k, v, slot_mapping, num_tokens, num_kv_heads, block_size,
-                                                            slots, kq, vq, k_scales, v_scales);
-    else
-      write_kv_int8_kernel<PA_BF16, 64><<<g, 256, 0, st>>>(k, v, slot_mapping, num_tokens, num_kv_heads, block_size,
-                                                           slots, kq, vq, k_scales, v_scales);
-  } else {
-    if (head_dim == 128)
-      write_kv_int8_kernel<PA_F16, 128><<<g, 256, 0, st>>>(k, v, slot_mapping, num_tokens, num_kv_heads, block_size,
-                                                           slots, kq, vq, k_scales, v_scales);
-    else
-      write_kv_int8_kernel<PA_F16, 64><<<g, 256, 0, st>>>(k, v, slot_mapping, num_tokens, num_kv_heads, block_size,
-                                                          slots, kq, vq, k_scales, v_scales);
-  }
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  auto kern = dtype == PA_BF16 ? (head_dim == 128 ? write_kv_int8_kernel<PA_BF16, 128> : write_kv_int8_kernel<PA_BF16, 64>)
+                               : (head_dim == 128 ? write_kv_int8_kernel<PA_F16, 128> : write_kv_int8_kernel<PA_F16, 64>);
+  return launch_programmatic(kern, dim3(g), dim3(256), 0, st, k, v, slot_mapping, num_tokens, num_kv_heads, block_size,
+                             slots, kq, vq, k_scales, v_scales);
 }
 
 extern "C" int pa_copy_blocks_int8(const int32_t* pairs, int num_pairs, void* k_codes, void* v_codes, float* k_scales,

@@ -42,6 +42,14 @@
 // for a half when any warp of the pair asked.  Without it the high term alone
 // moves an output by at most 2^-9 |v| / 16.  3 of every 8 exponentials run
 // as a polynomial on the FMA pipe to relieve the MUFU unit.
+//
+// The same kernel serves the cascade decode's shared-prefix pass (pages "Nano-vLLM-Ascend..." section
+// 2.1, reference-counted shared blocks, and "Ascend NPU LLM inference optimisation..." section 4, block
+// sharing): a "sequence" is then a group of decode sequences forked from one parent, its query rows are
+// the members' single decode queries (consecutive rows of the decode q), every row attends to the whole
+// shared prefix through the first member's block table (no causal limit; keys past the prefix are masked
+// in the last tile), and the epilogue merges the prefix's softmax with the member's suffix result already
+// in `out` by their log-sum-exps.
 
 #include <algorithm>
 #include <atomic>
@@ -108,6 +116,15 @@ struct PrefillParams {
   int mtiles;         // ceil(max_chunk_len / BM)
   int units;          // CTA pairs per (sequence, KV head)
   float scale_log2;
+  // Shared-prefix mode (the cascade decode's prefix pass): "sequence" b is a group of decode sequences
+  // group_start[b] .. group_start[b+1]-1 sharing their first seq_prefix[group_start[b]] tokens; query row i
+  // is member group_start[b] + i (its one decode query), every row attends to the whole prefix (no causal
+  // limit) through the first member's block table, and the epilogue merges the prefix's softmax with the
+  // member's suffix result (out, lse_s) already in `out`.
+  int prefix_mode;
+  const int32_t* group_start;
+  const int32_t* seq_prefix;
+  const float* lse_s;
 };
 
 // --------------------------------------------------------------- cluster / tcgen05 helpers
@@ -321,18 +338,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mrow_hi = mrow_lo + BM;
   }
 
-  const int q0 = __ldg(p.query_start_loc + b), q1 = __ldg(p.query_start_loc + b + 1);
+  const int32_t* rowstart = p.prefix_mode ? p.group_start : p.query_start_loc;
+  const int q0 = __ldg(rowstart + b), q1 = __ldg(rowstart + b + 1);
   const int C = q1 - q0;
   // both CTAs of a pair take the same early exits (they depend on the pair only)
   if (mrow_lo >= C) return;
-  const int L = __ldg(p.context_lens + b);
   const int cap = p.max_blocks_per_seq * p.block_size;
-  if (L > cap || L < C) {  // broken caller invariant: record and produce nothing for this pair
-    if (threadIdx.x == 0) PA_RECORD_ERROR(PA_ERRBIT_INDEX);
-    return;
+  int L, kend;
+  if (p.prefix_mode) {  // keys [0, P) for every row: the group's shared prefix (a multiple of 16)
+    const int P0 = __ldg(p.seq_prefix + q0);
+    const int P = min(max(P0, 0), cap) & ~15;
+    if (P != P0 && threadIdx.x == 0) PA_RECORD_ERROR(PA_ERRBIT_INDEX);
+    if (P == 0) return;  // no shared prefix: the suffix result already is the answer
+    L = P;
+    kend = P;
+  } else {
+    L = __ldg(p.context_lens + b);
+    if (L > cap || L < C) {  // broken caller invariant: record and produce nothing for this pair
+      if (threadIdx.x == 0) PA_RECORD_ERROR(PA_ERRBIT_INDEX);
+      return;
+    }
+    // keys [0, kend) are visible to some row of the pair
+    kend = L - C + min(mrow_hi + BM, C);
   }
-  // keys [0, kend) are visible to some row of the pair
-  const int kend = L - C + min(mrow_hi + BM, C);
   const int nkv = (kend + BN - 1) / BN;
 
   if (threadIdx.x == 0) {
@@ -375,7 +403,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
     }
-    const int32_t* bt = p.block_tables + (size_t)b * p.max_blocks_per_seq;
+    const int32_t* bt = p.block_tables + (size_t)(p.prefix_mode ? q0 : b) * p.max_blocks_per_seq;
     const uint32_t kfull0 = map_rank(smem_u32(k_full), 0), vfull0 = map_rank(smem_u32(v_full), 0);
     // first key of box i of key tile j: K boxes cover this CTA's 64 keys, V boxes all 128
     auto kbox_key = [&](int j, int i) { return j * BN + (int)rank * (BN / 2) + i * 16; };
@@ -547,7 +575,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int r = threadIdx.x & 127;
     const int row = mrow + r;
     const int pos = L - C + row;                              // this row's position (keys 0..pos visible)
-    const int last_key = min(pos, L - 1);
+    const int last_key = p.prefix_mode ? L - 1 : min(pos, L - 1);
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;  // this warp's TMEM lane quarter
     const int pair_bar = 3 + (warp & 3);                      // the two warps that own rows 32*(warp&3)..
     const uint32_t qfull0 = map_rank(smem_u32(q_full), 0), pfull0 = map_rank(smem_u32(p_full), 0);
@@ -718,7 +746,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (ok && mbar_wait_warp(&o_done[(nkv - 1) & 1], ((nkv - 1) >> 1) & 1)) {
       tc_fence_after();
       T* orow = reinterpret_cast<T*>(p.out) + ((size_t)(q0 + row) * p.num_q_heads + head) * HD + hf * 64;
-      const float inv = 1.f / lsum;
+      // out = wp * O + ws * (what out holds): wp = 1/l and ws = 0 for prefill; in shared-prefix mode the
+      // prefix's softmax and the member's suffix result are weighted by their log-sum-exps, the prefix's
+      // being m_ref + log2(l) in the log2 domain and the suffix's lse_s (natural log; -inf when empty)
+      float wp = 1.f / lsum, ws = 0.f;
+      if (p.prefix_mode && row < C) {
+        const float mp = m_ref + __log2f(lsum);
+        const float ms = __ldg(p.lse_s + (size_t)(q0 + row) * p.num_q_heads + head) * kLog2e;
+        const float M = fmaxf(mp, ms);
+        const float ep = exp2f(mp - M), es = exp2f(ms - M);
+        wp = ep / ((ep + es) * lsum);
+        ws = es / (ep + es);
+      }
 #pragma unroll
       for (int c = 0; c < 64; c += 32) {
         uint32_t o[32];
@@ -727,11 +766,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (row < C) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(o[e + i]) * wp;
+            if (p.prefix_mode) {
+              const uint4 u = *reinterpret_cast<const uint4*>(orow + c + e);
+              const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float2 sv = Elt<DT>::to_f2(w4[i]);
+                f[2 * i] = fmaf(ws, sv.x, f[2 * i]);
+                f[2 * i + 1] = fmaf(ws, sv.y, f[2 * i + 1]);
+              }
+            }
             uint4 v;
-            v.x = Elt<DT>::from_f2(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
-            v.y = Elt<DT>::from_f2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
-            v.z = Elt<DT>::from_f2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
-            v.w = Elt<DT>::from_f2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
+            v.x = Elt<DT>::from_f2(f[0], f[1]);
+            v.y = Elt<DT>::from_f2(f[2], f[3]);
+            v.z = Elt<DT>::from_f2(f[4], f[5]);
+            v.w = Elt<DT>::from_f2(f[6], f[7]);
             *reinterpret_cast<uint4*>(orow + c + e) = v;
           }
         }
@@ -747,6 +799,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   if (warp == 9)
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+}
+
+}  // namespace
+
+namespace {
+
+// One launch of the pair kernel: tensor maps over the caches, the dynamic shared-memory attribute set once
+// per dtype and device, grid 2 * batch * Hkv * units CTAs.
+int launch_pairs(PrefillParams& p, const void* k_cache, const void* v_cache, int dtype, long grid, cudaStream_t st) {
+  CUtensorMap km, vm;
+  const uint64_t rows = (uint64_t)p.num_blocks * p.block_size;
+  const uint64_t cols = (uint64_t)p.num_kv_heads * HD;
+  if (pa::encode_2d_sw128(&km, k_cache, cols, rows, cols * 2, 64, 16) != PA_OK) return PA_ERR_CUDA;
+  if (pa::encode_2d_sw128(&vm, v_cache, cols, rows, cols * 2, 64, 16) != PA_OK) return PA_ERR_CUDA;
+  auto kern = dtype == PA_BF16 ? prefill_kernel<PA_BF16> : prefill_kernel<PA_F16>;
+  // per dtype and device; host threads may race to set it, which only repeats an idempotent call
+  static std::atomic<bool> attr_set[2][64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  const int di = dtype == PA_BF16 ? 1 : 0;
+  if (dev < 0 || dev >= 64 || !attr_set[di][dev].load(std::memory_order_acquire)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC) != cudaSuccess)
+      return PA_ERR_CUDA;
+    if (dev >= 0 && dev < 64) attr_set[di][dev].store(true, std::memory_order_release);
+  }
+  kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(km, vm, p);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 }  // namespace
@@ -776,7 +855,7 @@ extern "C" int pa_prefill_chunk(const void* q, const int32_t* query_start_loc, i
   const long grid = 2L * batch * num_kv_heads * units;
   if (grid > 0x7fffffffL) return PA_ERR_UNSUPPORTED;
 
-  PrefillParams p;
+  PrefillParams p = {};
   p.q = q;
   p.out = out;
   p.query_start_loc = query_start_loc;
@@ -791,24 +870,45 @@ extern "C" int pa_prefill_chunk(const void* q, const int32_t* query_start_loc, i
   p.mtiles = mtiles;
   p.units = units;
   p.scale_log2 = scale * kLog2e;
-
-  CUtensorMap km, vm;
-  const uint64_t rows = (uint64_t)num_blocks * block_size;
-  const uint64_t cols = (uint64_t)num_kv_heads * HD;
-  if (pa::encode_2d_sw128(&km, k_cache, cols, rows, cols * 2, 64, 16) != PA_OK) return PA_ERR_CUDA;
-  if (pa::encode_2d_sw128(&vm, v_cache, cols, rows, cols * 2, 64, 16) != PA_OK) return PA_ERR_CUDA;
-
-  auto kern = dtype == PA_BF16 ? prefill_kernel<PA_BF16> : prefill_kernel<PA_F16>;
-  // per dtype and device; host threads may race to set it, which only repeats an idempotent call
-  static std::atomic<bool> attr_set[2][64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
-  const int di = dtype == PA_BF16 ? 1 : 0;
-  if (dev < 0 || dev >= 64 || !attr_set[di][dev].load(std::memory_order_acquire)) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC) != cudaSuccess)
-      return PA_ERR_CUDA;
-    if (dev >= 0 && dev < 64) attr_set[di][dev].store(true, std::memory_order_release);
-  }
-  kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, (cudaStream_t)stream>>>(km, vm, p);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  p.prefix_mode = 0;
+  return launch_pairs(p, k_cache, v_cache, dtype, grid, (cudaStream_t)stream);
 }
+
+namespace pa {
+
+// The cascade decode's shared-prefix pass on the tensor cores (head_dim 128): for every group g of
+// decode sequences group_start[g] .. group_start[g+1]-1, its members' queries attend to the group's
+// shared prefix (seq_prefix of its first member, read through that member's block table), and the
+// result is merged in place with each member's suffix result (out, lse_s).  Arguments are checked by the
+// caller.
+int prefix_pass_pairs(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                      int max_blocks_per_seq, int num_groups, const int32_t* group_start, const int32_t* seq_prefix,
+                      int max_group_size, const float* lse_s, int num_q_heads, int num_kv_heads, int block_size,
+                      int num_blocks, float scale, int dtype, void* out, cudaStream_t st) {
+  const int G = num_q_heads / num_kv_heads;
+  const int mtiles = (max_group_size + BM - 1) / BM;
+  const int units = G >= 2 ? (G / 2) * mtiles : (mtiles + 1) / 2;
+  const long grid = 2L * num_groups * num_kv_heads * units;
+  if (grid == 0) return PA_OK;
+  if (grid > 0x7fffffffL) return PA_ERR_UNSUPPORTED;
+  PrefillParams p = {};
+  p.q = q;
+  p.out = out;
+  p.block_tables = block_tables;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.batch = num_groups;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.block_size = block_size;
+  p.num_blocks = num_blocks;
+  p.mtiles = mtiles;
+  p.units = units;
+  p.scale_log2 = scale * kLog2e;
+  p.prefix_mode = 1;
+  p.group_start = group_start;
+  p.seq_prefix = seq_prefix;
+  p.lse_s = lse_s;
+  return launch_pairs(p, k_cache, v_cache, dtype, grid, st);
+}
+
+}  // namespace pa

@@ -72,6 +72,8 @@ __global__ void __launch_bounds__(256) rope_write_kv_kernel(const RopeArgs a) {
   // a decode kernel launched after this one may start its set-up now; it waits for this grid to
   // complete before it reads q_out or the cache (programmatic dependent launch)
   asm volatile("griddepcontrol.launch_dependents;");
+  // launched programmatically itself: wait for the preceding grid before reading inputs or writing
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int rot = a.rot, vec = 2 * rot;  // 16-byte vectors per half head / per head
   const int rq = a.hq * rot, rk = a.hkv * rot;
   const int ipt = rq + rk + a.hkv * vec;
@@ -174,6 +176,5 @@ extern "C" int pa_rope_write_kv(const void* q, void* q_out, const void* k, const
   int64_t blocks = (total + threads - 1) / threads;
   const int64_t cap = (int64_t)pa::sm_count() * per_sm;
   if (blocks > cap) blocks = cap;
-  kern<<<(unsigned)blocks, threads, 0, (cudaStream_t)stream>>>(a);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return pa::launch_programmatic(kern, dim3((unsigned)blocks), dim3(threads), 0, (cudaStream_t)stream, a);
 }

@@ -29,6 +29,9 @@ __global__ void __launch_bounds__(256) write_kv_kernel(const uint4* __restrict__
   // a decode launched after this may start its set-up now; it waits for this grid to complete
   // before it reads the cache (programmatic dependent launch)
   asm volatile("griddepcontrol.launch_dependents;");
+  // this grid may itself have started early (launched programmatically behind a decode that is still
+  // reading the cache): wait for the preceding grid before reading inputs or writing slots
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total_vecs;
        i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t t = i / vecs_per_row;
@@ -91,10 +94,9 @@ extern "C" int pa_write_kv(const void* k, const void* v, const int64_t* slot_map
   int64_t blocks = (total + threads - 1) / threads;
   const int64_t cap = (int64_t)pa::sm_count() * 8;
   if (blocks > cap) blocks = cap;
-  write_kv_kernel<<<(unsigned)blocks, threads, 0, (cudaStream_t)stream>>>(
-      (const uint4*)k, (const uint4*)v, slot_mapping, total, vecs_per_row, (int64_t)num_blocks * block_size,
-      (uint4*)k_cache, (uint4*)v_cache);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return pa::launch_programmatic(write_kv_kernel, dim3((unsigned)blocks), dim3(threads), 0, (cudaStream_t)stream,
+                                 (const uint4*)k, (const uint4*)v, slot_mapping, total, vecs_per_row,
+                                 (int64_t)num_blocks * block_size, (uint4*)k_cache, (uint4*)v_cache);
 }
 
 extern "C" int pa_copy_blocks(const int32_t* pairs, int num_pairs, void* k_cache, void* v_cache, int num_blocks,
