@@ -57,7 +57,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kChunk = 16;  // tokens per chunk = rows per TMA box
 constexpr int kPlanRing = 8;  // producer plan ring slots
 constexpr int kMaxPieces = 32;  // pieces per segment the epilogue merges with precomputed weights
-constexpr int kLookahead = 6; // stages planned (block-table entries in flight) ahead of the one issued
+constexpr int kLookahead = 3; // stages planned (block-table entries in flight) ahead of the one issued
 static_assert(kPlanRing > kLookahead, "plan ring must hold the stages in flight plus the one issued");
 
 struct DecodeParams {
@@ -795,6 +795,7 @@ struct Walker {
   int win_base, win_len;      // lens window: lane i holds the clamped length of sequence win_base + i
   int batch, hkv, cap, grid;
   long long total;            // chunks on the whole line
+  bool narrow;                // total * grid < 2^32: every division of the walk fits in 32 bits
   int vid;                    // this CTA (see StageMeta)
   const int32_t* lens;
   const int32_t* starts;      // per-sequence first token (null: 0); the walk sees L - start tokens
@@ -802,11 +803,34 @@ struct Walker {
   int nq;
   long long q0_start, q0_end, q0_pre, q1_start, q1_end, q1_pre;
   int q0_b, q1_b;
+  // batches of at most kRegBatch sequences: lane l holds the walk lengths of sequences 8l .. 8l+7 and the
+  // chunks of all sequences before them, so lookups are shuffles instead of loads
+  bool regs;
+  int le[8];
+  long long lane_pre;
 };
 
+constexpr int kRegBatch = 256;
+
+// Counter add at device scope with release (writes ordered before it, including other lanes' through a
+// preceding warp barrier, are visible before the count) and acquire (writes of the CTAs counted before
+// are visible after it): one L2 round trip where a fence and then an atomic take two.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* ptr, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(ptr), "r"(v) : "memory");
+  return old;
+}
+
+// Floor division of a >= 0 by b > 0; `narrow` (uniform over the warp) says a and b fit in 32 bits, and then
+// the division is the 32-bit one: 64-bit integer division is a long software sequence, and the producer's
+// set-up runs several before its first load.
+__device__ __forceinline__ long long udiv(long long a, long long b, bool narrow) {
+  return narrow ? (long long)((uint32_t)a / (uint32_t)b) : a / b;
+}
+
 // CTA that owns chunk x of the line: the largest c with total*c/grid <= x.
-__device__ __forceinline__ long long owner_of(long long x, long long total, long long grid) {
-  return ((x + 1) * grid - 1) / total;
+__device__ __forceinline__ long long owner_of(long long x, long long total, long long grid, bool narrow) {
+  return udiv((x + 1) * grid - 1, total, narrow);
 }
 
 __device__ __forceinline__ int clamp_len(int L, int cap) { return L < 0 ? 0 : (L > cap ? cap : L); }
@@ -822,10 +846,25 @@ __device__ __forceinline__ int eff_len(const int32_t* lens, const int32_t* start
   return L > s0 ? L - s0 : 0;
 }
 
+// Walk length of sequence s (each lane its own s) from the lanes' registers: lane s/8, entry s%8.
+__device__ __forceinline__ int reg_len(const Walker& w, int s) {
+  const int src = (s >> 3) & 31, e = s & 7;
+  int r = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int t = __shfl_sync(0xffffffffu, w.le[j], src);
+    if (e == j) r = t;
+  }
+  return s >= 0 && s < w.batch ? r : 0;
+}
+
 __device__ __forceinline__ void load_window(Walker& w, int base, int lane) {
   w.win_base = base;
   const int i = base + lane;
-  w.win_len = i < w.batch ? eff_len(w.lens, w.starts, i, w.cap) : 0;
+  if (w.regs)
+    w.win_len = reg_len(w, i);
+  else
+    w.win_len = i < w.batch ? eff_len(w.lens, w.starts, i, w.cap) : 0;
 }
 
 // Sequence b holding chunk x of the line (x < total) and pre = chunks of all sequences before it.
@@ -834,6 +873,27 @@ __device__ __forceinline__ void find_seq(const Walker& w, long long x, int lane,
   long long run = 0;
   fb = -1;
   fpre = 0;
+  if (w.regs) {  // the same search over the register-held lengths: no loads, one ballot
+    long long pre = w.lane_pre;
+    int found = -1;
+    long long found_pre = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int v = (w.le[j] + kChunk - 1) / kChunk;
+      if (v > 0 && pre * w.hkv <= x && x < (pre + v) * w.hkv) {
+        found = lane * 8 + j;
+        found_pre = pre;
+      }
+      pre += v;
+    }
+    const unsigned hit = __ballot_sync(0xffffffffu, found >= 0);
+    if (hit) {
+      const int src = __ffs(hit) - 1;
+      fb = __shfl_sync(0xffffffffu, found, src);
+      fpre = __shfl_sync(0xffffffffu, found_pre, src);
+    }
+    return;
+  }
   for (int base = 0; base < w.batch; base += 256) {
     int v[8];
     long long s = 0;
@@ -872,7 +932,7 @@ __device__ __forceinline__ void walker_seek(Walker& w, long long x, long long en
   w.b = b;
   w.L = __shfl_sync(0xffffffffu, w.win_len, b - w.win_base);
   w.nch = (w.L + kChunk - 1) / kChunk;
-  w.g = (int)((x - pre * w.hkv) / w.nch);
+  w.g = (int)udiv(x - pre * w.hkv, w.nch, w.narrow);
   w.seg_start = pre * w.hkv + (long long)w.g * w.nch;
   w.pos = x;
   w.piece_start = x;
@@ -928,11 +988,13 @@ __device__ __forceinline__ StageMeta walker_next(Walker& w, int cta, int lane) {
   d.c0 = w.vid;
   d.npieces = 1;
   if ((d.flags & F_LAST) && !(d.flags & F_DIRECT)) {
-    const long long c0 = owner_of(w.seg_start, w.total, w.grid), c1 = owner_of(seg_end - 1, w.total, w.grid);
+    const long long c0 = owner_of(w.seg_start, w.total, w.grid, w.narrow);
+    const long long c1 = owner_of(seg_end - 1, w.total, w.grid, w.narrow);
     int n = (int)(c1 - c0 + 1);
     if (w.total < w.grid) {  // some CTAs have an empty range and hold no piece
       n = 0;
-      for (long long c = c0; c <= c1; ++c) n += (w.total * c / w.grid != w.total * (c + 1) / w.grid);
+      for (long long c = c0; c <= c1; ++c)
+        n += (udiv(w.total * c, w.grid, w.narrow) != udiv(w.total * (c + 1), w.grid, w.narrow));
     }
     d.c0 = (int)c0;
     d.npieces = n;
@@ -984,7 +1046,13 @@ __global__ void __launch_bounds__((NW + 2) * 32, Q8 ? 3 : 1) decode_kernel(const
     // ================================================= producer warp
     const int B = p.batch, Hkv = p.num_kv_heads;
     const int cap = p.max_blocks_per_seq * p.block_size;
-    // pass 1: total chunks over all sequences
+    // pass 1: total chunks over all sequences (lane l takes sequences base + 8l .. base + 8l + 7); the
+    // first 256 sequences' walk lengths and chunk prefixes stay in registers for the lookups below
+    Walker w;
+    w.regs = B <= kRegBatch;
+    w.lane_pre = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) w.le[j] = 0;
     long long tot = 0;
     bool clamped = false;
     for (int base = 0; base < B; base += 256) {
@@ -992,33 +1060,41 @@ __global__ void __launch_bounds__((NW + 2) * 32, Q8 ? 3 : 1) decode_kernel(const
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int i = base + lane * 8 + j;
+        int Le = 0;
         if (i < B) {
           const int L = __ldg(p.context_lens + i);
           clamped |= (L < 0 || L > cap);
+          int s0 = 0;
           if (p.ctx_start) {
-            const int s0 = __ldg(p.ctx_start + i);
-            clamped |= (s0 < 0 || (s0 & (kChunk - 1)) != 0);
+            const int s0raw = __ldg(p.ctx_start + i);
+            clamped |= (s0raw < 0 || (s0raw & (kChunk - 1)) != 0);
+            s0 = max(0, s0raw) & ~(kChunk - 1);  // as start_of()
           }
-          const int Le = eff_len(p.context_lens, p.ctx_start, i, cap);
-          s += (Le + kChunk - 1) / kChunk;
+          const int Lc = clamp_len(L, cap);
+          Le = Lc > s0 ? Lc - s0 : 0;            // as eff_len()
         }
+        if (base == 0) w.le[j] = Le;
+        s += (Le + kChunk - 1) / kChunk;
       }
-      tot += warp_sum_ll(s);
+      const long long incl = warp_incl_scan_ll(s, lane);
+      if (base == 0) w.lane_pre = incl - s;
+      tot += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (clamped && cta == 0 && lane == 0) PA_RECORD_ERROR(PA_ERRBIT_INDEX);
     const long long C = tot * Hkv;
     if (lane == 0) *reinterpret_cast<long long*>(smem + LY::MISC_OFF) = C;  // published by the first full barrier
-    const long long x0 = C * cta / p.grid, x1 = C * (cta + 1) / p.grid;
+    const bool narrow = C * p.grid < (1LL << 32);
+    const long long x0 = udiv(C * cta, p.grid, narrow), x1 = udiv(C * (cta + 1), p.grid, narrow);
     // Walk order: the first piece, then the last piece, then the whole segments between.  Only
     // those two pieces can be partial, so both halves of every segment cut between two CTAs
     // finish early and its merge overlaps the rest of the stream instead of trailing it.
-    Walker w;
     w.pos = w.end = 0;
     w.batch = B;
     w.hkv = Hkv;
     w.cap = cap;
     w.grid = p.grid;
     w.total = C;
+    w.narrow = narrow;
     w.vid = cta;
     w.lens = p.context_lens;
     w.starts = p.ctx_start;
@@ -1031,8 +1107,9 @@ __global__ void __launch_bounds__((NW + 2) * 32, Q8 ? 3 : 1) decode_kernel(const
       find_seq(w, x1 - 1, lane, bl, pl);
       walker_seek(w, x0, x1, b0, p0, lane);
       const long long s0 = w.seg_start, e0 = s0 + w.nch;
-      const int Ll = eff_len(p.context_lens, p.ctx_start, bl, cap), nl = (Ll + kChunk - 1) / kChunk;
-      const long long sl = pl * Hkv + ((x1 - 1 - pl * Hkv) / nl) * nl, el = sl + nl;
+      const int Ll = w.regs ? reg_len(w, bl) : eff_len(p.context_lens, p.ctx_start, bl, cap);
+      const int nl = (Ll + kChunk - 1) / kChunk;
+      const long long sl = pl * Hkv + udiv(x1 - 1 - pl * Hkv, nl, narrow) * nl, el = sl + nl;
       const bool last_sep = sl > s0 && x1 < el;
       const long long first_end = e0 < x1 ? e0 : x1, mid_end = last_sep ? sl : x1;
       w.end = first_end;
@@ -1049,6 +1126,7 @@ __global__ void __launch_bounds__((NW + 2) * 32, Q8 ? 3 : 1) decode_kernel(const
     // ring, so no lookup latency sits between a freed stage and its refill.
     const int32_t* bt_all = p.block_tables;
     const int mb = p.max_blocks_per_seq, bs = p.block_size;
+    const int bs_shift = __ffs(bs) - 1;  // block sizes are powers of two
     StageMeta* plan = reinterpret_cast<StageMeta*>(smem + LY::PLAN_OFF);
     int32_t* plan_phys = reinterpret_cast<int32_t*>(smem + LY::PLAN_OFF + kPlanRing * sizeof(StageMeta));
     auto plan_push = [&](int j) {
@@ -1057,7 +1135,7 @@ __global__ void __launch_bounds__((NW + 2) * 32, Q8 ? 3 : 1) decode_kernel(const
       if (lane == 0) plan[slot] = dn;
       if (!(dn.flags & F_END) && lane < stage_chunks(dn))
         cp_async4(plan_phys + slot * 8 + lane,
-                  bt_all + (size_t)dn.b * mb + (start_of(p.ctx_start, dn.b) + dn.tok0 + lane * kChunk) / bs);
+                  bt_all + (size_t)dn.b * mb + ((start_of(p.ctx_start, dn.b) + dn.tok0 + lane * kChunk) >> bs_shift));
       cp_async_commit();
     };
     for (int j = 0; j < kLookahead; ++j) plan_push(j);
@@ -1107,7 +1185,7 @@ __global__ void __launch_bounds__((NW + 2) * 32, Q8 ? 3 : 1) decode_kernel(const
         const bool in_range = phys >= 0 && phys < p.num_blocks;
         if (!in_range) PA_RECORD_ERROR(PA_ERRBIT_INDEX);  // TMA zero-fills out of range
         const int tok = start_of(p.ctx_start, d.b) + d.tok0 + lane * kChunk;  // token of the sequence
-        const int y = phys * bs + (tok % bs);
+        const int y = phys * bs + (tok & (bs - 1));
         uint8_t* kd = smem + LY::K_OFF + st * LY::STAGE_BYTES + lane * kChunk * LY::BOXB;
         uint8_t* vd = smem + LY::V_OFF + st * LY::STAGE_BYTES + lane * kChunk * LY::BOXB;
         // tensor-map columns are 16-bit units: a row of one KV head starts at column g * ROWB / 2
@@ -1119,7 +1197,7 @@ __global__ void __launch_bounds__((NW + 2) * 32, Q8 ? 3 : 1) decode_kernel(const
         if constexpr (Q8) {
           // the chunk's 16 scales of KV head g: one 64-byte run of [num_blocks][Hkv][block_size] (a block id
           // out of range reads block 0 instead; the error bit is set above)
-          const size_t so = ((size_t)(in_range ? phys : 0) * p.num_kv_heads + d.g) * bs + (tok % bs);
+          const size_t so = ((size_t)(in_range ? phys : 0) * p.num_kv_heads + d.g) * bs + (tok & (bs - 1));
           bulk_load(smem + LY::SK_OFF + (st * LY::TOK + lane * kChunk) * 4, p.k_scales + so, kChunk * 4, &full[st]);
           bulk_load(smem + LY::SV_OFF + (st * LY::TOK + lane * kChunk) * 4, p.v_scales + so, kChunk * 4, &full[st]);
         }
@@ -1210,6 +1288,7 @@ __global__ void __launch_bounds__((NW + 2) * 32, Q8 ? 3 : 1) decode_kernel(const
         // CTAs holding a piece of this segment: c0, c0+1, ... (when the line has fewer chunks than
         // CTAs, some CTAs hold nothing and are skipped)
         const bool dense = C_s >= p.grid;
+        const int np = d.npieces;
         auto piece_cta = [&](int n) -> long long {
           if (dense) return d.c0 + n;
           for (long long k2 = d.c0, m2 = 0;; ++k2)
@@ -1221,7 +1300,6 @@ __global__ void __launch_bounds__((NW + 2) * 32, Q8 ? 3 : 1) decode_kernel(const
         // a few L2 round trips, not one per piece.
         float* wts = reinterpret_cast<float*>(smem + LY::WTS_OFF);
         int* vids = reinterpret_cast<int*>(smem + LY::VIDS_OFF);
-        const int np = d.npieces;
         if (np <= kMaxPieces) {
           const size_t myrow = lane < np ? ((size_t)sg + piece_cta(lane)) * G : 0;
           if (lane < np) vids[lane] = (int)(myrow / G - sg);
