@@ -379,8 +379,10 @@ def pipelined_e2e(stage: StagedInputs, out_like, step, K: int, repeats: int, war
     copy stream, the step's library calls on the compute stream, the D2H of its output on a second copy
     stream; inputs and outputs are double-buffered, so copies of neighbouring steps overlap the compute.
     Returns the median over `repeats` of the ms per step (device events, first copy to last copy back), the
-    repeats, the bytes copied in and out per step, and the median host time per step spent issuing them."""
+    repeats, the bytes copied in and out per step, and the median host time per step spent issuing them.
+    Copies go through the library's pa_copy_async on the copy streams (no torch stream switch per copy)."""
     import torch
+    import paged_kv_cache_330_b200 as pa
     main = torch.cuda.current_stream(dev)
     cin, cout = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     outs = [torch.empty_like(out_like) for _ in range(2)]
@@ -389,21 +391,20 @@ def pipelined_e2e(stage: StagedInputs, out_like, step, K: int, repeats: int, war
     freed = [torch.cuda.Event() for _ in range(2)]   # the slot's output is back on the host
     landed = [torch.cuda.Event() for _ in range(2)]  # the slot's inputs are on the device
     nb = stage.nbytes
+    h_in, d_in = stage.h[:nb], [d[:nb] for d in stage.d]
 
     def run(n):
         for k in range(n):
             i = k & 1
             cin.wait_event(done[i])                  # step k-2 no longer reads this input slot
-            with torch.cuda.stream(cin):
-                stage.d[i][:nb].copy_(stage.h[:nb], non_blocking=True)
+            pa.copy_async(d_in[i], h_in, stream=cin)
             landed[i].record(cin)
             main.wait_event(landed[i])
             main.wait_event(freed[i])                # step k-2's output has left this output slot
             step(main, stage.views[i], outs[i])
             done[i].record(main)
             cout.wait_event(done[i])
-            with torch.cuda.stream(cout):
-                h_outs[i].copy_(outs[i], non_blocking=True)
+            pa.copy_async(h_outs[i], outs[i], stream=cout)
             freed[i].record(cout)
 
     run(warmup)

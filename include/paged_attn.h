@@ -77,6 +77,17 @@ const char* pa_strerror(int status);
 /* Library version as "major.minor.patch" (static string). */
 const char* pa_version(void);
 
+/* Asynchronous copy of `bytes` bytes from src to dst on `stream`            */
+/* (cudaStream_t, NULL = legacy default stream), in whichever direction the  */
+/* two addresses give (host, pinned host or device memory of the current     */
+/* device; unified addressing decides).  Plumbing for callers that stage a   */
+/* step's inputs into device memory without switching streams on their side:*/
+/* it returns once the copy is queued; pinned host memory makes a host-side  */
+/* copy asynchronous.  The caller keeps both buffers alive and unchanged     */
+/* until the stream passes the copy.  bytes == 0 is a no-op; NULL dst or src */
+/* with bytes > 0 -> PA_ERR_INVALID; a failed enqueue -> PA_ERR_CUDA.        */
+int pa_copy_async(void* dst, const void* src, size_t bytes, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* KV write (P1 s2.1 Block layout; P2 s2.2 "fill requests into fixed-size     */
 /* blocks").                                                                  */

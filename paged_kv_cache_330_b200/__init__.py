@@ -28,7 +28,7 @@ __all__ = ["PagedAttnError", "PoolOutOfBlocks", "BlockPool", "write_kv", "copy_b
            "decode_static_scratch",
            "prefill_chunk", "device_error", "lib", "LIB_PATH", "replay_ops", "version",
            "write_kv_int8", "copy_blocks_int8", "decode_int8", "decode_int8_plan", "decode_lse", "merge_attn_states",
-           "decode_cascade", "decode_cascade_workspace_size"]
+           "decode_cascade", "decode_cascade_workspace_size", "copy_async"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpaged_attn.so")
 
@@ -53,6 +53,7 @@ class _PoolStats(ctypes.Structure):
 _SIGS = {
     "pa_strerror": (ctypes.c_char_p, [_i]),
     "pa_version": (ctypes.c_char_p, []),
+    "pa_copy_async": (_i, [_vp, _vp, _sz, _vp]),
     "pa_write_kv": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "pa_copy_blocks": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "pa_rope_write_kv": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
@@ -119,18 +120,37 @@ def version() -> str:
     return lib.pa_version().decode()
 
 
+def copy_async(dst, src, stream=None) -> None:
+    """Copy the bytes of contiguous tensor src into dst (same byte size; host, pinned host or device memory on
+    either side) on `stream`, without waiting for it: one pa_copy_async call, no stream switch on the torch
+    side.  Pinned host memory is what makes a host-side copy asynchronous."""
+    n = src.numel() * src.element_size()
+    if dst.numel() * dst.element_size() != n:
+        raise ValueError(f"copy_async: {n} bytes into {dst.numel() * dst.element_size()}")
+    if not (src.is_contiguous() and dst.is_contiguous()):
+        raise ValueError("copy_async takes contiguous tensors")
+    _check(lib.pa_copy_async(ctypes.c_void_p(dst.data_ptr()), ctypes.c_void_p(src.data_ptr()), n,
+                             _stream_handle(stream)), "pa_copy_async")
+
+
 # ---------------------------------------------------------------------------------------------- device calls
+_TORCH = None
+
+
 def _torch():
-    import torch
-    return torch
+    global _TORCH
+    if _TORCH is None:
+        import torch
+        _TORCH = torch
+    return _TORCH
 
 
 def _dtype_code(t) -> int:
     torch = _torch()
-    if t.dtype == torch.float16:
-        return 0
     if t.dtype == torch.bfloat16:
         return 1
+    if t.dtype == torch.float16:
+        return 0
     raise ValueError(f"unsupported dtype {t.dtype}")
 
 
@@ -156,22 +176,22 @@ def _want(name, t, dtype=None, shape=None, ndim=None):
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if ndim is not None and t.dim() != ndim:
         raise ValueError(f"{name} must have {ndim} dimensions, got shape {tuple(t.shape)}")
-    if shape is not None and tuple(t.shape) != tuple(shape):
+    if shape is not None and t.shape != tuple(shape):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
 def _caches(k_cache, v_cache):
     """Both caches [num_blocks, block_size, Hkv, D], same shape and 16-bit dtype; returns the shape."""
-    _want("k_cache", k_cache, ndim=4)
-    _want("v_cache", v_cache, dtype=k_cache.dtype, shape=k_cache.shape)
+    ks = k_cache.shape
+    if len(ks) != 4 or v_cache.dtype != k_cache.dtype or v_cache.shape != ks:
+        _want("k_cache", k_cache, ndim=4)
+        _want("v_cache", v_cache, dtype=k_cache.dtype, shape=ks)
     _dtype_code(k_cache)
-    return tuple(int(x) for x in k_cache.shape)
+    return tuple(ks)
 
 
-def _device(stream, *tensors):
-    """Every tensor argument must live on the current CUDA device (a host pointer, or another device's memory,
-    must never reach a kernel), and a given stream must belong to that device.  Checked after the dtype and
-    shape checks, before anything is launched."""
+def _device_slow(stream, tensors):
+    """The precise error for a failed _device check."""
     torch = _torch()
     dev = None
     for t in tensors:
@@ -188,7 +208,27 @@ def _device(stream, *tensors):
             raise ValueError(f"tensors are on {dev} but the current device is cuda:{torch.cuda.current_device()}")
         if stream is not None and stream.device != dev:
             raise ValueError(f"stream belongs to {stream.device}, tensors to {dev}")
-    return dev
+    raise AssertionError("device check failed without a reason")
+
+
+def _device(stream, *tensors):
+    """Every tensor argument must live on the current CUDA device (a host pointer, or another device's memory,
+    must never reach a kernel), and a given stream must belong to that device.  Checked after the dtype and
+    shape checks, before anything is launched.  (Device indices as ints; the torch.device objects only to
+    word an error.)"""
+    idx = None
+    for t in tensors:
+        if t is None:
+            continue
+        d = t.get_device()  # -1 for host memory
+        if idx is None:
+            idx = d
+        elif d != idx:
+            _device_slow(stream, tensors)
+    if idx is None:
+        return
+    if idx < 0 or idx != _torch().cuda.current_device() or (stream is not None and stream.device_index != idx):
+        _device_slow(stream, tensors)
 
 
 def write_kv(k, v, slot_mapping, k_cache, v_cache, stream=None) -> None:
@@ -262,6 +302,13 @@ def _decode_args(q, k_cache, v_cache, block_tables, context_lens, out):
     """Shapes and dtypes of a decode call: q [B, Hq, D] in the caches' dtype, block_tables int32 [B, n],
     context_lens int32 [B], out (if given) like q.  Returns (B, Hq, D)."""
     torch = _torch()
+    ks, qs, dt = k_cache.shape, q.shape, k_cache.dtype
+    if (len(ks) == 4 and v_cache.shape == ks and v_cache.dtype == dt and len(qs) == 3 and q.dtype == dt
+            and qs[2] == ks[3] and block_tables.dtype == torch.int32 and block_tables.dim() == 2
+            and block_tables.shape[0] == qs[0] and context_lens.dtype == torch.int32
+            and context_lens.shape == (qs[0],) and (out is None or (out.dtype == dt and out.shape == qs))):
+        _dtype_code(k_cache)
+        return qs[0], qs[1], qs[2]
     _, _, _, D = _caches(k_cache, v_cache)
     _want("q", q, dtype=k_cache.dtype, ndim=3)
     B, Hq = int(q.shape[0]), int(q.shape[1])

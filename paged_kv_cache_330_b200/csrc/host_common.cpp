@@ -30,6 +30,13 @@ extern "C" const char* pa_strerror(int status) {
 
 extern "C" const char* pa_version(void) { return "0.1.0"; }
 
+extern "C" int pa_copy_async(void* dst, const void* src, size_t bytes, void* stream) {
+  if (bytes == 0) return PA_OK;
+  if (!dst || !src) return PA_ERR_INVALID;
+  return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDefault, (cudaStream_t)stream) == cudaSuccess ? PA_OK
+                                                                                               : PA_ERR_CUDA;
+}
+
 extern "C" int pa_device_error(int* out) {
   if (!out) return PA_ERR_INVALID;
   if (cudaDeviceSynchronize() != cudaSuccess) return PA_ERR_CUDA;

@@ -43,6 +43,13 @@ MISALIGNED = ctypes.c_void_p(0x10008)
 NULL = ctypes.c_void_p(0)
 
 
+def test_copy_async_host_checks():
+    """pa_copy_async: zero bytes is a no-op and NULL addresses are rejected, both before any CUDA call."""
+    assert pa.lib.pa_copy_async(None, None, 0, None) == pa.PA_OK
+    assert pa.lib.pa_copy_async(None, ctypes.c_void_p(16), 64, None) == -1
+    assert pa.lib.pa_copy_async(ctypes.c_void_p(16), None, 64, None) == -1
+
+
 def test_write_kv_validation():
     L = pa.lib
     # unsupported dtype / block size / negative sizes

@@ -186,3 +186,21 @@ def test_decode_workspace_reuse_across_calls():
         assert_close(out.float().cpu().numpy(), ref, f"reuse partitions={n}")
     torch.cuda.synchronize()
     assert int(ws[: wl.batch * 8 * 4].view(torch.int32).abs().sum().item()) == 0
+
+
+def test_copy_async_round_trip():
+    """pa_copy_async moves bytes host -> device -> device -> host on given streams, unchanged."""
+    import paged_kv_cache_330_b200 as pa
+    g = torch.Generator().manual_seed(5)
+    h = torch.randint(0, 256, ((1 << 20) + 48,), dtype=torch.uint8, generator=g).pin_memory()
+    d1 = torch.empty(h.numel(), dtype=torch.uint8, device="cuda")
+    d2 = torch.empty_like(d1)
+    back = torch.zeros(h.numel(), dtype=torch.uint8).pin_memory()
+    st = torch.cuda.Stream()
+    pa.copy_async(d1, h, stream=st)
+    pa.copy_async(d2, d1, stream=st)
+    pa.copy_async(back, d2, stream=st)
+    st.synchronize()
+    assert torch.equal(back, h)
+    with pytest.raises(ValueError):
+        pa.copy_async(d1[:10], h)
