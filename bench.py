@@ -63,15 +63,16 @@ WORKLOAD_TEXT = {
 DECODE_SRC = ("decode.cu", "common.cuh")
 PREFILL_SRC = ("prefill.cu", "common.cuh")
 ROPE_SRC = ("rope_write_kv.cu", "common.cuh")
+CASCADE_SRC = ("decode.cu", "prefill.cu", "common.cuh")  # suffix decode + prefill kernel in shared-prefix mode
 NCU_TRAFFIC = {
-    "qwen_decode": {"bytes": 313_008_640, "src": "4eb4742cfc8cb957", "files": DECODE_SRC},
-    "qwen_decode_int8": {"bytes": 165_265_408, "src": "4eb4742cfc8cb957", "files": DECODE_SRC},
-    "llama70b_long_int8": {"bytes": 843_906_048, "src": "4eb4742cfc8cb957", "files": DECODE_SRC},
+    "qwen_decode": {"bytes": 312_951_296, "src": "2a2553a6f98e281a", "files": DECODE_SRC},
+    "qwen_decode_int8": {"bytes": 164_487_680, "src": "2a2553a6f98e281a", "files": DECODE_SRC},
+    "llama70b_long_int8": {"bytes": 844_053_248, "src": "2a2553a6f98e281a", "files": DECODE_SRC},
     # both kernels of one cascade call at block size 16 (suffix decode + shared-prefix pass)
-    "prefix_sweep_cascade": {"bytes": 353_382_144, "src": "4eb4742cfc8cb957", "files": DECODE_SRC},
-    "llama70b_long": {"bytes": 1_584_901_888, "src": "84d9feaada7e0320", "files": DECODE_SRC},
-    "prefill": {"bytes": 348_481_024, "src": "0a0c45baf16bf168", "files": PREFILL_SRC},
-    "rope_write": {"bytes": 55_164_160, "src": "9b1a5d7fb8331db7", "files": ROPE_SRC},
+    "prefix_sweep_cascade": {"bytes": 351_853_824, "src": "3542be76217774c2", "files": CASCADE_SRC},
+    "llama70b_long": {"bytes": 1_584_877_312, "src": "2a2553a6f98e281a", "files": DECODE_SRC},
+    "prefill": {"bytes": 347_661_312, "src": "2cbc89d535bde70d", "files": PREFILL_SRC},
+    "rope_write": {"bytes": 55_998_208, "src": "e527154b96c52f4d", "files": ROPE_SRC},
 }
 
 

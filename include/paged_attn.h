@@ -228,7 +228,11 @@ int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int
 /* zero-filled before first use; every completed call leaves its counters   */
 /* at zero.  Two launches on `stream`; same argument checks and return      */
 /* codes as pa_decode.  A prefix length that is not a multiple of 16 is     */
-/* rounded down and sets PA_ERRBIT_INDEX.                                   */
+/* rounded down and sets PA_ERRBIT_INDEX.  At head_dim 128 step 2 is a      */
+/* programmatic dependent launch: its CTAs may start in step 1's tail     */
+/* (step 1 lets it launch only after the kernel before step 1 completed)   */
+/* and read q, the tables and the prefix rows then; they wait for step 1   */
+/* to complete before reading or writing out (no caller action needed).    */
 /* ------------------------------------------------------------------------ */
 size_t pa_decode_cascade_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
                                         int max_context_len, int num_partitions_or_0, int num_groups,

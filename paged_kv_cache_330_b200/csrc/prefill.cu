@@ -750,6 +750,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // prefix's softmax and the member's suffix result are weighted by their log-sum-exps, the prefix's
       // being m_ref + log2(l) in the log2 domain and the suffix's lse_s (natural log; -inf when empty)
       float wp = 1.f / lsum, ws = 0.f;
+      // shared-prefix mode is launched while the suffix decode may still run: its (out, lse) are read only
+      // after that grid has completed (everything before reads inputs and older cache rows only)
+      if (p.prefix_mode) asm volatile("griddepcontrol.wait;" ::: "memory");
       if (p.prefix_mode && row < C) {
         const float mp = m_ref + __log2f(lsum);
         const float ms = __ldg(p.lse_s + (size_t)(q0 + row) * p.num_q_heads + head) * kLog2e;
@@ -824,6 +827,8 @@ int launch_pairs(PrefillParams& p, const void* k_cache, const void* v_cache, int
       return PA_ERR_CUDA;
     if (dev >= 0 && dev < 64) attr_set[di][dev].store(true, std::memory_order_release);
   }
+  if (p.prefix_mode)  // programmatic: its CTAs may take the SMs the suffix decode frees in its tail
+    return pa::launch_programmatic(kern, dim3((unsigned)grid), dim3(kThreads), SMEM_ALLOC, st, km, vm, p);
   kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(km, vm, p);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
