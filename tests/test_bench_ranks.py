@@ -111,3 +111,28 @@ def test_reference_arm_times_the_matching_oracle(monkeypatch, capsys, workload, 
     assert line["impl"] == "reference" and line["metric"] == getattr(bench, metric_attr) and line["unit"] == unit
     assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["unit"] == unit
     assert line["e2e"] == {"value": line["value"], "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_staged_inputs_pack_and_views(monkeypatch):
+    """The end-to-end loop's staging buffer: every input at a 256-byte offset of one buffer, one copy of
+    `nbytes` moves all of them, and the typed device views read back each input unchanged (CPU stand-in for
+    pinned and device memory)."""
+    bench = _load_bench()
+    monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)
+    g = torch.Generator().manual_seed(11)
+    host = dict(q=torch.randn(3, 4, 128, generator=g).to(torch.bfloat16), sm=torch.arange(5, dtype=torch.int64),
+                bt=torch.randint(0, 9, (3, 7), dtype=torch.int32, generator=g), empty=torch.zeros(0, dtype=torch.int32),
+                lens=torch.tensor([1, 2, 3], dtype=torch.int32))
+    st = bench.StagedInputs(host, "cpu")
+    ends = []
+    for name, t in host.items():
+        v = st.views[1][name]
+        assert v.dtype == t.dtype and v.shape == t.shape
+        if t.numel():
+            off = v.data_ptr() - st.d[1].data_ptr()
+            assert off % 256 == 0
+            ends.append(off + t.numel() * t.element_size())
+    assert st.nbytes == max(ends)
+    st.d[1][:st.nbytes].copy_(st.h[:st.nbytes])
+    for name, t in host.items():
+        assert torch.equal(st.views[1][name], t), name
