@@ -69,9 +69,9 @@ NCU_TRAFFIC = {
     "qwen_decode_int8": {"bytes": 164_487_680, "src": "2a2553a6f98e281a", "files": DECODE_SRC},
     "llama70b_long_int8": {"bytes": 844_053_248, "src": "2a2553a6f98e281a", "files": DECODE_SRC},
     # both kernels of one cascade call at block size 16 (suffix decode + shared-prefix pass)
-    "prefix_sweep_cascade": {"bytes": 351_852_800, "src": "a7ed74521176f7ed", "files": CASCADE_SRC},
+    "prefix_sweep_cascade": {"bytes": 352_267_520, "src": "caed4f9e43241e80", "files": CASCADE_SRC},
     "llama70b_long": {"bytes": 1_584_877_312, "src": "2a2553a6f98e281a", "files": DECODE_SRC},
-    "prefill": {"bytes": 347_392_256, "src": "07dd29c96fd2fe65", "files": PREFILL_SRC},
+    "prefill": {"bytes": 347_595_264, "src": "06a1cc1b4135c2f1", "files": PREFILL_SRC},
     "rope_write": {"bytes": 55_998_208, "src": "e527154b96c52f4d", "files": ROPE_SRC},
 }
 

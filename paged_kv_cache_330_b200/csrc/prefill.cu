@@ -62,6 +62,34 @@
 #include "host_common.h"
 
 PA_DEFINE_ERROR_WORD(pa__err_prefill)
+namespace {
+// Bounded wait that polls with test_wait (never suspends the warp), for a wait on the critical path whose
+// phase completes within a few hundred nanoseconds: the PV issuer's wait for P.  Measured: +1 % for the
+// kernel; the same for every wait of both issuers; -2 % when the eight softmax warps also spin.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(pa::smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_spin_warp(uint64_t* bar, uint32_t parity) {
+  bool done = mbar_test(bar, parity);
+  if (!done) {
+    const uint64_t start = pa::global_ns();
+    for (;;) {
+      for (int k = 0; k < 256 && !done; ++k) done = mbar_test(bar, parity);
+      if (done || pa::global_ns() - start > PA_WAIT_LIMIT_NS) break;
+    }
+  }
+  return __all_sync(0xffffffffu, done) != 0;
+}
+}  // namespace
+
 
 namespace {
 
@@ -542,7 +570,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       } else {
         for (int i = 0; i < nkv && ok; ++i) {
           const int st = i % VS, buf = i & 1;
-          if (!mbar_wait_warp(&v_full[st], (i / VS) & 1) || !mbar_wait_warp(&p_full[buf], (i >> 1) & 1)) {
+          if (!mbar_wait_warp(&v_full[st], (i / VS) & 1) || !mbar_spin_warp(&p_full[buf], (i >> 1) & 1)) {
             ok = false;
             break;
           }
