@@ -204,3 +204,23 @@ def test_copy_async_round_trip():
     assert torch.equal(back, h)
     with pytest.raises(ValueError):
         pa.copy_async(d1[:10], h)
+
+
+# Batches above 256 sequences: the producer's range lookups then scan the lengths in memory, 256 per pass,
+# instead of the register-held lengths of smaller batches.  Ragged lengths with empty sequences spread over
+# every 256-sequence pass, at several cuts of the chunk line.
+@pytest.mark.parametrize("B", [257, 600])
+@pytest.mark.parametrize("Hq,Hkv", [(8, 4), (16, 2)])
+def test_decode_batches_over_256(B, Hq, Hkv):
+    rng = np.random.default_rng(B + Hq)
+    lens = rng.integers(0, 300, B)
+    lens[::97] = 0
+    lens[1::131] = 1
+    wl = make_custom(seed=B * 7 + Hq, lens=lens.tolist(), num_q_heads=Hq, num_kv_heads=Hkv, head_dim=128,
+                     block_size=16, dtype="bf16")
+    ref = _oracle_decode(wl)
+    for ns in (0, 7, 1000):
+        out, *_ = gpu_step(wl, num_partitions=ns)
+        got = out.float().cpu().numpy()
+        assert_close(got, ref, f"B{B} G{Hq // Hkv} partitions{ns}")
+        assert (got[lens == 0] == 0).all()

@@ -206,3 +206,19 @@ def test_decode_int8_zero_value_rows():
     ref, _ = _oracle_decode_int8(wl)
     assert (out.float().cpu() == 0).all()
     assert_close(out.float().cpu().numpy(), ref, "int8 zero rows")
+
+
+@pytest.mark.parametrize("B", [257, 600])
+def test_decode_int8_batches_over_256(B):
+    """Above 256 sequences the producer's lookups scan the lengths in memory (see the 16-bit case)."""
+    rng = np.random.default_rng(B)
+    lens = rng.integers(0, 300, B)
+    lens[::89] = 0
+    wl = make_custom(seed=B * 11, lens=lens.tolist(), num_q_heads=16, num_kv_heads=2, head_dim=128, block_size=16,
+                     dtype="bf16")
+    ref, _ = _oracle_decode_int8(wl)
+    for ns in (0, 7):
+        out = gpu_step_int8(wl, num_partitions=ns)[0]
+        got = out.float().cpu().numpy()
+        assert_close(got, ref, f"int8 B{B} partitions{ns}")
+        assert (got[lens == 0] == 0).all()
