@@ -65,12 +65,12 @@ PREFILL_SRC = ("prefill.cu", "common.cuh")
 ROPE_SRC = ("rope_write_kv.cu", "common.cuh")
 CASCADE_SRC = ("decode.cu", "prefill.cu", "common.cuh")  # suffix decode + prefill kernel in shared-prefix mode
 NCU_TRAFFIC = {
-    "qwen_decode": {"bytes": 312_951_296, "src": "2a2553a6f98e281a", "files": DECODE_SRC},
-    "qwen_decode_int8": {"bytes": 164_487_680, "src": "2a2553a6f98e281a", "files": DECODE_SRC},
-    "llama70b_long_int8": {"bytes": 844_053_248, "src": "2a2553a6f98e281a", "files": DECODE_SRC},
+    "qwen_decode": {"bytes": 313_386_240, "src": "f18f3a27d6c38f97", "files": DECODE_SRC},
+    "qwen_decode_int8": {"bytes": 164_545_024, "src": "f18f3a27d6c38f97", "files": DECODE_SRC},
+    "llama70b_long_int8": {"bytes": 843_744_768, "src": "f18f3a27d6c38f97", "files": DECODE_SRC},
     # both kernels of one cascade call at block size 16 (suffix decode + shared-prefix pass)
-    "prefix_sweep_cascade": {"bytes": 352_267_520, "src": "caed4f9e43241e80", "files": CASCADE_SRC},
-    "llama70b_long": {"bytes": 1_584_877_312, "src": "2a2553a6f98e281a", "files": DECODE_SRC},
+    "prefix_sweep_cascade": {"bytes": 352_109_312, "src": "4115bd3bedbbc994", "files": CASCADE_SRC},
+    "llama70b_long": {"bytes": 1_584_700_160, "src": "f18f3a27d6c38f97", "files": DECODE_SRC},
     "prefill": {"bytes": 347_595_264, "src": "06a1cc1b4135c2f1", "files": PREFILL_SRC},
     "rope_write": {"bytes": 55_998_208, "src": "e527154b96c52f4d", "files": ROPE_SRC},
 }

@@ -544,6 +544,7 @@ struct Q8Consumer {
   float o[NT][KS][4];                     // O^T relative to (m, rho): rows d (permuted), columns heads
   float m[NT][2], l[NT][2];               // heads 8nt + 2(lane%4) + {0,1}; l is this lane's partial sum
   float rho[NT][2];                       // running max of (s - m) + log2(scale_v) per head
+  float qbias[NT][2];                     // -1152 * sum over d of the fp16 q^T of heads 8nt + 2(lane%4) + {0,1}
   float qs;                               // scale * log2(e) / prescale
 
   static __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -551,12 +552,13 @@ struct Q8Consumer {
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
     return d;
   }
-  // fp16x2 of bytes 0,1 (lo) or 2,3 (hi) of a word of codes already XORed with 0x80808080
-  static __device__ __forceinline__ uint32_t to_h2(uint32_t xb, uint32_t sel) {
-    uint32_t h = prmt(xb, 0x64646464u, sel), d;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(h), "r"(0x64806480u));
-    return d;
-  }
+  // fp16x2 of bytes 0,1 (lo) or 2,3 (hi) of a word of codes already XORed with 0x80808080: the byte lands in
+  // the low mantissa bits under the exponent of 1024, so each half is exactly 1152 + code (codes -128 .. 127
+  // give 1024 .. 1279, integers fp16 holds exactly).  The 1152 is taken out in fp32 instead of here: for K it
+  // starts the score accumulators (qbias), for V one product of the tile's P with a constant -1152 operand
+  // comes off O in the rescale (a per-head term, the same for every row d).
+  static constexpr uint32_t kNegBias = 0xE480E480u;  // fp16x2 (-1152, -1152)
+  static __device__ __forceinline__ uint32_t to_h2(uint32_t xb, uint32_t sel) { return prmt(xb, 0x64646464u, sel); }
   static __device__ __forceinline__ void mma_f16(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                  uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -622,6 +624,12 @@ struct Q8Consumer {
         qb[nt][ks][0] = b0;
         qb[nt][ks][1] = b1;
       }
+      // -1152 * sum_d q^T[d][h] in fp32, in the layout of the score accumulators (rows tokens, columns heads)
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) mma_f16(acc, kNegBias, kNegBias, kNegBias, kNegBias, qb[nt][ks][0], qb[nt][ks][1]);
+      qbias[nt][0] = acc[0];
+      qbias[nt][1] = acc[1];
     }
   }
 
@@ -635,7 +643,10 @@ struct Q8Consumer {
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) s[mt][nt][0] = s[mt][nt][1] = s[mt][nt][2] = s[mt][nt][3] = 0.f;
+      for (int nt = 0; nt < NT; ++nt) {
+        s[mt][nt][0] = s[mt][nt][2] = qbias[nt][0];  // the codes enter as 1152 + code: start at -1152 * sum q
+        s[mt][nt][1] = s[mt][nt][3] = qbias[nt][1];
+      }
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt) {
       const int ta = r0 + 16 * mt + g, tb = ta + 8;
@@ -712,14 +723,19 @@ struct Q8Consumer {
         l[nt][e] = l[nt][e] * alpha + ls;
       }
 #pragma unroll
-      for (int i = 0; i < KS; ++i) {
-        o[nt][i][0] *= beta[0]; o[nt][i][2] *= beta[0];
-        o[nt][i][1] *= beta[1]; o[nt][i][3] *= beta[1];
-      }
-#pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
         pb[nt][mt][0] = trans8x8(pack_h2(s[mt][nt][0], s[mt][nt][1]));  // tokens 2c, 2c+1 of head g
         pb[nt][mt][1] = trans8x8(pack_h2(s[mt][nt][2], s[mt][nt][3]));  // tokens 2c+8, 2c+9
+      }
+      // -1152 * (sum of the tile's fp16 P' per head), laid out as O^T (every row d the same): the V codes
+      // below enter as 1152 + code, so this comes off O as it is rescaled
+      float pv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks) mma_f16(pv, kNegBias, kNegBias, kNegBias, kNegBias, pb[nt][ks][0], pb[nt][ks][1]);
+#pragma unroll
+      for (int i = 0; i < KS; ++i) {
+        o[nt][i][0] = fmaf(o[nt][i][0], beta[0], pv[0]); o[nt][i][2] = fmaf(o[nt][i][2], beta[0], pv[2]);
+        o[nt][i][1] = fmaf(o[nt][i][1], beta[1], pv[1]); o[nt][i][3] = fmaf(o[nt][i][3], beta[1], pv[3]);
       }
     }
     // ---- O^T += V^T P'^T: k-steps of 16 tokens; m-tiles (j, sub) hold d = 4g + 32j + 2sub + {0 (row g), 1 (row g+8)}
