@@ -208,6 +208,25 @@ def test_decode_int8_zero_value_rows():
     assert_close(out.float().cpu().numpy(), ref, "int8 zero rows")
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_decode_int8_offset_cancellation(D):
+    """The codes enter the fp16 products as 1152 + code and the offset is taken out in fp32: 1152 * sum(q)
+    per score, 1152 * sum(P') per output.  Stress both subtractions: q with a common component 50x its spread
+    (sum(q) large against sum(q * code)), small K rows so the attention spreads evenly over thousands of
+    tokens (the V offset accumulates over every tile of a piece), zero-mean V, ragged lengths."""
+    wl = make_custom(seed=31, lens=[8192, 5000, 1, 33, 2048], num_q_heads=16, num_kv_heads=2, head_dim=D,
+                     block_size=16)
+    g = torch.Generator().manual_seed(7)
+    wl.q = (4.0 + 0.08 * torch.randn(tuple(wl.q.shape), generator=g)).to(wl.q.dtype)
+    for name in ("k_cache0", "k_new"):
+        t = getattr(wl, name)
+        setattr(wl, name, (t.float() * 0.05).to(t.dtype))
+    ref, _ = _oracle_decode_int8(wl)
+    for ns in (0, 64):
+        out = gpu_step_int8(wl, num_partitions=ns)[0]
+        assert_close(out.float().cpu().numpy(), ref, f"int8 offset cancellation D{D} partitions{ns}")
+
+
 @pytest.mark.parametrize("B", [257, 600])
 def test_decode_int8_batches_over_256(B):
     """Above 256 sequences the producer's lookups scan the lengths in memory (see the 16-bit case)."""
