@@ -660,15 +660,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       {
-        uint32_t raw[32];
-        tmem_ld32(sbuf, raw);
+        // both column halves in flight before the one wait (it covers every earlier load of the thread)
+        uint32_t raw0[32], raw1[32];
+        tmem_ld32(sbuf, raw0);
+        tmem_ld32(sbuf + 32, raw1);
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(raw[c]);
-        tmem_ld32(sbuf + 32, raw);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) s[32 + c] = __uint_as_float(raw[c]);
+        for (int c = 0; c < 32; ++c) {
+          s[c] = __uint_as_float(raw0[c]);
+          s[32 + c] = __uint_as_float(raw1[c]);
+        }
       }
       const int lim = last_key - (j * BN + hf * 64);  // last visible column of this half-tile
       const bool diag = lim < 63;
