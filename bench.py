@@ -65,12 +65,12 @@ PREFILL_SRC = ("prefill.cu", "common.cuh")
 ROPE_SRC = ("rope_write_kv.cu", "common.cuh")
 CASCADE_SRC = ("decode.cu", "prefill.cu", "common.cuh")  # suffix decode + prefill kernel in shared-prefix mode
 NCU_TRAFFIC = {
-    "qwen_decode": {"bytes": 313_386_240, "src": "f18f3a27d6c38f97", "files": DECODE_SRC},
-    "qwen_decode_int8": {"bytes": 164_545_024, "src": "f18f3a27d6c38f97", "files": DECODE_SRC},
-    "llama70b_long_int8": {"bytes": 843_744_768, "src": "f18f3a27d6c38f97", "files": DECODE_SRC},
+    "qwen_decode": {"bytes": 313_004_032, "src": "95dca1d0ca960523", "files": DECODE_SRC},
+    "qwen_decode_int8": {"bytes": 164_869_376, "src": "95dca1d0ca960523", "files": DECODE_SRC},
+    "llama70b_long_int8": {"bytes": 844_040_448, "src": "95dca1d0ca960523", "files": DECODE_SRC},
     # both kernels of one cascade call at block size 16 (suffix decode + shared-prefix pass)
-    "prefix_sweep_cascade": {"bytes": 352_588_800, "src": "1a32c912c13e5174", "files": CASCADE_SRC},
-    "llama70b_long": {"bytes": 1_584_700_160, "src": "f18f3a27d6c38f97", "files": DECODE_SRC},
+    "prefix_sweep_cascade": {"bytes": 351_881_984, "src": "f86ad8eda4abdac4", "files": CASCADE_SRC},
+    "llama70b_long": {"bytes": 1_584_821_760, "src": "95dca1d0ca960523", "files": DECODE_SRC},
     "prefill": {"bytes": 347_949_824, "src": "168c732c524f5c1a", "files": PREFILL_SRC},
     "rope_write": {"bytes": 55_998_208, "src": "e527154b96c52f4d", "files": ROPE_SRC},
 }

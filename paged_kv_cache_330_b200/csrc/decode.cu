@@ -540,6 +540,7 @@ struct Q8Consumer {
   static constexpr int NT = (G + 7) / 8;  // n-tiles of 8 heads
   static constexpr int KS = D / 16;       // k-steps of QK^T, and m-tiles (16 rows of d) of O^T
   static constexpr int QB = D / 4;        // bytes of a K row one lane reads (its quarter of the row)
+  static constexpr bool kPieceV = G <= 4;  // V codes read as one piece per row (see tile)
   uint32_t qb[NT][KS][2];                 // B fragments of q^T (fp16, prescaled)
   float o[NT][KS][4];                     // O^T relative to (m, rho): rows d (permuted), columns heads
   float m[NT][2], l[NT][2];               // heads 8nt + 2(lane%4) + {0,1}; l is this lane's partial sum
@@ -738,28 +739,52 @@ struct Q8Consumer {
         o[nt][i][1] = fmaf(o[nt][i][1], beta[1], pv[1]); o[nt][i][3] = fmaf(o[nt][i][3], beta[1], pv[3]);
       }
     }
-    // ---- O^T += V^T P'^T: k-steps of 16 tokens; m-tiles (j, sub) hold d = 4g + 32j + 2sub + {0 (row g), 1 (row g+8)}
+    // ---- O^T += V^T P'^T, k-steps of 16 tokens.  Rows t0, t0+1, t0+8, t0+9 (t0 = 16ks + 2c) give the
+    // A operands of two m-tiles per 4-byte word (bytes d .. d+3 of each row): m-tile i0 holds d (row g) and
+    // d+1 (row g+8), m-tile i0+1 holds d+2 and d+3.  Two load forms, chosen per group size by measurement
+    // (same box, alternated): one 16-byte (D 64: 8-byte) load per row piece, d = VB*g + 4w, is faster at
+    // G 2 (Qwen batch 46.6 -> 45.4 us, a long-context G 2 batch 156.9 -> 154.9 us) and slower at G 8 (Llama
+    // batch 194.7 -> 197.2 us, a short-context G 8 batch 83.1 -> 84.0 us) than 4-byte loads, d = 4g + 32j;
+    // stash() undoes the m-tile order of the form in use
+    auto pv_word = [&](int ks, int i0, uint32_t wa, uint32_t wb, uint32_t wc, uint32_t wd) {
+      const uint32_t xab = prmt(wa, wb, 0x5140u) ^ 0x80808080u, yab = prmt(wa, wb, 0x7362u) ^ 0x80808080u;
+      const uint32_t xcd = prmt(wc, wd, 0x5140u) ^ 0x80808080u, ycd = prmt(wc, wd, 0x7362u) ^ 0x80808080u;
+      const uint32_t a00 = to_h2(xab, 0x4140u), a01 = to_h2(xab, 0x4342u);
+      const uint32_t a02 = to_h2(xcd, 0x4140u), a03 = to_h2(xcd, 0x4342u);
+      const uint32_t a10 = to_h2(yab, 0x4140u), a11 = to_h2(yab, 0x4342u);
+      const uint32_t a12 = to_h2(ycd, 0x4140u), a13 = to_h2(ycd, 0x4342u);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        mma_f16(o[nt][i0], a00, a01, a02, a03, pb[nt][ks][0], pb[nt][ks][1]);
+        mma_f16(o[nt][i0 + 1], a10, a11, a12, a13, pb[nt][ks][0], pb[nt][ks][1]);
+      }
+    };
 #pragma unroll
     for (int ks = 0; ks < 2; ++ks) {
       if (ks * 16 >= nv) break;
       const int t0 = r0 + 16 * ks + 2 * c;
+      if constexpr (kPieceV) {
+        constexpr int VB = LY::ROWB / 8, VW = VB / 4;  // bytes and words of a lane's piece of a row
+        uint32_t wv[4][VW];                            // rows t0, t0 + 1, t0 + 8, t0 + 9
 #pragma unroll
-      for (int j = 0; j < D / 32; ++j) {
-        const int byte = 4 * g + 32 * j;
-        const uint32_t wa = lds32(swz8_addr<LY::ROWB>(vbase, t0, byte));
-        const uint32_t wb = lds32(swz8_addr<LY::ROWB>(vbase, t0 + 1, byte));
-        const uint32_t wc = lds32(swz8_addr<LY::ROWB>(vbase, t0 + 8, byte));
-        const uint32_t wd = lds32(swz8_addr<LY::ROWB>(vbase, t0 + 9, byte));
-        const uint32_t xab = prmt(wa, wb, 0x5140u) ^ 0x80808080u, yab = prmt(wa, wb, 0x7362u) ^ 0x80808080u;
-        const uint32_t xcd = prmt(wc, wd, 0x5140u) ^ 0x80808080u, ycd = prmt(wc, wd, 0x7362u) ^ 0x80808080u;
-        const uint32_t a00 = to_h2(xab, 0x4140u), a01 = to_h2(xab, 0x4342u);
-        const uint32_t a02 = to_h2(xcd, 0x4140u), a03 = to_h2(xcd, 0x4342u);
-        const uint32_t a10 = to_h2(yab, 0x4140u), a11 = to_h2(yab, 0x4342u);
-        const uint32_t a12 = to_h2(ycd, 0x4140u), a13 = to_h2(ycd, 0x4342u);
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t a = swz8_addr<LY::ROWB>(vbase, t0 + (q & 1) + 8 * (q >> 1), VB * g);
+          if constexpr (VW == 4) {
+            const uint4 u = lds128(a);
+            wv[q][0] = u.x; wv[q][1] = u.y; wv[q][2] = u.z; wv[q][3] = u.w;
+          } else {
+            const uint2 u = lds64(a);
+            wv[q][0] = u.x; wv[q][1] = u.y;
+          }
+        }
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          mma_f16(o[nt][2 * j], a00, a01, a02, a03, pb[nt][ks][0], pb[nt][ks][1]);
-          mma_f16(o[nt][2 * j + 1], a10, a11, a12, a13, pb[nt][ks][0], pb[nt][ks][1]);
+        for (int w = 0; w < VW; ++w) pv_word(ks, 2 * w, wv[0][w], wv[1][w], wv[2][w], wv[3][w]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) {
+          const int byte = 4 * g + 32 * j;
+          pv_word(ks, 2 * j, lds32(swz8_addr<LY::ROWB>(vbase, t0, byte)), lds32(swz8_addr<LY::ROWB>(vbase, t0 + 1, byte)),
+                  lds32(swz8_addr<LY::ROWB>(vbase, t0 + 8, byte)), lds32(swz8_addr<LY::ROWB>(vbase, t0 + 9, byte)));
         }
       }
     }
@@ -786,7 +811,8 @@ struct Q8Consumer {
       }
 #pragma unroll
       for (int i = 0; i < KS; ++i) {
-        const int d = 4 * g + 32 * (i >> 1) + 2 * (i & 1);
+        const int d = kPieceV ? (LY::ROWB / 8) * g + 4 * (i >> 1) + 2 * (i & 1)  // the m-tile order of the PV
+                              : 4 * g + 32 * (i >> 1) + 2 * (i & 1);           // products (see tile)
         const int h0 = nt * 8 + 2 * c;
         if (h0 < G) {
           merge_o[h0 * D + d] = o[nt][i][0] * rel[0];
